@@ -1,0 +1,161 @@
+/*
+ * pa.h -- C ABI of libpa.so: attention over a paged KV cache on NVIDIA B200 (sm_100a).
+ *
+ * The KV cache of one attention layer is a pool of fixed-size physical blocks
+ * of 16 or 32 tokens.  Each sequence has a block table that maps its logical
+ * token positions to physical block IDs; blocks are taken as a sequence grows
+ * and may be shared by several sequences ("vLLM serving internals", AI
+ * Engineering from Scratch, Phase 17 / 04, section "PagedAttention as a
+ * virtual memory system"; "Inference optimization", Phase 10 / 12, section
+ * "Paged attention").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor pointer is CUDA device memory owned by the caller.  The
+ *    library never allocates, frees or synchronises; each call enqueues its
+ *    kernels on `stream` (a cudaStream_t, NULL = the legacy default stream)
+ *    and returns.  Calls are stateless and thread-safe.
+ *  - Layouts (row-major, no padding):
+ *      q, out        bf16  [num_q_tokens, num_q_heads, head_dim]
+ *      k_new, v_new  bf16  [num_tokens, num_kv_heads, head_dim]
+ *      k_cache,
+ *      v_cache       bf16  [num_blocks, num_kv_heads, block_size, head_dim]
+ *      block_tables  int32 [num_seqs, max_blocks_per_seq]   (unused entries: any value, e.g. -1)
+ *      context_lens  int32 [num_seqs]   tokens of each sequence INCLUDING this step's new ones
+ *      query_start   int32 [num_seqs + 1]  query rows of sequence s are query_start[s] .. query_start[s+1]-1
+ *      slot_mapping  int32 [num_tokens]    slot = block_id * block_size + offset; negative = padding
+ *  - Supported shapes: head_dim in {64, 128, 256}; block_size in {16, 32};
+ *    num_q_heads a multiple of num_kv_heads with group = num_q_heads /
+ *    num_kv_heads <= 16 (<= 8 when head_dim = 256).  Query head h reads KV head
+ *    h / group.  Pointers must be 16-byte aligned.
+ *  - Errors the host can see (null pointer, bad shape, workspace too small)
+ *    are returned before anything is launched.  A launch failure returns
+ *    PA_ERR_CUDA.  Data-dependent faults (a block ID outside [0, num_blocks),
+ *    a context longer than the block table, a slot outside the pool, a wait
+ *    that gave up) are detected on the device: if `dev_status` is non-NULL
+ *    the kernel ORs the matching PA_ERR_* magnitude bit (see PA_STATUS_BIT)
+ *    into *dev_status and the offending access is skipped or reads zeros.
+ *    Nothing traps.
+ *  - Attention uses bf16 inputs, fp32 accumulation and a bf16 output rounded
+ *    to nearest even.  A row whose context is empty produces zeros.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_NULL = -1,        /* a required pointer is NULL */
+  PA_ERR_SHAPE = -2,       /* inconsistent or negative sizes */
+  PA_ERR_UNSUPPORTED = -3, /* head_dim / block_size / group outside the supported set */
+  PA_ERR_WORKSPACE = -4,   /* workspace smaller than pa_workspace_bytes() */
+  PA_ERR_RANGE = -5,       /* device: block ID, slot or context outside its table or pool */
+  PA_ERR_CUDA = -6,        /* a CUDA runtime or driver call failed */
+  PA_ERR_TIMEOUT = -7      /* device: a bounded wait gave up */
+} pa_status;
+
+/* Bit that a kernel ORs into *dev_status for device-detected error `code`. */
+#define PA_STATUS_BIT(code) (1 << (-(code)))
+
+/*
+ * pa_cache_append -- write this step's new K/V rows into their cache slots.
+ *
+ * Defined by "Inference optimization", section "Build it -- Step 1: a KV
+ * cache from scratch" (the new keys and values of a step are stored at the
+ * sequence's current length before attention reads the cache), in the paged
+ * form of "vLLM serving internals", "PagedAttention as a virtual memory
+ * system" (the position lands in the block the table gives).
+ *
+ * For every token t with slot_mapping[t] >= 0 and every KV head h:
+ *   k_cache[slot / block_size, h, slot % block_size, :] = k_new[t, h, :]   (and v likewise)
+ * A bit-exact copy.  Negative slots are skipped.  A slot >= num_blocks *
+ * block_size is skipped and reported through dev_status.  Two tokens mapped
+ * to the same slot race (the caller's allocator never does that).
+ */
+PA_API int pa_cache_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                    const int32_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                    int head_dim, int block_size, int* dev_status, void* stream);
+
+/*
+ * pa_workspace_bytes -- bytes of device workspace pa_decode / pa_prefill_chunk
+ * need for a batch with at most `num_query_tokens` query rows, on the CURRENT
+ * device (the figure depends on its SM count).  Returns 0 for invalid sizes.
+ *
+ * Workspace contract: the caller allocates it, ZERO-FILLS it once before its
+ * first use, and may then reuse it for any later call on the same stream;
+ * every call that returns PA_OK and whose dev_status stays clear leaves it
+ * zero-filled again.  Calls that overlap in time must use different
+ * workspaces.  After a call that reported a device error, zero it again.
+ */
+PA_API size_t pa_workspace_bytes(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim);
+
+/*
+ * pa_decode -- one decode step: each sequence has exactly one query row (the
+ * newest token, position context_lens[s] - 1) that attends to all of its
+ * cached keys 0 .. context_lens[s] - 1.
+ *
+ * Defined by "Inference optimization", section "KV cache" (token N computes
+ * its own K, V and reads those of tokens 1..N-1 from the cache) and section
+ * "Build it -- Step 2: attention with the KV cache" (softmax of the scaled
+ * scores with the maximum subtracted, normalised, times V); the keys are
+ * gathered through the block table ("PagedAttention as a virtual memory
+ * system").  GQA: query head h uses KV head h / (num_q_heads / num_kv_heads)
+ * ("Inference optimization", exercise on grouped-query attention).
+ *
+ *   out[s, h, :] = sum_j softmax_j(scale * q[s, h, :] . K_j) V_j,  j < context_lens[s]
+ *
+ * q / out have num_seqs rows.  `scale` is usually 1/sqrt(head_dim).  Call
+ * pa_cache_append first if this step's rows must be visible.
+ */
+PA_API int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+              const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+              int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+              int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
+              void* stream);
+
+/*
+ * pa_prefill_chunk -- attention for a varlen batch that mixes prefill chunks
+ * and decodes in one call.  Sequence s contributes qlen = query_start[s+1] -
+ * query_start[s] query rows: the LAST qlen positions of its context_lens[s]
+ * tokens (a chunk of a long prompt, or qlen = 1 for a decode).  Row i of
+ * sequence s sits at position p = context_lens[s] - qlen + i and attends
+ * causally to keys 0 .. p.
+ *
+ * Defined by "vLLM serving internals", section "Chunked prefill protects the
+ * TTFT tail" (a long prompt is processed in ~512-token chunks interleaved with
+ * decodes) and section "What the scheduler looks like" (prefill chunks and
+ * single decode tokens form one batch and one fused GPU call); the causal mask
+ * of a query block that ends at the last key is the one of "Inference
+ * optimization", "Build it -- Step 2" (row i sees keys j <= i + Lk - Lq).
+ *
+ * q / out have total_q_tokens = query_start[num_seqs] rows.  Rows of
+ * sequences with qlen > 1 run on the tcgen05 tensor-core path; rows with
+ * qlen = 1 run on the decode path, concurrently.  A row with no key (p < 0)
+ * produces zeros.
+ */
+PA_API int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const void* k_cache,
+                     const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                     const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                     void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/* Human-readable name of a pa_status value (static storage). */
+PA_API const char* pa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -45,7 +45,8 @@ PINS = {
         "test_dominant_key_selects_its_v_row", "test_gqa_equals_repeated_mha",
         "test_causal_chunk_from_zero_equals_textbook_sdpa", "test_chunk_split_invariance",
         "test_decode_row_equals_prefill_row", "test_shared_prefix_equals_private_copy",
-        "test_empty_context_gives_zeros", "test_mutations_are_caught",
+        "test_empty_context_gives_zeros", "test_sampled_rows_equal_full_rows",
+        "test_mutations_are_caught",
     ],
     "cache_append": ["test_append_is_a_byte_copy", "test_append_then_attend_reads_new_row"],
     "slot_mapping": ["test_slot_mapping_closed_form", "test_allocator_slots_match_oracle"],

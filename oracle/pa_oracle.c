@@ -149,11 +149,13 @@ int oracle_cache_append(const uint16_t *k_new, const uint16_t *v_new, uint16_t *
  * One output row [SDPA] over keys 0..last_key of sequence s, for query head h
  * which reads KV head kvh.  scores[j] = scale * sum_d q[d] * K_j[d]; m = max_j
  * scores[j]; w_j = exp(scores[j] - m); out = sum_j w_j V_j / sum_j w_j.
+ * The sum is built in `acc` (head_dim doubles) and only then stored, so two
+ * calls for the same row write the same values.
  */
 static int attend_one(double *out, const uint16_t *q_row, const uint16_t *k_cache,
                       const uint16_t *v_cache, const int32_t *block_tables, int max_blocks,
                       int s, int last_key, int kvh, int num_kv_heads, int head_dim,
-                      int block_size, int num_blocks, double scale, double *scores)
+                      int block_size, int num_blocks, double scale, double *scores, double *acc)
 {
 #if ORACLE_MUTATION == 1
     int nkeys = last_key;
@@ -164,9 +166,11 @@ static int attend_one(double *out, const uint16_t *q_row, const uint16_t *k_cach
     scale = 1.0;
 #endif
     for (int d = 0; d < head_dim; ++d)
-        out[d] = 0.0;
-    if (nkeys <= 0)
+        acc[d] = 0.0;
+    if (nkeys <= 0) {
+        memcpy(out, acc, sizeof(double) * (size_t)head_dim);
         return ORACLE_OK; /* softmax over an empty set: the output is defined as zeros */
+    }
 
     double m = -INFINITY;
     for (int j = 0; j < nkeys; ++j) {
@@ -197,15 +201,16 @@ static int attend_one(double *out, const uint16_t *q_row, const uint16_t *k_cach
         long long blk = row / block_size, off = row % block_size;
         const uint16_t *vrow = v_cache + ((blk * num_kv_heads + kvh) * block_size + off) * head_dim;
         for (int d = 0; d < head_dim; ++d)
-            out[d] += w * bf16_bits_to_double(vrow[d]);
+            acc[d] += w * bf16_bits_to_double(vrow[d]);
         denom += w;
     }
 #if ORACLE_MUTATION != 5
     for (int d = 0; d < head_dim; ++d)
-        out[d] /= denom;
+        acc[d] /= denom;
 #else
     (void)denom;
 #endif
+    memcpy(out, acc, sizeof(double) * (size_t)head_dim);
     return ORACLE_OK;
 }
 
@@ -246,13 +251,14 @@ int oracle_paged_attention(double *out, const uint16_t *q, const uint16_t *k_cac
 #pragma omp parallel
     {
         double *scores = (double *)malloc(sizeof(double) * (size_t)(max_ctx > 0 ? max_ctx : 1));
-        if (!scores) {
+        double *acc = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        if (!scores || !acc) {
 #pragma omp atomic write
             status = ORACLE_ERR_NOMEM;
         }
 #pragma omp for schedule(dynamic, 1)
         for (long long it = 0; it < n_items; ++it) {
-            if (!scores)
+            if (!scores || !acc)
                 continue;
             int t, h;
             if (only_rows) {
@@ -273,13 +279,14 @@ int oracle_paged_attention(double *out, const uint16_t *q, const uint16_t *k_cac
 #else
                                 h / group,
 #endif
-                                num_kv_heads, head_dim, block_size, num_blocks, scale, scores);
+                                num_kv_heads, head_dim, block_size, num_blocks, scale, scores, acc);
             if (rc != ORACLE_OK) {
 #pragma omp atomic write
                 status = rc;
             }
         }
         free(scores);
+        free(acc);
     }
     free(seq_of);
     return status;

@@ -11,7 +11,7 @@ from __future__ import annotations
 
 __all__ = [
     "pa_cache_append", "pa_decode", "pa_prefill_chunk", "pa_workspace_bytes",
-    "pa_status_string", "PAError", "library_path",
+    "pa_status_string", "PAError", "library_path", "make_workspace", "status_bit",
 ]
 
 

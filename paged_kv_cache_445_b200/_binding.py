@@ -1,0 +1,160 @@
+"""ctypes binding of libpa.so: argument marshalling only.
+
+Every function here checks the tensors' dtype, device, contiguity and shape,
+passes raw device pointers, sizes and the current CUDA stream to the C entry
+point of the same name (``include/pa.h``), and raises ``PAError`` on a
+non-zero status.  All computation happens in the library's kernels; if the
+library is missing this module fails to import -- there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpa.so")
+if not os.path.exists(library_path):
+    raise ImportError(f"{library_path} is missing: build it with `python -m paged_kv_cache_445_b200.csrc.build` "
+                      "(needs nvcc); there is no CPU fallback")
+_lib = ctypes.CDLL(library_path)
+
+_vp, _ci, _i32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+_lib.pa_cache_append.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _ci, _ci, _ci, _ci, _vp, _vp]
+_lib.pa_cache_append.restype = _ci
+_lib.pa_workspace_bytes.argtypes = [_ci, _ci, _ci, _ci]
+_lib.pa_workspace_bytes.restype = ctypes.c_size_t
+_lib.pa_decode.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci, ctypes.c_float,
+                           _vp, ctypes.c_size_t, _vp, _vp]
+_lib.pa_decode.restype = _ci
+_lib.pa_prefill_chunk.argtypes = [_vp, _vp, _i32p, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci, _ci,
+                                  ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
+_lib.pa_prefill_chunk.restype = _ci
+_lib.pa_status_string.argtypes = [_ci]
+_lib.pa_status_string.restype = ctypes.c_char_p
+
+PA_OK = 0
+PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE = -1, -2, -3, -4
+PA_ERR_RANGE, PA_ERR_CUDA, PA_ERR_TIMEOUT = -5, -6, -7
+
+
+def status_bit(code: int) -> int:
+    """Bit a kernel ORs into the device status word for device error ``code``."""
+    return 1 << (-code)
+
+
+class PAError(RuntimeError):
+    def __init__(self, code: int):
+        self.code = code
+        super().__init__(pa_status_string(code))
+
+
+def pa_status_string(code: int) -> str:
+    return _lib.pa_status_string(int(code)).decode()
+
+
+def _check(rc: int) -> None:
+    if rc != PA_OK:
+        raise PAError(rc)
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = None) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {tuple(t.shape)}")
+    return t.data_ptr()
+
+
+def _status_ptr(dev_status) -> int | None:
+    if dev_status is None:
+        return None
+    return _dev(dev_status, "dev_status", torch.int32)
+
+
+def _stream_ptr(stream) -> int | None:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream if hasattr(s, "cuda_stream") else int(s)
+
+
+def pa_cache_append(k_new, v_new, k_cache, v_cache, slot_mapping, dev_status=None, stream=None) -> None:
+    """Scatter k_new/v_new [T, Hkv, d] (bf16) into k_cache/v_cache
+    [num_blocks, Hkv, block_size, d] at slot_mapping [T] (int32; < 0 = skip)."""
+    kp = _dev(k_new, "k_new", torch.bfloat16, 3)
+    vp = _dev(v_new, "v_new", torch.bfloat16, 3)
+    kc = _dev(k_cache, "k_cache", torch.bfloat16, 4)
+    vc = _dev(v_cache, "v_cache", torch.bfloat16, 4)
+    sm = _dev(slot_mapping, "slot_mapping", torch.int32, 1)
+    nb, hkv, bs, d = k_cache.shape
+    if v_cache.shape != k_cache.shape or k_new.shape != v_new.shape:
+        raise ValueError("k and v tensors must have the same shapes")
+    if k_new.shape[1:] != (hkv, d) or slot_mapping.shape[0] != k_new.shape[0]:
+        raise ValueError("k_new must be [T, Hkv, d] and slot_mapping [T]")
+    _check(_lib.pa_cache_append(kp, vp, kc, vc, sm, k_new.shape[0], nb, hkv, d, bs, _status_ptr(dev_status),
+                                _stream_ptr(stream)))
+
+
+def pa_workspace_bytes(num_query_tokens: int, num_q_heads: int, num_kv_heads: int, head_dim: int) -> int:
+    n = int(_lib.pa_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim))
+    if n == 0:
+        raise PAError(PA_ERR_UNSUPPORTED)
+    return n
+
+
+def make_workspace(num_query_tokens: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                   device=None) -> torch.Tensor:
+    """A zero-filled workspace of pa_workspace_bytes() bytes (the zero fill is required once)."""
+    n = pa_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _attention_args(out, q, k_cache, v_cache, block_tables, context_lens, workspace):
+    op = _dev(out, "out", torch.bfloat16, 3)
+    qp = _dev(q, "q", torch.bfloat16, 3)
+    kc = _dev(k_cache, "k_cache", torch.bfloat16, 4)
+    vc = _dev(v_cache, "v_cache", torch.bfloat16, 4)
+    bt = _dev(block_tables, "block_tables", torch.int32, 2)
+    cl = _dev(context_lens, "context_lens", torch.int32, 1)
+    ws = _dev(workspace, "workspace", torch.uint8, 1)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    if v_cache.shape != k_cache.shape or k_cache.shape[3] != q.shape[2]:
+        raise ValueError("k_cache/v_cache must be [num_blocks, Hkv, block_size, d] with q's d")
+    if block_tables.shape[0] != context_lens.shape[0]:
+        raise ValueError("block_tables and context_lens must have one row per sequence")
+    return op, qp, kc, vc, bt, cl, ws
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, workspace, dev_status=None,
+              stream=None) -> None:
+    """One decode row per sequence: q/out [B, Hq, d]; see include/pa.h."""
+    op, qp, kc, vc, bt, cl, ws = _attention_args(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    nb, hkv, bs, d = k_cache.shape
+    if q.shape[0] != context_lens.shape[0]:
+        raise ValueError("pa_decode takes exactly one query row per sequence")
+    _check(_lib.pa_decode(op, qp, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0], q.shape[1], hkv, d,
+                          bs, nb, float(scale), ws, workspace.numel(), _status_ptr(dev_status), _stream_ptr(stream)))
+
+
+def pa_prefill_chunk(out, q, query_start, k_cache, v_cache, block_tables, context_lens, scale, workspace,
+                     dev_status=None, stream=None) -> None:
+    """Varlen batch of prefill chunks and decodes: q/out [Tq, Hq, d],
+    query_start [B + 1]; see include/pa.h."""
+    op, qp, kc, vc, bt, cl, ws = _attention_args(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    qs = _dev(query_start, "query_start", torch.int32, 1)
+    if query_start.shape[0] != context_lens.shape[0] + 1:
+        raise ValueError("query_start must have num_seqs + 1 entries")
+    nb, hkv, bs, d = k_cache.shape
+    _check(_lib.pa_prefill_chunk(op, qp, qs, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0], q.shape[0],
+                                 q.shape[1], hkv, d, bs, nb, float(scale), ws, workspace.numel(),
+                                 _status_ptr(dev_status), _stream_ptr(stream)))
+
+
+def exported_symbols() -> list[str]:
+    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_prefill_chunk", "pa_status_string"]

@@ -1,0 +1,196 @@
+// pa_api.cu -- the C ABI of libpa.so: argument checks, tensor maps, workspace
+// layout and dispatch to the kernels.  See include/pa.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+constexpr int MAX_DEVICES = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+// Workspace: [arrival counters: Tq * Hkv int32][rows-kernel partial slots]
+size_t counters_bytes(int num_query_tokens, int num_kv_heads) {
+  return round256(static_cast<size_t>(num_query_tokens) * num_kv_heads * sizeof(int32_t));
+}
+
+}  // namespace
+
+int device_info(DeviceInfo* info) {
+  static int sms[MAX_DEVICES] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return PA_ERR_CUDA;
+  if (sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return PA_ERR_CUDA;
+    sms[dev] = n;
+  }
+  info->num_sms = sms[dev];
+  return PA_OK;
+}
+
+// [num_blocks, Hkv, block_size, D] bf16 viewed as a 4-D tensor (D fastest);
+// box = 64 columns x 16 token rows of one (block, head), 128-byte swizzle.
+int encode_kv_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
+                   int head_dim) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return PA_ERR_CUDA;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(block_size),
+                              static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * 2;
+  const cuuint64_t strides[3] = {row, row * block_size, row * block_size * num_kv_heads};
+  const cuuint32_t box[4] = {64, 16, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(cache), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+static int check_attention_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                 int num_blocks, int max_blocks) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks <= 0)
+    return PA_ERR_SHAPE;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_SHAPE;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (!rows_supported(num_q_heads / num_kv_heads, head_dim)) return PA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_blocks) * block_size > 0x7fffffffLL) return PA_ERR_SHAPE;
+  return PA_OK;
+}
+
+static size_t workspace_needed(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim, int num_sms) {
+  return counters_bytes(num_query_tokens, num_kv_heads) +
+         round256(rows_partials_bytes(num_q_heads, num_kv_heads, head_dim, num_sms));
+}
+
+static int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache,
+                         const void* v_cache, const int32_t* block_tables, int max_blocks,
+                         const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace) return PA_ERR_NULL;
+  int rc = check_attention_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks);
+  if (rc != PA_OK) return rc;
+  if (total_q_tokens < 0) return PA_ERR_SHAPE;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_ERR_SHAPE;
+  if (num_seqs == 0 || total_q_tokens == 0) return PA_OK;
+  DeviceInfo di;
+  if ((rc = device_info(&di)) != PA_OK) return rc;
+  if (workspace_bytes < workspace_needed(total_q_tokens, num_q_heads, num_kv_heads, head_dim, di.num_sms))
+    return PA_ERR_WORKSPACE;
+
+  CUtensorMap tmk, tmv;
+  if ((rc = encode_kv_tmap(&tmk, k_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
+  if ((rc = encode_kv_tmap(&tmv, v_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  RowsParams p{};
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.query_start = query_start;
+  p.num_seqs = num_seqs;
+  p.max_blocks = max_blocks;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.block_size = block_size;
+  p.num_blocks = num_blocks;
+  p.skip_multi = 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.counters = reinterpret_cast<int*>(ws);
+  p.partials = reinterpret_cast<float*>(ws + counters_bytes(total_q_tokens, num_kv_heads));
+  p.status = dev_status;
+  return launch_rows(p, tmk, tmv, head_dim, static_cast<cudaStream_t>(stream), di.num_sms);
+}
+
+}  // namespace pa
+
+extern "C" {
+
+int pa_cache_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache, const int32_t* slot_mapping,
+                    int num_tokens, int num_blocks, int num_kv_heads, int head_dim, int block_size, int* dev_status,
+                    void* stream) {
+  if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0) return PA_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PA_ERR_NULL;
+  if (!pa::aligned16(k_new) || !pa::aligned16(v_new) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache))
+    return PA_ERR_SHAPE;
+  pa::DeviceInfo di;
+  int rc = pa::device_info(&di);
+  if (rc != PA_OK) return rc;
+  return pa::launch_append(k_new, v_new, k_cache, v_cache, slot_mapping, num_tokens, num_blocks, num_kv_heads,
+                           head_dim, block_size, dev_status, static_cast<cudaStream_t>(stream), di.num_sms);
+}
+
+size_t pa_workspace_bytes(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim) {
+  if (num_query_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads) return 0;
+  if (!pa::rows_supported(num_q_heads / num_kv_heads, head_dim)) return 0;
+  pa::DeviceInfo di;
+  if (pa::device_info(&di) != PA_OK) return 0;
+  return pa::workspace_needed(num_query_tokens, num_q_heads, num_kv_heads, head_dim, di.num_sms);
+}
+
+int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+              int max_blocks_per_seq, const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+              int head_dim, int block_size, int num_blocks, float scale, void* workspace, size_t workspace_bytes,
+              int* dev_status, void* stream) {
+  return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                           num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                           workspace, workspace_bytes, dev_status, stream);
+}
+
+int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,
+                     const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                     int total_q_tokens, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                     int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
+                     void* stream) {
+  if (!query_start) return PA_ERR_NULL;
+  return pa::run_attention(out, q, query_start, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                           num_seqs, total_q_tokens, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                           scale, workspace, workspace_bytes, dev_status, stream);
+}
+
+const char* pa_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_NULL: return "PA_ERR_NULL: a required pointer is NULL";
+    case PA_ERR_SHAPE: return "PA_ERR_SHAPE: inconsistent sizes or misaligned pointer";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: head_dim, block_size or group outside the supported set";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace smaller than pa_workspace_bytes()";
+    case PA_ERR_RANGE: return "PA_ERR_RANGE: block ID, slot or context outside its table or pool";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: a CUDA call failed";
+    case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT: a bounded device wait gave up";
+    default: return "unknown pa_status";
+  }
+}
+
+}  // extern "C"

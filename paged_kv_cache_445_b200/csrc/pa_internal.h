@@ -1,0 +1,54 @@
+// pa_internal.h -- host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+// Parameters of the single-row attention kernel (decode rows, and the rows of
+// any sequence the chunk kernel does not take).
+struct RowsParams {
+  void* out;                    // bf16 [Tq, Hq, D]
+  const void* q;                // bf16 [Tq, Hq, D]
+  const int32_t* block_tables;  // [B, max_blocks]
+  const int32_t* context_lens;  // [B]
+  const int32_t* query_start;   // [B + 1], or nullptr: one query row per sequence
+  int num_seqs;
+  int max_blocks;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int block_size;
+  int num_blocks;
+  int skip_multi;   // 1: sequences with more than one query row belong to the chunk kernel
+  float scale_log2; // softmax scale * log2(e)
+  float* partials;  // workspace: two partial-result slots per warp
+  int* counters;    // workspace: one arrival counter per (query row, KV head), zero between calls
+  int* status;      // optional device status word
+  int total_warps;
+};
+
+struct DeviceInfo {
+  int num_sms;
+};
+
+int device_info(DeviceInfo* info);
+int encode_kv_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
+                   int head_dim);
+
+// Each returns a pa_status.
+int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache, const int32_t* slot_mapping,
+                  int num_tokens, int num_blocks, int num_kv_heads, int head_dim, int block_size, int* dev_status,
+                  cudaStream_t stream, int num_sms);
+int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
+                cudaStream_t stream, int num_sms);
+// Upper bound of the rows kernel's workspace for this shape on a device with num_sms SMs.
+size_t rows_partials_bytes(int num_q_heads, int num_kv_heads, int head_dim, int num_sms);
+int rows_supported(int group, int head_dim);
+
+}  // namespace pa

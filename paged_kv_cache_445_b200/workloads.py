@@ -213,18 +213,13 @@ def build(spec: Spec, seed: int, poison: bool = False, max_blocks: int | None = 
     q = normal_bf16(seed, 5, (tq, hq, d), std=spec.q_std)
 
     if poison:
-        valid = np.zeros(nb * bs, dtype=bool)
+        valid = np.zeros((nb, bs), dtype=bool)
         for s in seq_ids:
-            tab = block_tables[s]
-            for pos in range(int(prefix[s])):
-                valid[tab[pos // bs] * bs + pos % bs] = True
-        slots_bad = ~valid
-        kv = k_cache.reshape(nb, hkv, bs, d).transpose(0, 2, 1, 3).reshape(nb * bs, hkv, d)
-        vv = v_cache.reshape(nb, hkv, bs, d).transpose(0, 2, 1, 3).reshape(nb * bs, hkv, d)
-        kv[slots_bad] = BF16_NAN
-        vv[slots_bad] = BF16_NAN
-        k_cache = np.ascontiguousarray(kv.reshape(nb, bs, hkv, d).transpose(0, 2, 1, 3))
-        v_cache = np.ascontiguousarray(vv.reshape(nb, bs, hkv, d).transpose(0, 2, 1, 3))
+            pos = np.arange(int(prefix[s]), dtype=np.int64)
+            valid[block_tables[s, pos // bs], pos % bs] = True
+        bad = ~valid
+        k_cache.transpose(0, 2, 1, 3)[bad] = BF16_NAN  # views: writes land in the caches
+        v_cache.transpose(0, 2, 1, 3)[bad] = BF16_NAN
 
     return Workload(spec.name, hq, hkv, d, bs, nb, 1.0 / math.sqrt(d), q, k_new, v_new,
                     k_cache, v_cache, block_tables, context_lens, query_start, slot_mapping,

@@ -1,0 +1,209 @@
+"""GPU parity: libpa.so (through the C-ABI binding) against the fp64 oracle.
+
+Append and slot indexing must be bit-exact; attention outputs must be within
+1e-2 max-abs and 5e-3 relative-L2 error of the oracle (bf16 inputs, fp32
+accumulation, bf16 output).  Caches are poisoned: every slot that does not
+hold a valid token holds NaN, so reading past a context shows up.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_445_b200 import workloads
+from tests.gpu_helpers import DeviceStep, compare, dev_to_bits, i32, oracle_after_append
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    import paged_kv_cache_445_b200 as pa  # noqa: F401  (fails loudly without libpa.so)
+
+
+def _attend_ref(w, kc, vc, only=None):
+    return oracle.paged_attention(w.q, kc, vc, w.block_tables, w.context_lens, w.query_start, w.scale, only=only)
+
+
+# ------------------------------------------------------------------ append
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+def test_append_is_bit_exact_on_the_standard_workloads(cfg):
+    w = workloads.standard(cfg, poison=True)
+    ds = DeviceStep(w)
+    ds.append()
+    torch.cuda.synchronize()
+    kc, vc = oracle_after_append(w)
+    assert np.array_equal(dev_to_bits(ds.k_cache), kc)
+    assert np.array_equal(dev_to_bits(ds.v_cache), vc)
+    assert int(ds.status.item()) == 0
+
+
+def test_append_skips_padding_and_reports_out_of_range_slots():
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.custom([10, 40, 3], [1, 1, 1], 4, 2, 128, 16, seed=21)
+    ds = DeviceStep(w)
+    slots = w.slot_mapping.copy()
+    slots[1] = -1
+    slots[2] = w.num_blocks * w.block_size + 7  # outside the pool
+    ds.slot_mapping = i32(slots)
+    before_k = dev_to_bits(ds.k_cache)
+    ds.append()
+    torch.cuda.synchronize()
+    got = dev_to_bits(ds.k_cache)
+    want = before_k.copy()
+    s0 = int(slots[0])
+    want[s0 // 16, :, s0 % 16, :] = w.k_new[0]
+    assert np.array_equal(got, want)
+    assert int(ds.status.item()) == pa.status_bit(pa._binding.PA_ERR_RANGE)
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_decode_matches_oracle_on_the_standard_workloads(cfg):
+    w = workloads.standard(cfg, poison=True)
+    ds = DeviceStep(w)
+    got = ds.step()
+    kc, vc = oracle_after_append(w)
+    compare(got, _attend_ref(w, kc, vc), f"config {cfg}")
+    assert int(ds.status.item()) == 0
+
+
+def test_mixed_chunk_and_decodes_match_oracle():
+    w = workloads.standard(5, poison=True)
+    ds = DeviceStep(w)
+    got = ds.step()
+    kc, vc = oracle_after_append(w)
+    hq = w.num_q_heads
+    rng = np.random.default_rng(5)
+    # every decode row, and chunk rows at both ends, the middle and random ones, over all heads in a group
+    chunk_tokens = sorted({0, 1, 15, 16, 255, 256, 510, 511, *rng.integers(0, 512, 8).tolist()})
+    only = [(t, h) for t in range(512, w.num_query_tokens) for h in range(hq)]
+    only += [(t, h) for t in chunk_tokens for h in (0, 7, 8, 31, 63, *rng.integers(0, hq, 3).tolist())]
+    only = sorted(set(only))
+    ref = _attend_ref(w, kc, vc, only=np.array(only))
+    idx = tuple(np.array(only).T)
+    compare(got[idx], ref[idx], "config 5 sampled rows")
+    assert int(ds.status.item()) == 0
+
+
+SMALL = [  # ctx list, qlen list, Hq, Hkv, d, bs
+    ([1, 15, 16, 17, 33, 100, 257], [1] * 7, 8, 1, 128, 16),
+    ([1, 31, 32, 33, 65, 300], [1] * 6, 8, 4, 64, 32),
+    ([5, 16, 40, 129, 700], [1] * 5, 12, 2, 256, 16),
+    ([3, 32, 64, 500], [1] * 4, 16, 1, 128, 32),
+    ([17, 90, 1000], [1] * 3, 32, 2, 128, 16),
+    ([2, 77, 400, 1300], [1] * 4, 4, 4, 64, 16),
+    ([64, 200], [40, 1], 8, 2, 128, 16),
+    ([50, 9, 300, 1], [50, 3, 17, 1], 6, 3, 64, 32),
+    ([600], [77], 24, 4, 256, 32),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"Hq{c[2]}-Hkv{c[3]}-d{c[4]}-bs{c[5]}-q{max(c[1])}")
+def test_small_shapes_match_oracle(case):
+    ctx, qlen, hq, hkv, d, bs = case
+    prefix = [c - q for c, q in zip(ctx, qlen)]
+    w = workloads.custom(prefix, qlen, hq, hkv, d, bs, seed=sum(ctx), poison=True)
+    ds = DeviceStep(w)
+    got = ds.step()
+    kc, vc = oracle_after_append(w)
+    compare(got, _attend_ref(w, kc, vc), str(case))
+    assert int(ds.status.item()) == 0
+
+
+def test_varlen_entry_on_a_pure_decode_batch_equals_decode_entry():
+    w = workloads.custom([30, 700, 4000], [1, 1, 1], 16, 2, 128, 16, seed=3, poison=True)
+    a = DeviceStep(w).step()
+    b = DeviceStep(w).step(force_varlen=True)
+    assert np.array_equal(a, b)
+
+
+def test_long_segments_split_over_many_warps_merge_exactly():
+    # two very long contexts: each (row, head) segment spans dozens of warps
+    w = workloads.custom([32000, 24999], [1, 1], 16, 2, 128, 16, seed=4, poison=True)
+    ds = DeviceStep(w)
+    got = ds.step()
+    kc, vc = oracle_after_append(w)
+    compare(got, _attend_ref(w, kc, vc), "long contexts")
+
+
+def test_results_are_deterministic_and_workspace_is_reusable():
+    w = workloads.custom([100, 2000, 5000, 9], [1, 1, 1, 1], 8, 1, 128, 16, seed=6)
+    ds = DeviceStep(w)
+    ds.append()
+    outs = []
+    for _ in range(3):
+        ds.attend()
+        torch.cuda.synchronize()
+        outs.append(ds.out.clone())
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+
+
+def test_empty_context_gives_zeros():
+    w = workloads.custom([0, 40, 0], [1, 1, 1], 8, 2, 128, 16, seed=7)
+    ds = DeviceStep(w)
+    ds.append()
+    cl = w.context_lens.copy()
+    cl[0] = 0  # sequence 0 has no key at all
+    ds.context_lens = i32(cl)
+    ds.out.fill_(7.0)
+    ds.attend()
+    torch.cuda.synchronize()
+    got = ds.out.float().cpu().numpy()
+    assert np.all(got[0] == 0)
+    kc, vc = oracle_after_append(w)
+    ref = oracle.paged_attention(w.q, kc, vc, w.block_tables, cl, w.query_start, w.scale)
+    compare(got, ref, "empty context")
+
+
+def test_guard_regions_are_untouched():
+    w = workloads.custom([33, 200, 5], [1, 1, 1], 8, 2, 128, 16, seed=8)
+    ds = DeviceStep(w)
+    big = torch.full((w.num_query_tokens + 4, w.num_q_heads, w.head_dim), 3.0, dtype=torch.bfloat16, device="cuda")
+    ds.out = big[2:-2]
+    ds.step()
+    assert torch.all(big[:2] == 3.0) and torch.all(big[-2:] == 3.0)
+
+
+def test_bad_block_ids_and_long_contexts_are_reported_not_faulted():
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.custom([40, 60], [1, 1], 8, 2, 128, 16, seed=9)
+    ds = DeviceStep(w)
+    ds.append()
+    bt = w.block_tables.copy()
+    bt[0, 1] = w.num_blocks + 1000  # outside the pool
+    ds.block_tables = i32(bt)
+    ds.attend()
+    torch.cuda.synchronize()
+    assert int(ds.status.item()) & pa.status_bit(pa._binding.PA_ERR_RANGE)
+    ds.status.zero_()
+    cl = w.context_lens.copy()
+    cl[1] = bt.shape[1] * w.block_size + 50  # longer than its table
+    ds.context_lens = i32(cl)
+    ds.block_tables = i32(w.block_tables)
+    ds.workspace.zero_()
+    ds.attend()
+    torch.cuda.synchronize()
+    assert int(ds.status.item()) & pa.status_bit(pa._binding.PA_ERR_RANGE)
+    # the context stays usable
+    ds.status.zero_()
+    ds.context_lens = i32(w.context_lens)
+    ds.workspace.zero_()
+    ds.attend()
+    torch.cuda.synchronize()
+    assert int(ds.status.item()) == 0
+
+
+def test_small_workspace_is_rejected():
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.custom([40], [1], 8, 2, 128, 16, seed=10)
+    ds = DeviceStep(w)
+    ds.workspace = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pa.PAError) as e:
+        ds.attend()
+    assert e.value.code == pa._binding.PA_ERR_WORKSPACE

@@ -1,0 +1,85 @@
+"""The C-ABI library loads and exports every entry point of include/pa.h;
+host-side argument checks answer without touching a GPU (CPU only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_445_b200.csrc import build as pabuild
+
+HEADER = os.path.join(pabuild.ROOT, "include", "pa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*PA_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*(pa_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = pabuild.build()
+    lib = ctypes.CDLL(path)
+    return lib
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("pa_cache_append", "pa_decode", "pa_prefill_chunk", "pa_workspace_bytes", "pa_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_only_the_boundary_is_exported():
+    out = os.popen(f"nm -D --defined-only {pabuild.LIB}").read()
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert {n for n in exported if n.startswith("pa_")} == set(declared_functions())
+
+
+def test_status_strings(lib):
+    lib.pa_status_string.restype = ctypes.c_char_p
+    for code in range(0, -8, -1):
+        s = lib.pa_status_string(code).decode()
+        assert s.startswith("PA_") or code == 0
+    assert lib.pa_status_string(0).decode() == "PA_OK"
+    assert b"unknown" in lib.pa_status_string(42)
+
+
+def test_host_checks_answer_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                              ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, vp, ctypes.c_size_t, vp, vp]
+    fake = 4096
+    # null output
+    assert lib.pa_decode(None, fake, fake, fake, fake, 4, fake, 4, 8, 2, 128, 16, 10, 0.1, fake, 1 << 20, None,
+                         None) == -1
+    # Hq not a multiple of Hkv
+    assert lib.pa_decode(fake, fake, fake, fake, fake, 4, fake, 4, 6, 4, 128, 16, 10, 0.1, fake, 1 << 20, None,
+                         None) == -2
+    # unsupported head_dim and block_size
+    assert lib.pa_decode(fake, fake, fake, fake, fake, 4, fake, 4, 8, 2, 96, 16, 10, 0.1, fake, 1 << 20, None,
+                         None) == -3
+    assert lib.pa_decode(fake, fake, fake, fake, fake, 4, fake, 4, 8, 2, 128, 8, 10, 0.1, fake, 1 << 20, None,
+                         None) == -3
+    # group too wide for head_dim 256
+    assert lib.pa_decode(fake, fake, fake, fake, fake, 4, fake, 4, 16, 1, 256, 16, 10, 0.1, fake, 1 << 20, None,
+                         None) == -3
+    lib.pa_cache_append.argtypes = [vp, vp, vp, vp, vp] + [ctypes.c_int] * 5 + [vp, vp]
+    assert lib.pa_cache_append(fake, fake, fake, fake, fake, 0, 4, 2, 128, 16, None, None) == 0  # nothing to do
+    assert lib.pa_cache_append(fake, fake, fake, fake, fake, 3, 4, 2, 100, 16, None, None) == -3
+    assert lib.pa_cache_append(None, fake, fake, fake, fake, 3, 4, 2, 128, 16, None, None) == -1
+    lib.pa_workspace_bytes.restype = ctypes.c_size_t
+    assert lib.pa_workspace_bytes(4, 6, 4, 128) == 0  # bad group -> 0
+
+
+def test_python_binding_imports_on_cpu():
+    import paged_kv_cache_445_b200 as pa
+    assert pa.pa_status_string(-4).startswith("PA_ERR_WORKSPACE")
+    assert pa.status_bit(-5) == 32

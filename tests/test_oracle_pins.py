@@ -272,6 +272,19 @@ def pin_slot_mapping_closed_form(lib):
     assert got.tolist() == [2 * 4 + 3, 5 * 4 + 0, 5 * 4 + 1, 0 * 4 + 0, 0 * 4 + 1]
 
 
+def pin_sampled_rows_equal_full_rows(lib):
+    rng = np.random.default_rng(17)
+    lens, qlens, hq, hkv, d, bs = [90, 33, 7], [20, 1, 3], 8, 2, 16, 16
+    k_seqs, v_seqs, q, nb = _contiguous_case(rng, lens, qlens, hq, hkv, d, bs)
+    kc, vc, bt = scatter_to_pool(k_seqs, v_seqs, bs, nb, rng.permutation(nb))
+    qs = np.concatenate([[0], np.cumsum(qlens)])
+    full = _attend(lib, q, kc, vc, bt, np.array(lens), qs, 0.3)
+    only = [(t, h) for t in (0, 5, 19, 20, 22) for h in (0, 3, 3, 7, 0)]  # with duplicates
+    part = oracle.paged_attention(q, kc, vc, bt, np.array(lens), qs, 0.3, only=np.array(only * 3), lib=lib)
+    for t, h in only:
+        assert np.array_equal(part[t, h], full[t, h])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
