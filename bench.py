@@ -1,0 +1,470 @@
+"""Benchmark of one engine step of paged attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3] [--impl ours|reference]
+
+A step is one pass of the hot path over one batch: ``pa_cache_append`` of the
+step's new K/V rows, then attention (``pa_decode`` for a decode batch,
+``pa_prefill_chunk`` for the mixed batch).  Block tables and slots come from
+the host allocator before timing.  The default workload is the Llama-3.3-70B-
+like attention layer at concurrency 128 (64 query heads, 8 KV heads, head_dim
+128, 16-token blocks, lognormal contexts with median 1500 clipped to
+[16, 8192]).
+
+Prints one JSON line.  ``value`` is KV GB/s: the KV bytes the step must read
+(every cached token once, K and V, all KV heads) times the number of ranks,
+over the device time per step (CUDA events, max over ranks).  ``e2e`` repeats
+the step through the same C-ABI calls with host buffers: the per-step inputs
+are copied from pinned host memory and the output back inside the timed
+region.  ``roofline`` rates the dominant kernel (attention) from its own
+per-launch CUDA-event times against the measured HBM copy bandwidth.
+
+Multi-GPU: one process per GPU (torchrun); each rank runs its own batch (weak
+scaling, no collective on the data path; an all-reduce of the timings only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_BYTES = 126 * 1024 * 1024
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_445_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """dram read+write bytes per launch from a committed ncu summary, if it was
+    taken on the current kernel sources; else None."""
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    t = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.e+]+)", text)
+    if not m or not t or m.group(1) != kernel_source_hash():
+        return None
+    return float(t.group(1))
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_device: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_device)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: the line says so
+            log(f"clock sampling unavailable: {e}")
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = get_reasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------- workload
+def step_bytes(w):
+    from paged_kv_cache_445_b200 import roofline
+    kv = roofline.decode_kv_bytes(w.context_lens, w.num_kv_heads, w.head_dim)
+    attn = roofline.attention_algorithmic_bytes(w.context_lens, w.query_start, w.num_q_heads, w.num_kv_heads,
+                                                w.head_dim, w.block_size)
+    app = roofline.append_algorithmic_bytes(len(w.slot_mapping), w.num_kv_heads, w.head_dim)
+    flops = roofline.prefill_flops(w.context_lens, w.query_start, w.num_q_heads, w.head_dim)
+    return kv, attn, app, flops
+
+
+class GpuStep:
+    def __init__(self, w, device):
+        import torch
+
+        import paged_kv_cache_445_b200 as pa
+        self.pa, self.torch, self.w = pa, torch, w
+
+        def bf(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+        def i32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(device)
+
+        self.k_cache, self.v_cache = bf(w.k_cache), bf(w.v_cache)
+        self.k_new, self.v_new, self.q = bf(w.k_new), bf(w.v_new), bf(w.q)
+        self.block_tables, self.context_lens = i32(w.block_tables), i32(w.context_lens)
+        self.query_start, self.slot_mapping = i32(w.query_start), i32(w.slot_mapping)
+        self.out = torch.empty_like(self.q)
+        self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim, device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.decode = w.is_decode
+
+    def append(self):
+        self.pa.pa_cache_append(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping, self.status)
+
+    def attend(self):
+        if self.decode:
+            self.pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
+                              self.w.scale, self.workspace, self.status)
+        else:
+            self.pa.pa_prefill_chunk(self.out, self.q, self.query_start, self.k_cache, self.v_cache,
+                                     self.block_tables, self.context_lens, self.w.scale, self.workspace, self.status)
+
+
+def run_ours(args, peaks):
+    import torch
+
+    from paged_kv_cache_445_b200 import workloads
+    rank, world, local = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    t0 = time.time()
+    w = workloads.standard(args.workload, seed=445 + args.workload + 1000 * rank)
+    log(f"[rank {rank}] workload {w.name}: {w.num_seqs} seqs, {w.num_query_tokens} query rows, "
+        f"{int(w.context_lens.sum())} keys, pool {w.num_blocks} blocks ({time.time() - t0:.1f}s to generate)")
+    g = GpuStep(w, device)
+    kv_bytes, attn_bytes, app_bytes, flops = step_bytes(w)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        g.append()
+        g.attend()
+    torch.cuda.synchronize()
+    if int(g.status.item()) != 0:
+        raise SystemExit(f"device status {int(g.status.item())} after warm-up")
+
+    # ---- device-timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        start.record(stream)
+        for i in range(args.steps):
+            g.append()
+            ev[i][0].record(stream)
+            g.attend()
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = start.elapsed_time(end)
+    attn_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_step = max_over_ranks(ms_total / args.steps, world)
+    attn_avg_ms = max_over_ranks(sum(attn_ms) / len(attn_ms), world)
+    if int(g.status.item()) != 0:
+        raise SystemExit(f"device status {int(g.status.item())} after timing")
+
+    # ---- end to end through the public calls with host buffers
+    pin = {name: getattr(g, name).cpu().pin_memory() for name in
+           ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens", "query_start")}
+    out_host = torch.empty(g.out.shape, dtype=g.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for k, t in pin.items() if g.decode is False or k != "query_start")
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, t in pin.items():
+            if g.decode and k == "query_start":
+                continue
+            getattr(g, k).copy_(t, non_blocking=True)
+        g.append()
+        g.attend()
+        out_host.copy_(g.out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world)
+
+    # ---- CPU baseline: the oracle on this host's cores, rank 0 at N = 1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(w, args.cpu_seconds)
+
+    clocks = sampler.summary()
+    hbm, bf16_burst, bf16_sust, peak_src = peaks
+    achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
+    traffic = profiled_traffic("pa_rows_kernel", w.name)
+    line = {
+        "metric": "paged-attn decode KV GB/s + seq-steps/s (70B layer, bs128); % of HBM peak",
+        "value": round(world * kv_bytes / (ms_step * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded PCG64, bf16 N(0,1) K/V, q N(0,0.5^2)); no weights",
+        "config": {
+            "workload": w.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
+            "num_blocks": w.num_blocks, "query_rows": w.num_query_tokens,
+            "context_tokens": int(w.context_lens.sum()), "kv_bytes_per_step": kv_bytes,
+            "l2": f"no flush: every step reads {kv_bytes / 1e9:.2f} GB of KV, larger than the 126 MB L2",
+            "parallelism": f"dp{world} (independent batch per GPU)",
+        },
+        "seq_steps_per_s": round(world * w.num_seqs / (ms_step * 1e-3), 1),
+        "frac_of_hbm_peak": round(world * kv_bytes / (ms_step * 1e-3) / 1e9 / hbm / world, 4),
+        "frac_of_8tbs_nominal": round(kv_bytes / (ms_step * 1e-3) / 1e9 / 8000.0, 4),
+        "roofline": {
+            "kernel": "pa_rows_kernel (attention)", "bound": "hbm",
+            "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+            if peak_src == "measured" else "fallback 6.65 TB/s",
+            "traffic": traffic, "algorithmic_bytes_per_launch": attn_bytes,
+            "avg_launch_ms": round(attn_avg_ms, 5),
+        },
+        "append": {"algorithmic_bytes": app_bytes},
+        "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if not w.is_decode:
+        line["roofline_tensor"] = {"flops_per_step": flops, "achieved_tflops": round(flops / (attn_avg_ms * 1e-3) / 1e12, 1),
+                                   "peak": bf16_sust, "unit": "TFLOP/s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------- oracle
+def oracle_sample(w, max_rows: int):
+    """The first sequences of the batch (all heads), up to max_rows query rows."""
+    import oracle
+    rows = []
+    qs = w.query_start
+    for s in range(w.num_seqs):
+        for t in range(int(qs[s]), int(qs[s + 1])):
+            rows.append((s, t))
+        if len(rows) >= max_rows:
+            break
+    seqs = sorted({s for s, _ in rows})
+    only = np.array([(t, h) for _, t in rows for h in range(w.num_q_heads)], dtype=np.int32)
+    keys = sum(int(w.context_lens[s]) for s in seqs)
+    from paged_kv_cache_445_b200 import roofline
+    return oracle, only, seqs, roofline.kv_cache_bytes(1, w.num_kv_heads, w.head_dim, keys)
+
+
+def oracle_step(oracle, w, only, kc, vc):
+    slots = oracle.slot_mapping(w.block_tables, w.context_lens, w.query_start, w.block_size, w.num_blocks)
+    oracle.cache_append(w.k_new, w.v_new, kc, vc, slots)
+    oracle.paged_attention(w.q, kc, vc, w.block_tables, w.context_lens, w.query_start, w.scale, only=only)
+
+
+def oracle_baseline(w, seconds: float, max_rows: int = 16):
+    oracle, only, seqs, sample_bytes = oracle_sample(w, max_rows)
+    kc, vc = w.k_cache, w.v_cache  # appended in place: the same rows every step
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(oracle, w, only, kc, vc)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = (time.perf_counter() - t0) / n
+    return {"value": round(sample_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{len(seqs)} sequences x {w.num_q_heads} heads of the same workload (append of all "
+                      f"{len(w.slot_mapping)} rows + attention of the sampled rows), {n} steps in {n * dt:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: rank 0 only, on host cores.  Each step
+    is a bounded sample (the first query rows of the batch, all heads, sized so
+    that warm-up plus timed steps take about --reference-seconds)."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    from paged_kv_cache_445_b200 import roofline, workloads
+    import oracle
+    w = workloads.standard(args.workload)
+    kc, vc = w.k_cache, w.v_cache
+    # calibrate: seconds per (row, head) item on the first sequence
+    probe = np.array([(int(w.query_start[0]), h) for h in range(w.num_q_heads)], dtype=np.int32)
+    t0 = time.perf_counter()
+    oracle_step(oracle, w, probe, kc, vc)
+    per_item = max((time.perf_counter() - t0) / len(probe), 1e-6)
+    budget = args.reference_seconds / (args.steps + args.warmup)
+    n_items = int(max(1, min(len(probe), budget / per_item)))
+    only = probe[:n_items]
+    kv_heads = sorted({int(h) // (w.num_q_heads // w.num_kv_heads) for _, h in only})
+    sample_bytes = roofline.kv_cache_bytes(1, len(kv_heads), w.head_dim, int(w.context_lens[0]))
+    for _ in range(args.warmup):
+        oracle_step(oracle, w, only, kc, vc)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(oracle, w, only, kc, vc)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = round(sample_bytes / dt / 1e9, 6)
+    sample = (f"sequence 0 ({int(w.context_lens[0])} keys), {n_items} of {w.num_q_heads} query heads "
+              f"({len(kv_heads)} KV heads), plus the append of all {len(w.slot_mapping)} new rows, per step")
+    line = {
+        "impl": "reference",
+        "metric": "paged-attn decode KV GB/s + seq-steps/s (70B layer, bs128); % of HBM peak",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded PCG64)",
+        "config": {"workload": w.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": oracle.num_threads(),
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    from paged_kv_cache_445_b200.csrc import build as pabuild
+    pabuild.build()
+    run_ours(args, measured_peaks())
+
+
+if __name__ == "__main__":
+    main()
