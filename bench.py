@@ -213,7 +213,8 @@ class GpuStep:
         self.block_tables, self.context_lens = i32(w.block_tables), i32(w.context_lens)
         self.query_start, self.slot_mapping = i32(w.query_start), i32(w.slot_mapping)
         self.out = torch.empty_like(self.q)
-        self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim, device)
+        self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                           w.block_tables.shape[1], w.block_size, device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.decode = w.is_decode
 

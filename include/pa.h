@@ -90,16 +90,19 @@ PA_API int pa_cache_append(const void* k_new, const void* v_new, void* k_cache, 
 
 /*
  * pa_workspace_bytes -- bytes of device workspace pa_decode / pa_prefill_chunk
- * need for a batch with at most `num_query_tokens` query rows, on the CURRENT
- * device (the figure depends on its SM count).  Returns 0 for invalid sizes.
+ * need for a batch with at most `num_query_tokens` query rows whose block
+ * tables are `max_blocks_per_seq` wide, on the CURRENT device (the figure
+ * depends on its SM count).  Returns 0 for invalid sizes.
  *
- * Workspace contract: the caller allocates it, ZERO-FILLS it once before its
- * first use, and may then reuse it for any later call on the same stream;
- * every call that returns PA_OK and whose dev_status stays clear leaves it
- * zero-filled again.  Calls that overlap in time must use different
- * workspaces.  After a call that reported a device error, zero it again.
+ * Workspace contract: the caller allocates it and ZERO-FILLS it once before
+ * its first use; it may then reuse it for any later call on the same stream.
+ * The library keeps its counters in it and every call that returns PA_OK and
+ * whose dev_status stays clear puts them back to zero; the rest is scratch.
+ * Calls that overlap in time must use different workspaces.  After a call
+ * that reported a device error, zero it again.
  */
-PA_API size_t pa_workspace_bytes(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim);
+PA_API size_t pa_workspace_bytes(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int max_blocks_per_seq, int block_size);
 
 /*
  * pa_decode -- one decode step: each sequence has exactly one query row (the

@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(library_path)
 _vp, _ci, _i32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
 _lib.pa_cache_append.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _ci, _ci, _ci, _ci, _vp, _vp]
 _lib.pa_cache_append.restype = _ci
-_lib.pa_workspace_bytes.argtypes = [_ci, _ci, _ci, _ci]
+_lib.pa_workspace_bytes.argtypes = [_ci, _ci, _ci, _ci, _ci, _ci]
 _lib.pa_workspace_bytes.restype = ctypes.c_size_t
 _lib.pa_decode.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci, ctypes.c_float,
                            _vp, ctypes.c_size_t, _vp, _vp]
@@ -100,17 +100,19 @@ def pa_cache_append(k_new, v_new, k_cache, v_cache, slot_mapping, dev_status=Non
                                 _stream_ptr(stream)))
 
 
-def pa_workspace_bytes(num_query_tokens: int, num_q_heads: int, num_kv_heads: int, head_dim: int) -> int:
-    n = int(_lib.pa_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim))
+def pa_workspace_bytes(num_query_tokens: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                       max_blocks_per_seq: int, block_size: int) -> int:
+    n = int(_lib.pa_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                                    block_size))
     if n == 0:
         raise PAError(PA_ERR_UNSUPPORTED)
     return n
 
 
 def make_workspace(num_query_tokens: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                   device=None) -> torch.Tensor:
+                   max_blocks_per_seq: int, block_size: int, device=None) -> torch.Tensor:
     """A zero-filled workspace of pa_workspace_bytes() bytes (the zero fill is required once)."""
-    n = pa_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim)
+    n = pa_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size)
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 

@@ -32,12 +32,7 @@ constexpr int MAX_DEVICES = 64;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 
-// Workspace: [arrival counters: Tq * Hkv int32][rows-kernel partial slots]
-size_t counters_bytes(int num_query_tokens, int num_kv_heads) {
-  return round256(static_cast<size_t>(num_query_tokens) * num_kv_heads * sizeof(int32_t));
-}
 
 }  // namespace
 
@@ -83,9 +78,9 @@ static int check_attention_shape(int num_seqs, int num_q_heads, int num_kv_heads
   return PA_OK;
 }
 
-static size_t workspace_needed(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim, int num_sms) {
-  return counters_bytes(num_query_tokens, num_kv_heads) +
-         round256(rows_partials_bytes(num_q_heads, num_kv_heads, head_dim, num_sms));
+static size_t workspace_needed(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim,
+                               long long max_keys, int num_sms) {
+  return rows_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, num_sms);
 }
 
 static int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache,
@@ -101,14 +96,14 @@ static int run_attention(void* out, const void* q, const int32_t* query_start, c
   if (num_seqs == 0 || total_q_tokens == 0) return PA_OK;
   DeviceInfo di;
   if ((rc = device_info(&di)) != PA_OK) return rc;
-  if (workspace_bytes < workspace_needed(total_q_tokens, num_q_heads, num_kv_heads, head_dim, di.num_sms))
+  const long long max_keys = static_cast<long long>(max_blocks) * block_size;
+  if (workspace_bytes < workspace_needed(total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms))
     return PA_ERR_WORKSPACE;
 
   CUtensorMap tmk, tmv;
   if ((rc = encode_kv_tmap(&tmk, k_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
   if ((rc = encode_kv_tmap(&tmv, v_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
 
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
   RowsParams p{};
   p.out = out;
   p.q = q;
@@ -124,8 +119,7 @@ static int run_attention(void* out, const void* q, const int32_t* query_start, c
   p.num_blocks = num_blocks;
   p.skip_multi = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.counters = reinterpret_cast<int*>(ws);
-  p.partials = reinterpret_cast<float*>(ws + counters_bytes(total_q_tokens, num_kv_heads));
+  rows_workspace_layout(workspace, total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms, &p);
   p.status = dev_status;
   return launch_rows(p, tmk, tmv, head_dim, static_cast<cudaStream_t>(stream), di.num_sms);
 }
@@ -151,12 +145,15 @@ int pa_cache_append(const void* k_new, const void* v_new, void* k_cache, void* v
                            head_dim, block_size, dev_status, static_cast<cudaStream_t>(stream), di.num_sms);
 }
 
-size_t pa_workspace_bytes(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim) {
+size_t pa_workspace_bytes(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim,
+                          int max_blocks_per_seq, int block_size) {
   if (num_query_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads) return 0;
+  if (max_blocks_per_seq <= 0 || (block_size != 16 && block_size != 32)) return 0;
   if (!pa::rows_supported(num_q_heads / num_kv_heads, head_dim)) return 0;
   pa::DeviceInfo di;
   if (pa::device_info(&di) != PA_OK) return 0;
-  return pa::workspace_needed(num_query_tokens, num_q_heads, num_kv_heads, head_dim, di.num_sms);
+  return pa::workspace_needed(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
+                              static_cast<long long>(max_blocks_per_seq) * block_size, di.num_sms);
 }
 
 int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,

@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(256) append_kernel(const uint4* __restrict__ k
                                                      const int32_t* __restrict__ slot_mapping, int num_tokens,
                                                      int num_kv_heads, int vec_per_row, int block_size,
                                                      long long num_slots, int* status) {
+  grid_launch_dependents();  // the attention kernel after this one may start its prologue now
   const long long per_token = static_cast<long long>(num_kv_heads) * vec_per_row;
   const long long total = per_token * num_tokens;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
@@ -47,6 +48,15 @@ int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_c
   const int vec_per_row = head_dim / 8;
   const long long total = static_cast<long long>(num_tokens) * num_kv_heads * vec_per_row;
   if (total == 0) return PA_OK;
+  // Ask for the same L1/shared split as the attention kernels that follow,
+  // so that the SMs need no reconfiguration between the two launches.
+  static int carveout_dev = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && carveout_dev != dev) {
+    cudaFuncSetAttribute(append_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    carveout_dev = dev;
+  }
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
   const long long cap = static_cast<long long>(num_sms) * 8;

@@ -10,6 +10,10 @@
 
 namespace pa {
 
+// Batch size up to which the rows kernel keeps per-sequence prefix sums of
+// tile counts in shared memory (larger batches scan context_lens instead).
+constexpr int ROWS_SMEM_SEQS_HOST = 1024;
+
 // Parameters of the single-row attention kernel (decode rows, and the rows of
 // any sequence the chunk kernel does not take).
 struct RowsParams {
@@ -27,8 +31,12 @@ struct RowsParams {
   int num_blocks;
   int skip_multi;   // 1: sequences with more than one query row belong to the chunk kernel
   float scale_log2; // softmax scale * log2(e)
-  float* partials;  // workspace: two partial-result slots per warp
-  int* counters;    // workspace: one arrival counter per (query row, KV head), zero between calls
+  float* partials;             // workspace: partial-result slots, two per warp
+  long long* seginfo;          // workspace: (tiles << 40 | first unit + 1) of segments with partials, zero between calls
+  long long* table;            // workspace: (tiles << 32 | slot) of the piece that starts at each unit
+  long long table_len;         // entries in table
+  int* sched;                  // workspace: [warps at the barrier, warps done], zero between calls
+  int num_rows;                // query rows (Tq)
   int* status;      // optional device status word
   int total_warps;
 };
@@ -47,8 +55,13 @@ int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_c
                   cudaStream_t stream, int num_sms);
 int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
                 cudaStream_t stream, int num_sms);
-// Upper bound of the rows kernel's workspace for this shape on a device with num_sms SMs.
-size_t rows_partials_bytes(int num_q_heads, int num_kv_heads, int head_dim, int num_sms);
+// Workspace of the rows kernel for at most num_rows query rows on a device with
+// num_sms SMs, and the carving of a buffer of that size into RowsParams.
+// max_keys bounds the keys of any row (max_blocks_per_seq * block_size).
+size_t rows_workspace_bytes(int num_rows, int num_q_heads, int num_kv_heads, int head_dim, long long max_keys,
+                            int num_sms);
+void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_heads, int head_dim,
+                           long long max_keys, int num_sms, RowsParams* p);
 int rows_supported(int group, int head_dim);
 
 }  // namespace pa

@@ -39,6 +39,8 @@ namespace pa {
 constexpr int TILE_KEYS = 16;
 constexpr int ROWS_WARPS = 4;
 constexpr int ROWS_THREADS = ROWS_WARPS * 32;
+constexpr int ROWS_SLOTS_PER_WARP = 2;  // a warp's range cuts at most its first and its last segment
+constexpr int ROWS_SMEM_SEQS = ROWS_SMEM_SEQS_HOST;  // sequences whose tile prefix sums live in shared memory
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -137,24 +139,26 @@ __device__ __forceinline__ void advance(const RowsParams& p, Cursor& c) {
   c.s = p.num_seqs;
 }
 
-// Warp-uniform window of 32 block-table entries of one sequence.
+// Warp-uniform window of 128 block-table entries of one sequence (4 per lane).
 struct BtWindow {
-  int s, lo, reg;
+  int s, lo;
+  int r[4];
 };
 
 __device__ __forceinline__ int bt_lookup(const RowsParams& p, BtWindow& w, int s, int lb, int lane) {
-  if (s != w.s || lb < w.lo || lb >= w.lo + 32) {
+  if (s != w.s || lb < w.lo || lb >= w.lo + 128) {
     w.s = s;
     w.lo = lb;
-    const int idx = lb + lane;
-    w.reg = idx < p.max_blocks ? __ldg(p.block_tables + static_cast<long long>(s) * p.max_blocks + idx) : -1;
+    const int32_t* row = p.block_tables + static_cast<long long>(s) * p.max_blocks;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int idx = lb + 32 * k + lane;
+      w.r[k] = idx < p.max_blocks ? __ldg(row + idx) : -1;
+    }
   }
-  return __shfl_sync(FULL_MASK, w.reg, lb - w.lo);
-}
-
-// First warp whose range [T*w/W, T*(w+1)/W) contains unit u.
-__device__ __forceinline__ int owner_warp(long long u, long long T, long long W) {
-  return static_cast<int>(((u + 1) * W + T - 1) / T - 1);
+  const int e = lb - w.lo, k = e >> 5;
+  const int v = k == 0 ? w.r[0] : k == 1 ? w.r[1] : k == 2 ? w.r[2] : w.r[3];
+  return __shfl_sync(FULL_MASK, v, e & 31);
 }
 
 __device__ __forceinline__ long long range_start(long long w, long long T, long long W) { return T * w / W; }
@@ -166,7 +170,10 @@ struct RowsShape {
   static constexpr int HALF_BYTES = TILE_KEYS * D * 2; // K (or V) bytes of a tile
   static constexpr int STAGE_BYTES = 2 * HALF_BYTES;
   static constexpr int SLOT_O = KT * NT * 32 * 4;      // O^T fragment floats of a partial
-  static constexpr int SLOT_FLOATS = ((SLOT_O + 2 * NT * 8) + 63) / 64 * 64;
+  static constexpr int SLOT_M = SLOT_O;                // running maxima (8 NT floats)
+  static constexpr int SLOT_L = SLOT_O + 8 * NT;       // sums (8 NT floats)
+  static constexpr int SLOT_NEXT = SLOT_O + 16 * NT;   // next slot of the segment + 1 (int), 0 = end
+  static constexpr int SLOT_FLOATS = (SLOT_NEXT + 1 + 63) / 64 * 64;
 };
 
 // Write normalised O for one segment: O^T fragments -> bf16 -> movmatrix -> rows of out.
@@ -199,44 +206,26 @@ __device__ __forceinline__ void zero_rows(const RowsParams& p, int q0, int nrows
   for (long long k = 0; k < n; ++k) o[k] = make_uint4(0, 0, 0, 0);
 }
 
-template <int D, int NT, int R>
-__global__ void __launch_bounds__(ROWS_THREADS, 1)
-    rows_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                const RowsParams p) {
-  using S = RowsShape<D, NT>;
-  constexpr int KT = S::KT;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[ROWS_WARPS][R];
-
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int gw = blockIdx.x * ROWS_WARPS + warp;
-  const int g = lane >> 2, c = lane & 3;
-
-  // ---- pass 1: total tile count; rows without a key are written as zeros
-  long long T = 0;
-  for (int base = 0; base < p.num_seqs; base += 32) {
-    const int s = base + lane;
-    long long u = 0;
-    if (s < p.num_seqs) {
-      const SeqInfo si = seq_info(p, s);
-      u = seq_units(p, si);
-      const int nzero = min(si.qlen, max(0, si.qlen - si.ctx));
-      if (nzero > 0 && (s % p.total_warps) == gw) zero_rows(p, si.q0, nzero, D);
+// Position a cursor on global unit a (a < T).  The sequence comes from the
+// shared-memory prefix of per-sequence tile counts when there is one (binary
+// search), else from a scan of context_lens; the row from a binary search
+// over the closed-form tile counts of its rows.
+__device__ __forceinline__ void seek(const RowsParams& p, const long long* pfx, long long a, int lane, Cursor& cc) {
+  int s_found = -1;
+  long long seq_base = 0;
+  if (pfx) {
+    int lo = 0, hi = p.num_seqs;  // first k with pfx[k] > a, minus one
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (pfx[mid + 1] > a)
+        hi = mid;
+      else
+        lo = mid + 1;
     }
-    T += warp_sum64(u);
-  }
-  if (T == 0) return;
-  const long long W = T < p.total_warps ? T : p.total_warps;
-  if (gw >= W) return;
-  const long long a = range_start(gw, T, W), e = range_start(gw + 1, T, W);
-  const long long count = e - a;
-
-  // ---- pass 2: the segment that holds unit a
-  Cursor cc;
-  {
+    s_found = lo;
+    seq_base = pfx[lo];
+  } else {
     long long acc = 0;
-    int s_found = -1;
-    long long seq_base = 0;
     for (int base = 0; base < p.num_seqs && s_found < 0; base += 32) {
       const int s = base + lane;
       long long u = 0;
@@ -251,283 +240,461 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       }
       acc += chunk;
     }
-    const SeqInfo si = seq_info(p, s_found);
-    cc.s = s_found;
-    cc.qlen = si.qlen;
-    cc.q0 = si.q0;
-    cc.p0 = si.ctx - si.qlen;
-    const int i0 = cc.p0 < 0 ? -cc.p0 : 0;
-    const long long o = a - seq_base;
-    const long long base_tiles = tiles_upto(cc.p0 + i0);
-    int lo = i0, hi = si.qlen - 1;
-    while (lo < hi) {  // last row whose first unit is <= o
-      const int mid = (lo + hi + 1) >> 1;
-      if (static_cast<long long>(p.num_kv_heads) * (tiles_upto(cc.p0 + mid) - base_tiles) <= o)
-        lo = mid;
-      else
-        hi = mid - 1;
-    }
-    cc.i = lo;
-    cc.nkeys = cc.p0 + lo + 1;
-    cc.n = ceil16(cc.nkeys);
-    const long long rem = o - static_cast<long long>(p.num_kv_heads) * (tiles_upto(cc.p0 + lo) - base_tiles);
-    cc.h = static_cast<int>(rem / cc.n);
-    cc.t = static_cast<int>(rem % cc.n);
-    cc.u = a;
   }
-
-  // ---- per-warp TMA ring
-  uint8_t* ring = align1024(smem_raw) + static_cast<size_t>(warp) * R * S::STAGE_BYTES;
-  uint64_t* bar = bars[warp];
-  if (lane == 0) {
-    prefetch_tmap(&tmk);
-    prefetch_tmap(&tmv);
-#pragma unroll
-    for (int k = 0; k < R; ++k) mbar_init(&bar[k], 1);
-    fence_mbar_init();
+  const SeqInfo si = seq_info(p, s_found);
+  cc.s = s_found;
+  cc.qlen = si.qlen;
+  cc.q0 = si.q0;
+  cc.p0 = si.ctx - si.qlen;
+  const int i0 = cc.p0 < 0 ? -cc.p0 : 0;
+  const long long o = a - seq_base;
+  const long long base_tiles = tiles_upto(cc.p0 + i0);
+  int lo = i0, hi = si.qlen - 1;
+  while (lo < hi) {  // last row whose first unit is <= o
+    const int mid = (lo + hi + 1) >> 1;
+    if (static_cast<long long>(p.num_kv_heads) * (tiles_upto(cc.p0 + mid) - base_tiles) <= o)
+      lo = mid;
+    else
+      hi = mid - 1;
   }
-  __syncwarp();
-  const uint64_t pol = policy_evict_first();
+  cc.i = lo;
+  cc.nkeys = cc.p0 + lo + 1;
+  cc.n = ceil16(cc.nkeys);
+  const long long rem = o - static_cast<long long>(p.num_kv_heads) * (tiles_upto(cc.p0 + lo) - base_tiles);
+  cc.h = static_cast<int>(rem / cc.n);
+  cc.t = static_cast<int>(rem % cc.n);
+  cc.u = a;
+}
 
-  Cursor lc = cc;
-  BtWindow win{-1, 0, -1};
-  auto issue = [&](int stage) {
-    const int key0 = lc.t * TILE_KEYS;
-    const int lb = key0 / p.block_size, y = key0 - lb * p.block_size;
-    const int blk = bt_lookup(p, win, lc.s, lb, lane);
-    if (lane == 0) {
-      if (blk < 0 || blk >= p.num_blocks) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
-      uint8_t* st = ring + stage * S::STAGE_BYTES;
-      mbar_arrive_expect_tx(&bar[stage], S::STAGE_BYTES);
+// Merge the partial (m, l, O) results of the pieces of segment [segA, segA + n)
+// and write the normalised output row.  Piece k recorded (slot, tiles) at the
+// table entry of its first unit, so the walk visits the pieces in order; one
+// pass with a running maximum.
+template <int D, int NT>
+__device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, int n, int row, int kvh, int lane) {
+  using S = RowsShape<D, NT>;
+  constexpr int KT = S::KT;
+  const int c = lane & 3;
+  float mm[NT][2], acc[KT][NT][4], ll[NT][2];
 #pragma unroll
-      for (int pc = 0; pc < S::PIECES; ++pc) {
-        tma_load_4d(st + pc * 2048, &tmk, &bar[stage], pc * 64, y, lc.h, blk, pol);
-        tma_load_4d(st + S::HALF_BYTES + pc * 2048, &tmv, &bar[stage], pc * 64, y, lc.h, blk, pol);
-      }
-    }
-    advance(p, lc);
-  };
-
-  long long issued = 0;
-  for (; issued < R && issued < count; ++issued) issue(static_cast<int>(issued));
-
-  float o[KT][NT][4];
-  uint32_t qb[NT][KT][2];
-  float m[NT][2], l[NT][2];
-  bool began = false;
-  long long piece_j0 = 0;
-  long long stopped_at = -1;
-
-  for (long long j = 0; j < count; ++j) {
-    const int stage = static_cast<int>(j % R);
-    const uint32_t phase = static_cast<uint32_t>((j / R) & 1);
-
-    if (j == 0 || cc.t == 0) {  // a piece starts: load the G query rows of this KV head
-      began = (cc.t == 0);
-      piece_j0 = j;
-      const int row = cc.q0 + cc.i;
+  for (int nt = 0; nt < NT; ++nt) {
+    mm[nt][0] = mm[nt][1] = -INFINITY;
+    ll[nt][0] = ll[nt][1] = 0.f;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int head = nt * 8 + g;
-        const bool ok = head < p.group;
-        const uint32_t* qp = reinterpret_cast<const uint32_t*>(
-            static_cast<const __nv_bfloat16*>(p.q) +
-            (static_cast<long long>(row) * p.num_q_heads + cc.h * p.group + (ok ? head : 0)) * D);
-#pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-          qb[nt][kk][0] = ok ? __ldg(qp + 8 * kk + c) : 0u;
-          qb[nt][kk][1] = ok ? __ldg(qp + 8 * kk + 4 + c) : 0u;
-        }
-        m[nt][0] = m[nt][1] = -INFINITY;
-        l[nt][0] = l[nt][1] = 0.f;
-#pragma unroll
-        for (int mt = 0; mt < KT; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
-      }
-    }
-
-    if (!mbar_wait(&bar[stage], phase)) {
-      set_status(p.status, PA_STATUS_BIT(PA_ERR_TIMEOUT));
-      stopped_at = j;
+    for (int mt = 0; mt < KT; ++mt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+  }
+  for (int t = 0; t < n;) {
+    const long long e = __ldcg(p.table + segA + t);
+    const int slot = static_cast<int>(e & 0xffffffffll), tiles = static_cast<int>(e >> 32);
+    if (tiles <= 0 || slot < 0) {  // cannot happen when every piece recorded itself
+      set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
       break;
     }
-    uint8_t* kt = ring + stage * S::STAGE_BYTES;
-    uint8_t* vt = kt + S::HALF_BYTES;
-    const int nvalid = min(TILE_KEYS, cc.nkeys - cc.t * TILE_KEYS);
-    if (nvalid < TILE_KEYS) {  // rows past the context may hold anything: zero V there
-      const int nz = (TILE_KEYS - nvalid) * S::PIECES * 8;
-      for (int k = lane; k < nz; k += 32) {
-        const int r = nvalid + k / (S::PIECES * 8);
-        const int rest = k % (S::PIECES * 8);
-        *reinterpret_cast<uint4*>(vt + (rest >> 3) * 2048 + r * 128 + (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
-      }
-      __syncwarp();
-    }
-
-    // S^T[key, head] = K . Q^T
-    float sacc[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-    {
-      const int mi = lane >> 3;
-      const int r = (lane & 7) + (mi & 1) * 8;
-      const uint32_t kbase = smem_u32(kt);
-#pragma unroll
-      for (int kk = 0; kk < KT; ++kk) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(kbase + (kk >> 2) * 2048 + sw128(r, 2 * (kk & 3) + (mi >> 1)), a0, a1, a2, a3);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sacc[nt], a0, a1, a2, a3, qb[nt][kk][0], qb[nt][kk][1]);
-      }
-    }
-
-    // online softmax on the fragment: this lane holds keys g, g+8 of heads 2c, 2c+1
-    uint32_t pb[NT][2];
+    t += tiles;
+    const float* pk = p.partials + static_cast<long long>(slot) * S::SLOT_FLOATS;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      float s0 = sacc[nt][0] * p.scale_log2, s1 = sacc[nt][1] * p.scale_log2;
-      float s2 = sacc[nt][2] * p.scale_log2, s3 = sacc[nt][3] * p.scale_log2;
-      if (g >= nvalid) s0 = s1 = -INFINITY;
-      if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
-      float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+      float f[2], gk[2];
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
+      for (int e2 = 0; e2 < 2; ++e2) {
+        const float mk = __ldcg(pk + S::SLOT_M + nt * 8 + 2 * c + e2);
+        const float mn = fmaxf(mm[nt][e2], mk);
+        f[e2] = fast_exp2(mm[nt][e2] - mn);  // rescales what was merged so far
+        gk[e2] = fast_exp2(mk - mn);         // weight of this piece
+        mm[nt][e2] = mn;
+        ll[nt][e2] = ll[nt][e2] * f[e2] + gk[e2] * __ldcg(pk + S::SLOT_L + nt * 8 + 2 * c + e2);
       }
-      const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
-      const float al0 = fast_exp2(m[nt][0] - mn0), al1 = fast_exp2(m[nt][1] - mn1);
-      m[nt][0] = mn0;
-      m[nt][1] = mn1;
-      const float p0 = fast_exp2(s0 - mn0), p2 = fast_exp2(s2 - mn0);
-      const float p1 = fast_exp2(s1 - mn1), p3 = fast_exp2(s3 - mn1);
-      l[nt][0] = l[nt][0] * al0 + p0 + p2;
-      l[nt][1] = l[nt][1] * al1 + p1 + p3;
 #pragma unroll
       for (int mt = 0; mt < KT; ++mt) {
-        o[mt][nt][0] *= al0;
-        o[mt][nt][1] *= al1;
-        o[mt][nt][2] *= al0;
-        o[mt][nt][3] *= al1;
-      }
-      pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
-      pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
-    }
-
-    // O^T[d, head] += V^T . P^T
-    {
-      const int mi = lane >> 3;
-      const int r = (lane & 7) + (mi >> 1) * 8;
-      const uint32_t vbase = smem_u32(vt);
-#pragma unroll
-      for (int mt = 0; mt < KT; ++mt) {
-        const int cg = 2 * mt + (mi & 1);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_trans(vbase + (cg >> 3) * 2048 + sw128(r, cg & 7), a0, a1, a2, a3);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[mt][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(pk) + (mt * NT + nt) * 32 + lane);
+        acc[mt][nt][0] = acc[mt][nt][0] * f[0] + gk[0] * v.x;
+        acc[mt][nt][1] = acc[mt][nt][1] * f[1] + gk[1] * v.y;
+        acc[mt][nt][2] = acc[mt][nt][2] * f[0] + gk[0] * v.z;
+        acc[mt][nt][3] = acc[mt][nt][3] * f[1] + gk[1] * v.w;
       }
     }
+  }
+  store_output<D, NT>(p, acc, ll, row, kvh, lane);
+}
 
-    // refill this stage
-    __syncwarp();
-    if (issued < count) {
-      if (lane == 0) fence_proxy_async_smem();
-      issue(stage);
-      ++issued;
-    }
+// What the consumer needs to know about the tile in a ring stage; written by
+// the issuing lane before the TMA, read by the warp after the stage completes.
+struct TileMeta {
+  long long u;  // global unit index
+  int row, h, t, n, nkeys;
+  int flags;  // bit 0: first tile of this warp's range, bit 1: last tile of it
+};
 
-    // ---- end of a piece: write the output or a partial
-    if (j == count - 1 || cc.t == cc.n - 1) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-          float v = l[nt][q2];
-          v += __shfl_xor_sync(FULL_MASK, v, 4);
-          v += __shfl_xor_sync(FULL_MASK, v, 8);
-          v += __shfl_xor_sync(FULL_MASK, v, 16);
-          l[nt][q2] = v;
-        }
-      const int row = cc.q0 + cc.i;
-      if (began && cc.t == cc.n - 1) {
-        store_output<D, NT>(p, o, l, row, cc.h, lane);
-      } else {
-        const int slot = 2 * gw + (piece_j0 == 0 ? 0 : 1);
-        float* ps = p.partials + static_cast<long long>(slot) * S::SLOT_FLOATS;
-#pragma unroll
-        for (int mt = 0; mt < KT; ++mt)
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            reinterpret_cast<float4*>(ps)[(mt * NT + nt) * 32 + lane] =
-                make_float4(o[mt][nt][0], o[mt][nt][1], o[mt][nt][2], o[mt][nt][3]);
-        if (lane < 4) {
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            ps[S::SLOT_O + nt * 8 + 2 * lane] = m[nt][0];
-            ps[S::SLOT_O + nt * 8 + 2 * lane + 1] = m[nt][1];
-            ps[S::SLOT_O + NT * 8 + nt * 8 + 2 * lane] = l[nt][0];
-            ps[S::SLOT_O + NT * 8 + nt * 8 + 2 * lane + 1] = l[nt][1];
-          }
-        }
-        __threadfence();
-        __syncwarp();
-        const long long segA = cc.u - cc.t, segB = segA + cc.n;
-        const int w0 = owner_warp(segA, T, W), w1 = owner_warp(segB - 1, T, W);
-        const int npieces = w1 - w0 + 1;
-        int* counter = p.counters + static_cast<long long>(row) * p.num_kv_heads + cc.h;
-        int old = 0;
-        if (lane == 0) old = atomicAdd(counter, 1);
-        old = __shfl_sync(FULL_MASK, old, 0);
-        if (old == npieces - 1) {  // last arrival merges every piece of the segment
-          __threadfence();
-          float mm[NT][2], acc[KT][NT][4], ll[NT][2];
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mm[nt][0] = mm[nt][1] = -INFINITY;
-            ll[nt][0] = ll[nt][1] = 0.f;
-#pragma unroll
-            for (int mt = 0; mt < KT; ++mt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
-          }
-          for (int k = 0; k < npieces; ++k) {
-            const int wk = w0 + k;
-            const int sk = 2 * wk + ((k == 0 && range_start(wk, T, W) < segA) ? 1 : 0);
-            const float* pk = p.partials + static_cast<long long>(sk) * S::SLOT_FLOATS;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              mm[nt][0] = fmaxf(mm[nt][0], __ldcg(pk + S::SLOT_O + nt * 8 + 2 * c));
-              mm[nt][1] = fmaxf(mm[nt][1], __ldcg(pk + S::SLOT_O + nt * 8 + 2 * c + 1));
-            }
-          }
-          for (int k = 0; k < npieces; ++k) {
-            const int wk = w0 + k;
-            const int sk = 2 * wk + ((k == 0 && range_start(wk, T, W) < segA) ? 1 : 0);
-            const float* pk = p.partials + static_cast<long long>(sk) * S::SLOT_FLOATS;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const float f0 = fast_exp2(__ldcg(pk + S::SLOT_O + nt * 8 + 2 * c) - mm[nt][0]);
-              const float f1 = fast_exp2(__ldcg(pk + S::SLOT_O + nt * 8 + 2 * c + 1) - mm[nt][1]);
-              ll[nt][0] += f0 * __ldcg(pk + S::SLOT_O + NT * 8 + nt * 8 + 2 * c);
-              ll[nt][1] += f1 * __ldcg(pk + S::SLOT_O + NT * 8 + nt * 8 + 2 * c + 1);
-#pragma unroll
-              for (int mt = 0; mt < KT; ++mt) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(pk) + (mt * NT + nt) * 32 + lane);
-                acc[mt][nt][0] += f0 * v.x;
-                acc[mt][nt][1] += f1 * v.y;
-                acc[mt][nt][2] += f0 * v.z;
-                acc[mt][nt][3] += f1 * v.w;
-              }
-            }
-          }
-          store_output<D, NT>(p, acc, ll, row, cc.h, lane);
-          if (lane == 0) *counter = 0;  // leave the workspace zeroed for the next call
-        }
+template <int D, int NT, int R>
+__global__ void __launch_bounds__(ROWS_THREADS, 1)
+    rows_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                const RowsParams p) {
+  using S = RowsShape<D, NT>;
+  constexpr int KT = S::KT;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[ROWS_WARPS][R];
+  __shared__ TileMeta metas[ROWS_WARPS][R];
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gw = blockIdx.x * ROWS_WARPS + warp;
+  const int g = lane >> 2, c = lane & 3;
+  uint8_t* base = align1024(smem_raw);
+  const bool use_pfx = p.num_seqs <= ROWS_SMEM_SEQS;
+  long long* pfx = use_pfx ? reinterpret_cast<long long*>(base + ROWS_WARPS * R * S::STAGE_BYTES) : nullptr;
+
+  // ---- prologue: tiles of every sequence, their prefix sums, the total T.
+  // Rows without a key are written as zeros here (each by one thread).
+  long long T = 0;
+  if (use_pfx) {
+    for (int s = threadIdx.x; s < p.num_seqs; s += ROWS_THREADS) pfx[s + 1] = seq_units(p, seq_info(p, s));
+    if (threadIdx.x == 0) pfx[0] = 0;
+    __syncthreads();
+    if (warp == 0) {
+      long long carry = 0;
+      for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
+        const int s = b0 + lane;
+        const long long v = s < p.num_seqs ? pfx[s + 1] : 0;
+        const long long incl = warp_incl_scan64(v, lane);
+        if (s < p.num_seqs) pfx[s + 1] = carry + incl;
+        carry += __shfl_sync(FULL_MASK, incl, 31);
       }
     }
-    advance(p, cc);
+    __syncthreads();
+    T = pfx[p.num_seqs];
+  } else {
+    for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
+      const int s = b0 + lane;
+      T += warp_sum64(s < p.num_seqs ? seq_units(p, seq_info(p, s)) : 0);
+    }
   }
 
-  if (stopped_at >= 0) {  // let copies still in flight land before the shared memory goes away
-    for (long long j = stopped_at + 1; j < issued; ++j) mbar_wait(&bar[j % R], static_cast<uint32_t>((j / R) & 1));
+  // Everything above reads only the batch metadata.  From here on the kernel
+  // reads the cache (which the append kernel before it may still be writing)
+  // and writes out: wait for the grids this launch depends on.
+  grid_dependency_wait();
+  for (int s = blockIdx.x * ROWS_THREADS + threadIdx.x; s < p.num_seqs; s += gridDim.x * ROWS_THREADS) {
+    const SeqInfo si = seq_info(p, s);  // rows without a key are written as zeros
+    const int nzero = min(si.qlen, max(0, si.qlen - si.ctx));
+    if (nzero > 0) zero_rows(p, si.q0, nzero, D);
+  }
+  if (T > p.table_len) {  // the host sized the piece table for the largest possible batch
+    set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+    T = 0;
+  }
+
+  const long long W = T < p.total_warps ? T : p.total_warps;
+  uint64_t* bar = bars[warp];
+  TileMeta* meta = metas[warp];
+  uint8_t* ring = base + static_cast<size_t>(warp) * R * S::STAGE_BYTES;
+  long long issued = 0, stopped_at = -1;
+  int nslots = 0;
+
+  if (gw < W) {
+    if (lane == 0) {
+      prefetch_tmap(&tmk);
+      prefetch_tmap(&tmv);
+#pragma unroll
+      for (int k = 0; k < R; ++k) mbar_init(&bar[k], 1);
+      fence_mbar_init();
+    }
+    __syncwarp();
+    const uint64_t pol = policy_evict_first();
+
+    // ---- producer: the load cursor walks the warp's range [a, e)
+    const long long a = range_start(gw, T, W), e = range_start(gw + 1, T, W);
+    Cursor lc;
+    seek(p, pfx, a, lane, lc);
+    bool loading = true;
+    BtWindow win;
+    win.s = -1;
+
+    auto issue = [&](int stage) {
+      const bool first = lc.u == a, last = lc.u == e - 1;
+      const int key0 = lc.t * TILE_KEYS;
+      const int lb = key0 / p.block_size, y = key0 - lb * p.block_size;
+      const int blk = bt_lookup(p, win, lc.s, lb, lane);
+      if (lc.t == 0 || first) {
+        // warm L1 with query rows a segment ahead: the next segment's (row + 1
+        // after the last KV head: rows of consecutive sequences are consecutive),
+        // and at the start of a run the current one as well
+        const long long row = lc.q0 + lc.i;
+        const long long nq = (row + (lc.h + 1 == p.num_kv_heads)) * p.num_q_heads +
+                             ((lc.h + 1) % p.num_kv_heads) * p.group;
+        const long long cq = row * p.num_q_heads + lc.h * p.group;
+        if (nq < static_cast<long long>(p.num_rows) * p.num_q_heads)
+          for (int off = lane * 128; off < p.group * D * 2; off += 32 * 128)
+            prefetch_l1(static_cast<const char*>(p.q) + nq * D * 2 + off);
+        if (first)
+          for (int off = lane * 128; off < p.group * D * 2; off += 32 * 128)
+            prefetch_l1(static_cast<const char*>(p.q) + cq * D * 2 + off);
+      }
+      if (lane == 0) {
+        TileMeta& m = meta[stage];
+        m.u = lc.u;
+        m.row = lc.q0 + lc.i;
+        m.h = lc.h;
+        m.t = lc.t;
+        m.n = lc.n;
+        m.nkeys = lc.nkeys;
+        m.flags = (first ? 1 : 0) | (last ? 2 : 0);
+        if (blk < 0 || blk >= p.num_blocks) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+        uint8_t* st = ring + stage * S::STAGE_BYTES;
+        mbar_arrive_expect_tx(&bar[stage], S::STAGE_BYTES);
+#pragma unroll
+        for (int pc = 0; pc < S::PIECES; ++pc) {
+          tma_load_4d(st + pc * 2048, &tmk, &bar[stage], pc * 64, y, lc.h, blk, pol);
+          tma_load_4d(st + S::HALF_BYTES + pc * 2048, &tmv, &bar[stage], pc * 64, y, lc.h, blk, pol);
+        }
+      }
+      ++issued;
+      if (!last)
+        advance(p, lc);
+      else
+        loading = false;
+    };
+
+    for (int k = 0; k < R && loading; ++k) issue(k);
+
+    float o[KT][NT][4];
+    uint32_t qb[NT][KT][2];
+    float m[NT][2], l[NT][2];
+    bool began = false;
+    int piece_t0 = 0;
+
+    for (long long j = 0; j < issued; ++j) {
+      const int stage = static_cast<int>(j % R);
+      const uint32_t phase = static_cast<uint32_t>((j / R) & 1);
+      if (!mbar_wait(&bar[stage], phase)) {
+        set_status(p.status, PA_STATUS_BIT(PA_ERR_TIMEOUT));
+        stopped_at = j;
+        break;
+      }
+      const TileMeta tm = meta[stage];
+      const bool run_start = tm.flags & 1, run_end = tm.flags & 2;
+
+      if (tm.t == 0 || run_start) {  // a piece starts: load the G query rows of this KV head
+        began = (tm.t == 0);
+        piece_t0 = tm.t;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int head = nt * 8 + g;
+          const bool ok = head < p.group;
+          const uint32_t* qp = reinterpret_cast<const uint32_t*>(
+              static_cast<const __nv_bfloat16*>(p.q) +
+              (static_cast<long long>(tm.row) * p.num_q_heads + tm.h * p.group + (ok ? head : 0)) * D);
+#pragma unroll
+          for (int kk = 0; kk < KT; ++kk) {
+            qb[nt][kk][0] = ok ? __ldg(qp + 8 * kk + c) : 0u;
+            qb[nt][kk][1] = ok ? __ldg(qp + 8 * kk + 4 + c) : 0u;
+          }
+          m[nt][0] = m[nt][1] = -INFINITY;
+          l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+        }
+      }
+
+      uint8_t* kt = ring + stage * S::STAGE_BYTES;
+      uint8_t* vt = kt + S::HALF_BYTES;
+      const int nvalid = min(TILE_KEYS, tm.nkeys - tm.t * TILE_KEYS);
+
+      // Pull the tile into registers (K as the A operand of S^T = K Q^T, V^T via
+      // ldmatrix.trans as the A operand of O^T += V^T P^T) and hand the stage
+      // back to TMA at once, so the ring never waits on the math.  With
+      // head_dim 256 both fragments would not fit in registers: V is read after
+      // the softmax and the stage is released then.
+      constexpr bool kEarly = D <= 128;
+      uint32_t kf[KT][4], vf[KT][4];
+      const int mi = lane >> 3;
+      const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
+      auto load_v = [&]() {
+        const int rv = (lane & 7) + (mi >> 1) * 8;
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt) {
+          const int cg = 2 * mt + (mi & 1);
+          ldsm_x4_trans(vbase + (cg >> 3) * 2048 + sw128(rv, cg & 7), vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3]);
+        }
+        if (nvalid < TILE_KEYS) {
+          // keys past the context may hold anything (even NaN): their V rows must
+          // be exact zeros, since P = 0 times NaN is NaN.  This lane holds keys
+          // 2c, 2c+1 (fragments 0, 1) and 8+2c, 9+2c (fragments 2, 3).
+          const uint32_t lo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+          const uint32_t hi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            vf[mt][0] &= lo;
+            vf[mt][1] &= lo;
+            vf[mt][2] &= hi;
+            vf[mt][3] &= hi;
+          }
+        }
+      };
+      auto release = [&]() {
+        __syncwarp();
+        if (loading) {
+          if (lane == 0) fence_proxy_async_smem();
+          issue(stage);
+        }
+      };
+      {
+        const int rk = (lane & 7) + (mi & 1) * 8;
+#pragma unroll
+        for (int kk = 0; kk < KT; ++kk)
+          ldsm_x4(kbase + (kk >> 2) * 2048 + sw128(rk, 2 * (kk & 3) + (mi >> 1)), kf[kk][0], kf[kk][1], kf[kk][2],
+                  kf[kk][3]);
+      }
+      if constexpr (kEarly) {
+        load_v();
+        release();
+      }
+
+      // S^T[key, head] = K . Q^T
+      float sacc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KT; ++kk)
+          mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
+      }
+
+      // online softmax on the fragment: this lane holds keys g, g+8 of heads 2c, 2c+1
+      uint32_t pb[NT][2];
+      float al[NT][2];
+      bool moved = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        float s0 = sacc[nt][0] * p.scale_log2, s1 = sacc[nt][1] * p.scale_log2;
+        float s2 = sacc[nt][2] * p.scale_log2, s3 = sacc[nt][3] * p.scale_log2;
+        if (g >= nvalid) s0 = s1 = -INFINITY;
+        if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
+        }
+        const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+        moved |= (mn0 != m[nt][0]) | (mn1 != m[nt][1]);
+        al[nt][0] = fast_exp2(m[nt][0] - mn0);
+        al[nt][1] = fast_exp2(m[nt][1] - mn1);
+        m[nt][0] = mn0;
+        m[nt][1] = mn1;
+        const float p0 = fast_exp2(s0 - mn0), p2 = fast_exp2(s2 - mn0);
+        const float p1 = fast_exp2(s1 - mn1), p3 = fast_exp2(s3 - mn1);
+        l[nt][0] = l[nt][0] * al[nt][0] + p0 + p2;
+        l[nt][1] = l[nt][1] * al[nt][1] + p1 + p3;
+        pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+        pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+      }
+      if (__any_sync(FULL_MASK, moved)) {  // rescale O only when some running maximum grew
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            o[mt][nt][0] *= al[nt][0];
+            o[mt][nt][1] *= al[nt][1];
+            o[mt][nt][2] *= al[nt][0];
+            o[mt][nt][3] *= al[nt][1];
+          }
+      }
+
+      // O^T[d, head] += V^T . P^T
+      if constexpr (!kEarly) {
+        load_v();
+        release();
+      }
+#pragma unroll
+      for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_bf16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+
+      // ---- end of a piece: write the output, or a partial linked to its segment
+      if (tm.t == tm.n - 1 || run_end) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            float v = l[nt][q2];
+            v += __shfl_xor_sync(FULL_MASK, v, 4);
+            v += __shfl_xor_sync(FULL_MASK, v, 8);
+            v += __shfl_xor_sync(FULL_MASK, v, 16);
+            l[nt][q2] = v;
+          }
+        if (began && tm.t == tm.n - 1) {
+          store_output<D, NT>(p, o, l, tm.row, tm.h, lane);
+        } else if (nslots < ROWS_SLOTS_PER_WARP) {
+          const long long slot = static_cast<long long>(gw) * ROWS_SLOTS_PER_WARP + nslots++;
+          float* ps = p.partials + slot * S::SLOT_FLOATS;
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              reinterpret_cast<float4*>(ps)[(mt * NT + nt) * 32 + lane] =
+                  make_float4(o[mt][nt][0], o[mt][nt][1], o[mt][nt][2], o[mt][nt][3]);
+          if (lane < 4) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              ps[S::SLOT_M + nt * 8 + 2 * lane] = m[nt][0];
+              ps[S::SLOT_M + nt * 8 + 2 * lane + 1] = m[nt][1];
+              ps[S::SLOT_L + nt * 8 + 2 * lane] = l[nt][0];
+              ps[S::SLOT_L + nt * 8 + 2 * lane + 1] = l[nt][1];
+            }
+          }
+          // record the piece at its first unit and mark its segment; the
+          // segment is merged after the grid barrier (plain stores, no waiting)
+          if (lane == 0) {
+            const long long segA = tm.u - tm.t;
+            p.table[segA + piece_t0] = (static_cast<long long>(tm.t - piece_t0 + 1) << 32) | slot;
+            p.seginfo[static_cast<long long>(tm.row) * p.num_kv_heads + tm.h] =
+                (static_cast<long long>(tm.n) << 40) | (segA + 1);
+          }
+        } else {
+          set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));  // cannot happen: slots cover every run end
+        }
+      }
+    }
+
+    if (stopped_at >= 0) {  // let copies still in flight land before the shared memory goes away
+      for (long long j = stopped_at + 1; j < issued; ++j) mbar_wait(&bar[j % R], static_cast<uint32_t>((j / R) & 1));
+    }
+  }
+
+  // ---- grid barrier: every partial and table entry is stored before any merge reads it
+  __syncwarp();
+  if (lane == 0) {
+    __threadfence();
+    atomicAdd(p.sched, 1);
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu(p.sched) < p.total_warps) {
+      if (globaltimer_ns() - t0 > WAIT_NS) {
+        set_status(p.status, PA_STATUS_BIT(PA_ERR_TIMEOUT));
+        break;
+      }
+      __nanosleep(64);
+    }
+  }
+  __syncwarp();
+
+  // ---- merge every segment that has partial pieces
+  const long long nseg = static_cast<long long>(p.num_rows) * p.num_kv_heads;
+  for (long long seg = gw; seg < nseg; seg += p.total_warps) {
+    const long long info = __ldcg(p.seginfo + seg);
+    if (info == 0) continue;
+    merge_segment<D, NT>(p, (info & ((1ll << 40) - 1)) - 1, static_cast<int>(info >> 40),
+                         static_cast<int>(seg / p.num_kv_heads), static_cast<int>(seg % p.num_kv_heads), lane);
+    if (lane == 0) p.seginfo[seg] = 0;
+  }
+
+  // ---- the last warp out puts the barrier words back to zero
+  __syncwarp();
+  if (lane == 0) {
+    const int out = atomicAdd(p.sched + 1, 1);
+    if (out == p.total_warps - 1) {
+      p.sched[0] = 0;
+      p.sched[1] = 0;
+    }
   }
 }
 
@@ -537,7 +704,7 @@ template <int D, int NT, int R>
 static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream,
                          int num_sms) {
   using S = RowsShape<D, NT>;
-  const int smem = ROWS_WARPS * R * S::STAGE_BYTES + 1024;
+  const int smem = ROWS_WARPS * R * S::STAGE_BYTES + 1024 + (ROWS_SMEM_SEQS + 1) * 8;
   auto kern = rows_kernel<D, NT, R>;
   static int configured_dev = -1;
   static int blocks_per_sm = 1;
@@ -555,7 +722,24 @@ static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUt
   RowsParams p = p0;
   const int grid = num_sms * blocks_per_sm;
   p.total_warps = grid * ROWS_WARPS;
-  kern<<<grid, ROWS_THREADS, smem, stream>>>(tmk, tmv, p);
+  // Programmatic dependent launch: the prologue (a scan of the batch
+  // metadata) overlaps the kernel before it, typically the cache append;
+  // the kernel waits for that grid before it reads the cache.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(ROWS_THREADS);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  // Cooperative: every CTA is resident at once, which the grid barrier before
+  // the merge phase relies on.
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) return PA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -566,13 +750,46 @@ int rows_supported(int group, int head_dim) {
   return group <= 16;
 }
 
-size_t rows_partials_bytes(int num_q_heads, int num_kv_heads, int head_dim, int num_sms) {
-  const int group = num_q_heads / num_kv_heads;
+namespace {
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+constexpr size_t SCHED_BYTES = 256;
+size_t slot_bytes(int group, int head_dim) {
   const int nt = group > 8 ? 2 : 1;
   const size_t o = static_cast<size_t>(head_dim / 16) * nt * 32 * 4;
-  const size_t slot = (o + 2 * nt * 8 + 63) / 64 * 64;
-  const size_t max_warps = static_cast<size_t>(num_sms) * 2 * ROWS_WARPS;
-  return 2 * max_warps * slot * sizeof(float);
+  return (o + 16 * nt + 1 + 63) / 64 * 64 * sizeof(float);
+}
+size_t max_warps(int num_sms) { return static_cast<size_t>(num_sms) * 2 * ROWS_WARPS; }
+}  // namespace
+
+namespace {
+size_t table_entries(int num_rows, int num_kv_heads, long long max_keys) {
+  return static_cast<size_t>(num_rows) * num_kv_heads * static_cast<size_t>((max_keys + TILE_KEYS - 1) / TILE_KEYS);
+}
+}  // namespace
+
+size_t rows_workspace_bytes(int num_rows, int num_q_heads, int num_kv_heads, int head_dim, long long max_keys,
+                            int num_sms) {
+  const size_t w = max_warps(num_sms);
+  return SCHED_BYTES + round256(static_cast<size_t>(num_rows) * num_kv_heads * sizeof(long long)) +
+         round256(table_entries(num_rows, num_kv_heads, max_keys) * sizeof(long long)) +
+         w * ROWS_SLOTS_PER_WARP * slot_bytes(num_q_heads / num_kv_heads, head_dim);
+}
+
+void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_heads, int head_dim,
+                           long long max_keys, int num_sms, RowsParams* p) {
+  (void)num_q_heads;
+  (void)head_dim;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  (void)num_sms;
+  p->sched = reinterpret_cast<int*>(b);
+  b += SCHED_BYTES;
+  p->seginfo = reinterpret_cast<long long*>(b);
+  b += round256(static_cast<size_t>(num_rows) * num_kv_heads * sizeof(long long));
+  p->table = reinterpret_cast<long long*>(b);
+  p->table_len = static_cast<long long>(table_entries(num_rows, num_kv_heads, max_keys));
+  b += round256(table_entries(num_rows, num_kv_heads, max_keys) * sizeof(long long));
+  p->partials = reinterpret_cast<float*>(b);
+  p->num_rows = num_rows;
 }
 
 int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,

@@ -40,7 +40,8 @@ class DeviceStep:
         self.query_start = i32(w.query_start, device)
         self.slot_mapping = i32(w.slot_mapping, device)
         self.out = torch.empty_like(self.q)
-        self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim, device)
+        self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                           w.block_tables.shape[1], w.block_size, device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def append(self):

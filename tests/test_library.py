@@ -76,7 +76,9 @@ def test_host_checks_answer_before_any_launch(lib):
     assert lib.pa_cache_append(fake, fake, fake, fake, fake, 3, 4, 2, 100, 16, None, None) == -3
     assert lib.pa_cache_append(None, fake, fake, fake, fake, 3, 4, 2, 128, 16, None, None) == -1
     lib.pa_workspace_bytes.restype = ctypes.c_size_t
-    assert lib.pa_workspace_bytes(4, 6, 4, 128) == 0  # bad group -> 0
+    lib.pa_workspace_bytes.argtypes = [ctypes.c_int] * 6
+    assert lib.pa_workspace_bytes(4, 6, 4, 128, 8, 16) == 0  # bad group -> 0
+    assert lib.pa_workspace_bytes(4, 8, 4, 128, 8, 24) == 0  # bad block size -> 0
 
 
 def test_python_binding_imports_on_cpu():
