@@ -49,19 +49,22 @@ int device_info(DeviceInfo* info) {
   return PA_OK;
 }
 
-// [num_blocks, Hkv, block_size, D] bf16 viewed as a 4-D tensor (D fastest);
-// box = 64 columns x 16 token rows of one (block, head), 128-byte swizzle.
+// [num_blocks, Hkv, block_size, D] bf16 viewed as a 5-D tensor
+// (64 columns, block_size rows, D/64 column groups, Hkv, num_blocks): the
+// column groups get their own dimension (stride 128 bytes) so that one box
+// (64 x 16 x D/64) brings a whole 16-key tile of one (block, head) into shared
+// memory as D/64 swizzled [16 x 128-byte] panels, in a single TMA instruction.
 int encode_kv_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
                    int head_dim) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return PA_ERR_CUDA;
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(block_size),
-                              static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
   const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * 2;
-  const cuuint64_t strides[3] = {row, row * block_size, row * block_size * num_kv_heads};
-  const cuuint32_t box[4] = {64, 16, 1, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(cache), dims, strides, box, estr,
+  const cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(head_dim / 64),
+                              static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t strides[4] = {row, 128, row * block_size, row * block_size * num_kv_heads};
+  const cuuint32_t box[5] = {64, 16, static_cast<cuuint32_t>(head_dim / 64), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(cache), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;

@@ -11,18 +11,20 @@
 // How (B200):
 //  * Work unit = one 16-key tile of one (query row, KV head) "segment".  All
 //    G = Hq / Hkv query heads of the KV head ride along, so each K/V byte is
-//    read from HBM once per step.  Every warp scans context_lens itself,
-//    computes the batch's total tile count T and takes an equal contiguous
-//    range of it: the load balance is exact to one tile whatever the length
-//    mix, and no host-side plan is needed.
+//    read from HBM once per step.  Each CTA scans context_lens into shared
+//    memory (tile prefix sums per sequence), every warp takes an equal
+//    contiguous range of the batch's T tiles: the split is exact to one tile
+//    whatever the length mix, deterministic, and needs no host-side plan.
 //  * A segment cut by a range boundary is finished as partial (m, l, O)
-//    results; the last warp to arrive (atomic counter in the workspace)
-//    merges them, so there is no second launch and at most two partial
-//    slots per warp.
-//  * Tiles stream HBM -> shared memory through TMA (4-D tensor map over
-//    [num_blocks, Hkv, block_size, D], block ID as a coordinate, 128-byte
-//    swizzle), a ring of R stages per warp completed on mbarriers.  Each warp
-//    is its own producer and consumer: no block-wide barriers.
+//    results, written with plain stores and recorded in a per-unit piece
+//    table; after a grid barrier (cooperative launch) the pieces of every cut
+//    segment are merged in order.  At most two partial slots per warp, no
+//    second launch, no atomics on the streaming path.
+//  * Tiles stream HBM -> shared memory through TMA (one 5-D box per K or V
+//    tile of one (block, head), block ID as a coordinate, 128-byte swizzle),
+//    a ring of R stages per warp completed on mbarriers.  Each warp is its own
+//    producer and consumer and hands a stage back as soon as the tile is in
+//    registers.
 //  * Math on the tensor cores with the legacy warp MMA (m16n8k16, bf16 in,
 //    fp32 accumulate), keys in M and heads in N:  S^T[16 keys, 8 heads] =
 //    K_tile . Q^T;  the online softmax runs on the S^T fragment;  P goes from
@@ -440,11 +442,8 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
         if (blk < 0 || blk >= p.num_blocks) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
         uint8_t* st = ring + stage * S::STAGE_BYTES;
         mbar_arrive_expect_tx(&bar[stage], S::STAGE_BYTES);
-#pragma unroll
-        for (int pc = 0; pc < S::PIECES; ++pc) {
-          tma_load_4d(st + pc * 2048, &tmk, &bar[stage], pc * 64, y, lc.h, blk, pol);
-          tma_load_4d(st + S::HALF_BYTES + pc * 2048, &tmv, &bar[stage], pc * 64, y, lc.h, blk, pol);
-        }
+        tma_load_5d(st, &tmk, &bar[stage], 0, y, 0, lc.h, blk, pol);
+        tma_load_5d(st + S::HALF_BYTES, &tmv, &bar[stage], 0, y, 0, lc.h, blk, pol);
       }
       ++issued;
       if (!last)
