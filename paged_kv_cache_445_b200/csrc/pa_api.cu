@@ -9,12 +9,6 @@
 
 namespace pa {
 
-namespace {
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
@@ -27,6 +21,8 @@ EncodeTiledFn encode_fn() {
   });
   return fn;
 }
+
+namespace {
 
 constexpr int MAX_DEVICES = 64;
 
@@ -124,7 +120,28 @@ static int run_attention(void* out, const void* q, const int32_t* query_start, c
   p.scale_log2 = scale * 1.4426950408889634f;
   rows_workspace_layout(workspace, total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms, &p);
   p.status = dev_status;
-  return launch_rows(p, tmk, tmv, head_dim, static_cast<cudaStream_t>(stream), di.num_sms);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (query_start && chunk_supported(p.group, head_dim)) {
+    // sequences with more than one query row run on the tcgen05 chunk kernel,
+    // the single rows (decodes) on the rows kernel right after it
+    ChunkParams c{};
+    c.out = out;
+    c.block_tables = block_tables;
+    c.context_lens = context_lens;
+    c.query_start = query_start;
+    c.num_seqs = num_seqs;
+    c.max_blocks = max_blocks;
+    c.num_q_heads = num_q_heads;
+    c.num_kv_heads = num_kv_heads;
+    c.group = p.group;
+    c.block_size = block_size;
+    c.num_blocks = num_blocks;
+    c.scale_log2 = p.scale_log2;
+    c.status = dev_status;
+    if ((rc = launch_chunk(c, q, k_cache, v_cache, total_q_tokens, st, di.num_sms)) != PA_OK) return rc;
+    p.skip_multi = 1;
+  }
+  return launch_rows(p, tmk, tmv, head_dim, st, di.num_sms);
 }
 
 }  // namespace pa

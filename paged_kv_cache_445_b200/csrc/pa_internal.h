@@ -41,6 +41,28 @@ struct RowsParams {
   int total_warps;
 };
 
+// Parameters of the tcgen05 chunk kernel (sequences with more than one query row).
+struct ChunkParams {
+  void* out;                    // bf16 [Tq, Hq, 128]
+  const int32_t* block_tables;  // [B, max_blocks]
+  const int32_t* context_lens;  // [B]
+  const int32_t* query_start;   // [B + 1]
+  int num_seqs;
+  int max_blocks;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int block_size;
+  int num_blocks;
+  float scale_log2;
+  int* status;
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+
 struct DeviceInfo {
   int num_sms;
 };
@@ -63,5 +85,8 @@ size_t rows_workspace_bytes(int num_rows, int num_q_heads, int num_kv_heads, int
 void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_heads, int head_dim,
                            long long max_keys, int num_sms, RowsParams* p);
 int rows_supported(int group, int head_dim);
+int chunk_supported(int group, int head_dim);
+int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const void* v_cache, int total_q_tokens,
+                 cudaStream_t stream, int num_sms);
 
 }  // namespace pa

@@ -101,6 +101,12 @@ SMALL = [  # ctx list, qlen list, Hq, Hkv, d, bs
     ([64, 200], [40, 1], 8, 2, 128, 16),
     ([50, 9, 300, 1], [50, 3, 17, 1], 6, 3, 64, 32),
     ([600], [77], 24, 4, 256, 32),
+    # prefill chunks on the tcgen05 path (head_dim 128, G in {1, 2, 4, 8, 16})
+    ([300], [300], 8, 1, 128, 16),               # whole prompt from position 0, partial last token block
+    ([1000, 40], [130, 1], 16, 2, 128, 32),      # G 8, 32-token blocks, chunk deep in the context
+    ([700], [200], 4, 4, 128, 16),               # G 1: 128 tokens per tile
+    ([500, 77], [50, 1], 32, 2, 128, 16),        # G 16: 8 tokens per tile
+    ([260, 129, 1], [5, 129, 1], 8, 4, 128, 16), # G 2, several chunks and a decode in one batch
 ]
 
 
