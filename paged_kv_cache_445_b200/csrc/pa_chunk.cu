@@ -45,11 +45,13 @@ constexpr int CH_N = 128;                   // keys per N-tile
 constexpr int PANEL = CH_M * 128;           // one 128-row x 128-byte swizzled panel (16 KB)
 constexpr int Q_BYTES = 2 * PANEL;          // [2 head-dim halves][128 rows][128 B]
 constexpr int KV_BYTES = 2 * PANEL;         // one K (or V) tile
-constexpr int STAGES = 2;
+constexpr int KST = 3;                      // K stages (a K tile is free once its QK^T is done)
+constexpr int VST = 2;                      // V stages (a V tile is free once its PV is done)
 constexpr int SMEM_Q = 0;
-constexpr int SMEM_KV = SMEM_Q + Q_BYTES;                     // [stage][K, V]
-constexpr int SMEM_P = SMEM_KV + STAGES * 2 * KV_BYTES;
-constexpr int SMEM_TOTAL = SMEM_P + Q_BYTES;                  // + P (same shape as Q)
+constexpr int SMEM_K = SMEM_Q + Q_BYTES;
+constexpr int SMEM_V = SMEM_K + KST * KV_BYTES;
+constexpr int SMEM_P = SMEM_V + VST * KV_BYTES;
+constexpr int SMEM_TOTAL = SMEM_P + Q_BYTES;                  // + P (same shape as Q): 224 KB
 constexpr uint32_t TMEM_COLS = 512;                           // S0 [0,128), S1 [128,256), O [256,384)
 constexpr uint32_t TMEM_O = 256;
 constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when the max rises by > 2^8
@@ -129,7 +131,7 @@ struct Item {
 struct Shared {
   uint64_t q_full, q_empty, o_empty, pv_done, drain;
   uint64_t s_full[2], s_empty[2];
-  uint64_t kv_full[STAGES], kv_empty[STAGES];
+  uint64_t k_full[KST], k_empty[KST], v_full[VST], v_empty[VST];
   uint64_t p_full;
   uint32_t tmem_base;
   int abort;
@@ -220,9 +222,13 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       mbar_init(&sh.s_full[b], 1);
       mbar_init(&sh.s_empty[b], 128);
     }
-    for (int b = 0; b < STAGES; ++b) {
-      mbar_init(&sh.kv_full[b], 1);
-      mbar_init(&sh.kv_empty[b], 1);
+    for (int b = 0; b < KST; ++b) {
+      mbar_init(&sh.k_full[b], 1);
+      mbar_init(&sh.k_empty[b], 1);
+    }
+    for (int b = 0; b < VST; ++b) {
+      mbar_init(&sh.v_full[b], 1);
+      mbar_init(&sh.v_empty[b], 1);
     }
     sh.abort = 0;
     sh.total = chunk_total(p, TOK);
@@ -249,11 +255,27 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       prefetch_tmap(&tmv);
     }
     const uint64_t pol = policy_evict_last();  // a chunk's K/V is re-read by every M-tile of the chunk
-    uint32_t items = 0, kv_count = 0;
+    uint32_t items = 0, tcount = 0;  // tiles issued over all items (stage and phase bookkeeping)
     for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x, ++items) {
       Item it;
       if (!chunk_item(p, TOK, idx, it)) break;
       const int nt = item_tiles(it, TOK);
+      const int nblk_ctx = (it.ctx + p.block_size - 1) / p.block_size;
+      const int32_t* table = p.block_tables + static_cast<long long>(it.s) * p.max_blocks;
+      // lane b < 8 owns the b-th 16-key group of a tile: block id and row offset in the block
+      auto tile_ids = [&](int j, int& blk, int& y) {
+        blk = -1;
+        y = 0;
+        if (lane < CH_N / 16 && j < nt) {
+          const int key0 = j * CH_N + lane * 16;
+          const int lb = key0 / p.block_size;
+          y = key0 - lb * p.block_size;
+          if (lb < nblk_ctx) blk = __ldg(table + lb);
+        }
+      };
+      int blk_cur, y_cur, blk_prev = -1, y_prev = 0, blk_next, y_next;
+      tile_ids(0, blk_cur, y_cur);
+      tile_ids(1, blk_next, y_next);
       // the previous item's last QK^T has read Q
       if (items > 0 && !ch_wait(sh, &sh.q_empty, (items - 1) & 1, p.status)) break;
       if (lane == 0) {
@@ -261,39 +283,43 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         tma_load_3d(smem + SMEM_Q, &tmq, &sh.q_full, 0, it.kvh * G, it.q0 + it.tb * TOK);
         tma_load_3d(smem + SMEM_Q + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, it.q0 + it.tb * TOK);
       }
-      const int nblk_ctx = (it.ctx + p.block_size - 1) / p.block_size;
-      const int32_t* table = p.block_tables + static_cast<long long>(it.s) * p.max_blocks;
-      for (int j = 0; j < nt; ++j, ++kv_count) {
-        const int stage = kv_count % STAGES;
-        const uint32_t use = kv_count / STAGES;  // how often this stage was used before
-        if (use > 0 && !ch_wait(sh, &sh.kv_empty[stage], (use - 1) & 1, p.status)) break;
-        // lane b < 128/16 fetches the block id of the b-th 16-key group
-        int blk = -1, y = 0;
-        if (lane < CH_N / 16) {
-          const int key0 = j * CH_N + lane * 16;
-          const int lb = key0 / p.block_size;
-          y = key0 - lb * p.block_size;
-          if (lb < nblk_ctx) blk = __ldg(table + lb);
+      auto load_tile = [&](const CUtensorMap* tm, uint64_t* bars_full, uint64_t* bars_empty, int nst, int base_off,
+                           uint32_t t, int blk, int y) -> bool {
+        const int st = t % nst;
+        const uint32_t use = t / nst;  // earlier fills of this stage
+        if (use > 0 && !ch_wait(sh, &bars_empty[st], (use - 1) & 1, p.status)) return false;
+        if (lane == 0) mbar_arrive_expect_tx(&bars_full[st], KV_BYTES);
+        __syncwarp();
+        if (lane < CH_N / 16) {  // 16-row boxes (head-dim half, 16 keys) -> rows 16*lane.. of both panels
           if (blk >= p.num_blocks) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+          uint8_t* dst = smem + base_off + st * KV_BYTES + lane * 2048;
+          tma_load_4d(dst, tm, &bars_full[st], 0, y, it.kvh, blk, pol);
+          tma_load_4d(dst + PANEL, tm, &bars_full[st], 64, y, it.kvh, blk, pol);
         }
-        __syncwarp();
-        uint8_t* kst = smem + SMEM_KV + stage * 2 * KV_BYTES;
-        if (lane == 0) mbar_arrive_expect_tx(&sh.kv_full[stage], 2 * KV_BYTES);
-        __syncwarp();
-        if (lane < CH_N / 16) {  // 16-row boxes: (head-dim half, 16 keys) -> rows 16*lane.. of both panels
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            tma_load_4d(kst + hf * PANEL + lane * 2048, &tmk, &sh.kv_full[stage], hf * 64, y, it.kvh, blk, pol);
-            tma_load_4d(kst + KV_BYTES + hf * PANEL + lane * 2048, &tmv, &sh.kv_full[stage], hf * 64, y, it.kvh,
-                        blk, pol);
-          }
-        }
+        return true;
+      };
+      bool ok = true;
+      for (int j = 0; ok && j < nt; ++j) {
+        ok = load_tile(&tmk, sh.k_full, sh.k_empty, KST, SMEM_K, tcount + j, blk_cur, y_cur);
+        if (ok && j > 0) ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + j - 1, blk_prev, y_prev);
+        blk_prev = blk_cur;
+        y_prev = y_cur;
+        blk_cur = blk_next;
+        y_cur = y_next;
+        tile_ids(j + 2, blk_next, y_next);  // one tile of lead for the block-table reads
       }
+      if (ok && nt > 0) ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + nt - 1, blk_prev, y_prev);
+      tcount += nt;
+      if (!ok) break;
     }
     if (sh.abort) {  // let this CTA's copies still in flight land before its shared memory goes away
-      for (int st = 0; st < STAGES; ++st) {
-        const uint32_t uses = kv_count / STAGES + (static_cast<uint32_t>(st) < kv_count % STAGES ? 1u : 0u);
-        if (uses > 0) mbar_wait(&sh.kv_full[st], (uses - 1) & 1);
+      for (int st = 0; st < KST; ++st) {
+        const uint32_t uses = tcount / KST + (static_cast<uint32_t>(st) < tcount % KST ? 1u : 0u);
+        if (uses > 0) mbar_wait(&sh.k_full[st], (uses - 1) & 1);
+      }
+      for (int st = 0; st < VST; ++st) {
+        const uint32_t uses = tcount / VST + (static_cast<uint32_t>(st) < tcount % VST ? 1u : 0u);
+        if (uses > 0) mbar_wait(&sh.v_full[st], (uses - 1) & 1);
       }
       if (items > 0) mbar_wait(&sh.q_full, (items - 1) & 1);
     }
@@ -317,15 +343,15 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       first_item = false;
       bool ok = true;
       auto qk = [&](int j) -> bool {
-        const int stage = (kv_count + j) % STAGES;
-        const uint32_t use = (kv_count + j) / STAGES;
-        if (!ch_wait(sh, &sh.kv_full[stage], use & 1, p.status)) return false;
+        const int stage = (kv_count + j) % KST;
+        const uint32_t use = (kv_count + j) / KST;
+        if (!ch_wait(sh, &sh.k_full[stage], use & 1, p.status)) return false;
         const int sb = j & 1;
         if (s_use[sb] > 0 && !ch_wait(sh, &sh.s_empty[sb], (s_use[sb] - 1) & 1, p.status)) return false;
         ++s_use[sb];
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t sk = smem_u32(smem + SMEM_KV + stage * 2 * KV_BYTES);
+          const uint32_t sk = smem_u32(smem + SMEM_K + stage * KV_BYTES);
 #pragma unroll
           for (int kk = 0; kk < CH_D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
@@ -333,6 +359,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
                      kk > 0);
           }
           umma_commit(&sh.s_full[sb]);
+          umma_commit(&sh.k_empty[stage]);
           if (j == nt - 1) umma_commit(&sh.q_empty);
         }
         __syncwarp();
@@ -341,10 +368,11 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       auto pv = [&](int j) -> bool {
         if (!ch_wait(sh, &sh.p_full, p_phase, p.status)) return false;
         p_phase ^= 1;
+        const int stage = (kv_count + j) % VST;
+        if (!ch_wait(sh, &sh.v_full[stage], ((kv_count + j) / VST) & 1, p.status)) return false;
         tc_fence_after();
-        const int stage = (kv_count + j) % STAGES;
         if (lane == 0) {
-          const uint32_t sv = smem_u32(smem + SMEM_KV + stage * 2 * KV_BYTES + KV_BYTES);
+          const uint32_t sv = smem_u32(smem + SMEM_V + stage * KV_BYTES);
 #pragma unroll
           for (int kk = 0; kk < CH_N / 16; ++kk) {
             // A = P (K-major, keys 16kk..), B = V (MN-major: 16 key rows from row 16kk, both head-dim panels)
@@ -352,7 +380,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
                      umma_desc(sv + kk * 16 * 128, PANEL, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&sh.pv_done);
-          umma_commit(&sh.kv_empty[stage]);
+          umma_commit(&sh.v_empty[stage]);
         }
         __syncwarp();
         return true;
@@ -451,8 +479,9 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         // keys past the context may hold anything (even NaN): zero their V rows
         const int valid_keys = it.ctx - key0;
         if (valid_keys < CH_N) {
-          const int stage = (kv_count + j) % STAGES;
-          uint8_t* vst = smem + SMEM_KV + stage * 2 * KV_BYTES + KV_BYTES;
+          const int stage = (kv_count + j) % VST;
+          if (!(ok = ch_wait(sh, &sh.v_full[stage], ((kv_count + j) / VST) & 1, p.status))) break;
+          uint8_t* vst = smem + SMEM_V + stage * KV_BYTES;
           const int nz = (CH_N - max(valid_keys, 0)) * 2 * 8;  // 16-byte chunks in both panels
           for (int k = threadIdx.x - 64; k < nz; k += 128) {
             const int r = max(valid_keys, 0) + k / 16, rest = k % 16;
