@@ -427,55 +427,74 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
 
         const int key0 = j * CH_N;
         const bool diag = key0 + CH_N - 1 > it.p0 + it.tb * TOK;  // some row of the tile stops inside it
-        float mx = -INFINITY;
+        const float cs = p.scale_log2;
+        // Off the diagonal every key is visible: take the max of the raw scores
+        // and fold the scale into one FFMA per element below.  On a diagonal
+        // tile scale first, then mask (the scale may be zero).
+        float mx;
+        {
+          float m8[8];
+          if (diag) {
 #pragma unroll
-        for (int i = 0; i < CH_N; ++i) {
-          float x = s[i] * p.scale_log2;
-          if (diag && key0 + i > last_key) x = -INFINITY;
-          s[i] = x;
-          mx = fmaxf(mx, x);
+            for (int i = 0; i < CH_N; ++i) {
+              const float x = s[i] * cs;
+              s[i] = key0 + i > last_key ? -INFINITY : x;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) m8[k] = s[k];
+#pragma unroll
+          for (int i = 8; i < CH_N; i += 8)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[i + k]);
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          if (!diag) mx *= cs;
         }
-        // tile j-1's P V must be done before P is rewritten or O is rescaled
+        // Decide the reference maximum, compute P in registers (this overlaps the
+        // previous tile's P V on the tensor cores), and only then wait for that
+        // P V before P's shared memory is rewritten or O is rescaled.
+        const bool rescale = mx > m_ref + RESCALE_LOG2 || m_ref == -INFINITY;
+        const float m_new = rescale ? fmaxf(mx, m_ref) : m_ref;
+        uint32_t pk[CH_N / 2];
+        float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const float neg_m = -m_new;
+#pragma unroll
+        for (int i = 0; i < CH_N / 2; ++i) {
+          const float x0 = s[2 * i], x1 = s[2 * i + 1];
+          const float a = fast_exp2(diag ? x0 + neg_m : fmaf(x0, cs, neg_m));
+          const float b = fast_exp2(diag ? x1 + neg_m : fmaf(x1, cs, neg_m));
+          l8[i & 7] += a + b;
+          pk[i] = pack_bf16x2(a, b);
+        }
         if (j > 0) {
           if (!(ok = ch_wait(sh, &sh.pv_done, pv_phase, p.status))) break;
           pv_phase ^= 1;
           tc_fence_after();
         }
-        if (mx > m_ref + RESCALE_LOG2 || m_ref == -INFINITY) {
-          const float m_new = fmaxf(mx, m_ref);
-          if (m_ref != -INFINITY) {
-            const float alpha = fast_exp2(m_ref - m_new);
-            l *= alpha;
-            if (j > 0) {  // O holds tiles 0..j-1: scale it in tensor memory
+        if (rescale && m_ref != -INFINITY) {
+          const float alpha = fast_exp2(m_ref - m_new);
+          l *= alpha;
+          if (j > 0) {  // O holds tiles 0..j-1: scale it in tensor memory
 #pragma unroll
-              for (int c = 0; c < CH_D / 32; ++c) {
-                float v[32];
-                tmem_ld32(tmem + lane_addr + TMEM_O + c * 32, v);
-                tmem_wait_ld();
+            for (int c = 0; c < CH_D / 32; ++c) {
+              float v[32];
+              tmem_ld32(tmem + lane_addr + TMEM_O + c * 32, v);
+              tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= alpha;
-                tmem_st32(tmem + lane_addr + TMEM_O + c * 32, v);
-              }
-              tmem_wait_st();
+              for (int i = 0; i < 32; ++i) v[i] *= alpha;
+              tmem_st32(tmem + lane_addr + TMEM_O + c * 32, v);
             }
+            tmem_wait_st();
           }
-          m_ref = m_new;
         }
-        // P = exp2(s - m_ref) in bf16, row `row` of the K-major SW128 A panels
-        float lsum = 0.f;
+        m_ref = m_new;
+        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+        // P (bf16), row `row` of the K-major SW128 A panels
 #pragma unroll
         for (int c8 = 0; c8 < CH_N / 8; ++c8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = fast_exp2(s[c8 * 8 + 2 * e] - m_ref), b = fast_exp2(s[c8 * 8 + 2 * e + 1] - m_ref);
-            lsum += a + b;
-            w[e] = pack_bf16x2(a, b);
-          }
           uint8_t* dst = pbuf + (c8 >> 3) * PANEL + sw128(row, c8 & 7);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
         }
-        l += lsum;
         // keys past the context may hold anything (even NaN): zero their V rows
         const int valid_keys = it.ctx - key0;
         if (valid_keys < CH_N) {
