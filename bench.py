@@ -60,13 +60,18 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {  # the files whose text decides each kernel's code
+    "pa_rows_kernel": ("pa_rows.cu", "pa_device.cuh"),
+    "pa_chunk_kernel": ("pa_chunk.cu", "pa_device.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_445_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -79,7 +84,7 @@ def profiled_traffic(kernel: str, workload: str):
     text = open(path).read()
     m = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
     t = re.search(r"dram_bytes_per_launch_full_size:\s*([0-9.e+]+)", text)
-    if not m or not t or m.group(1) != kernel_source_hash():
+    if not m or not t or m.group(1) != kernel_source_hash(kernel):
         return None
     return float(t.group(1))
 
