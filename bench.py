@@ -154,8 +154,10 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------- distributed
-def dist_setup(n_gpus: int):
-    import torch
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU: read RANK / LOCAL_RANK / WORLD_SIZE from the
+    environment torchrun sets and join the process group (NCCL on GPUs; the
+    CPU tests use gloo)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -164,11 +166,16 @@ def dist_setup(n_gpus: int):
     if world > 1:
         import datetime
 
+        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
+    elif backend == "nccl":
+        import torch
         torch.cuda.set_device(0)
     return rank, world, local
 
@@ -179,14 +186,39 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def reduce_over_ranks(x: float, world: int, op: str = "max", device: str = "cuda") -> float:
+    """MAX or SUM of one number over all ranks (every rank gets the result)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    return reduce_over_ranks(x, world, "max", device)
+
+
+def rank_seed(workload: int, rank: int) -> int:
+    """Each rank runs its own batch of the same workload (weak scaling)."""
+    return 445 + workload + 1000 * rank
+
+
+def step_launches(w, chunk_head_dims=(128,), chunk_groups=(1, 2, 4, 8, 16)) -> int:
+    """Kernel launches of one step: the append, the rows kernel, and the
+    tcgen05 chunk kernel when the batch has a multi-row sequence it takes."""
+    qs = np.asarray(w.query_start)
+    multi = bool(np.any(np.diff(qs) > 1))
+    chunk = (not w.is_decode and multi and w.head_dim in chunk_head_dims
+             and (w.num_q_heads // w.num_kv_heads) in chunk_groups)
+    return 2 + int(chunk)
+
+
+def compose_value(total_kv_bytes: float, ms_step_max: float) -> float:
+    """Whole-job KV GB/s: the bytes all ranks read over the slowest rank's step."""
+    return total_kv_bytes / (ms_step_max * 1e-3) / 1e9
 
 
 # --------------------------------------------------------------------- workload
@@ -242,7 +274,7 @@ def run_ours(args, peaks):
     rank, world, local = dist_setup(args.gpus)
     device = torch.device("cuda", local)
     t0 = time.time()
-    w = workloads.standard(args.workload, seed=445 + args.workload + 1000 * rank)
+    w = workloads.standard(args.workload, seed=rank_seed(args.workload, rank))
     log(f"[rank {rank}] workload {w.name}: {w.num_seqs} seqs, {w.num_query_tokens} query rows, "
         f"{int(w.context_lens.sum())} keys, pool {w.num_blocks} blocks ({time.time() - t0:.1f}s to generate)")
     g = GpuStep(w, device)
@@ -308,6 +340,8 @@ def run_ours(args, peaks):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world)
+    total_kv = reduce_over_ranks(float(kv_bytes), world, "sum")
+    total_seqs = reduce_over_ranks(float(w.num_seqs), world, "sum")
 
     # ---- CPU baseline: the oracle on this host's cores, rank 0 at N = 1 only
     cpu = None
@@ -320,7 +354,7 @@ def run_ours(args, peaks):
     traffic = profiled_traffic("pa_rows_kernel", w.name)
     line = {
         "metric": "paged-attn decode KV GB/s + seq-steps/s (70B layer, bs128); % of HBM peak",
-        "value": round(world * kv_bytes / (ms_step * 1e-3) / 1e9, 2),
+        "value": round(compose_value(total_kv, ms_step), 2),
         "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 5),
@@ -337,9 +371,9 @@ def run_ours(args, peaks):
             "l2": f"no flush: every step reads {kv_bytes / 1e9:.2f} GB of KV, larger than the 126 MB L2",
             "parallelism": f"dp{world} (independent batch per GPU)",
         },
-        "seq_steps_per_s": round(world * w.num_seqs / (ms_step * 1e-3), 1),
-        "frac_of_hbm_peak": round(world * kv_bytes / (ms_step * 1e-3) / 1e9 / hbm / world, 4),
-        "frac_of_8tbs_nominal": round(kv_bytes / (ms_step * 1e-3) / 1e9 / 8000.0, 4),
+        "seq_steps_per_s": round(total_seqs / (ms_step * 1e-3), 1),
+        "frac_of_hbm_peak": round(compose_value(total_kv, ms_step) / hbm / world, 4),
+        "frac_of_8tbs_nominal": round(compose_value(total_kv, ms_step) / 8000.0 / world, 4),
         "roofline": {
             "kernel": "pa_rows_kernel (attention)", "bound": "hbm",
             "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
@@ -349,9 +383,9 @@ def run_ours(args, peaks):
             "avg_launch_ms": round(attn_avg_ms, 5),
         },
         "append": {"algorithmic_bytes": app_bytes},
-        "e2e": {"value": round(world * kv_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(compose_value(total_kv, e2e_ms), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": step_launches(w) * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
