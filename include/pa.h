@@ -14,7 +14,8 @@
  *  - Every tensor pointer is CUDA device memory owned by the caller.  The
  *    library never allocates, frees or synchronises; each call enqueues its
  *    kernels on `stream` (a cudaStream_t, NULL = the legacy default stream)
- *    and returns.  Calls are stateless and thread-safe.
+ *    and returns.  Calls are stateless and thread-safe (pa_decode_static_scratch
+ *    is the one exception: see its comment).
  *  - Layouts (row-major, no padding):
  *      q, out        bf16  [num_q_tokens, num_q_heads, head_dim]
  *      k_new, v_new  bf16  [num_tokens, num_kv_heads, head_dim]
@@ -153,6 +154,38 @@ PA_API int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start
                      const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
                      int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
                      void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/*
+ * pa_decode_static_scratch -- pa_decode without a caller workspace.  Same
+ * arguments, layouts, result and errors as pa_decode, minus `workspace` and
+ * `workspace_bytes`.  The sources this library follows describe no such call:
+ * it exists for callers that cannot hand the library device memory when they
+ * launch (a runtime that may not call the allocator while it replays a
+ * recorded sequence of launches, or a host with a fixed memory budget).
+ *
+ * Scratch: a library-owned device array of PA_STATIC_SCRATCH_BYTES per device
+ * (64 MiB), part of the library's device image, so this call allocates
+ * nothing.  A batch whose pa_workspace_bytes(num_seqs, ...) exceeds that size
+ * is rejected with PA_ERR_WORKSPACE before any launch (for example, 8 query
+ * heads per KV head at head_dim 128 on a 148-SM B200 fits about 1,700
+ * sequences with 512-block tables).
+ *
+ * Sharing: every call on a device uses the same array.  Calls that overlap in
+ * time on one device (other streams, other host threads) race on it and give
+ * wrong results: serialise them.  The array keeps what the previous call
+ * left; each call clears the part that must start at zero on `stream` before
+ * its kernel, so a call after a failed one needs no reset.
+ *
+ * Set-up: the first call on a device, with that device current, looks up the
+ * array's device address (which may load the library's device code there).
+ * Make that first call before any stream capture on that device.
+ */
+#define PA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+PA_API int pa_decode_static_scratch(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, int max_blocks_per_seq,
+                                    const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                                    int head_dim, int block_size, int num_blocks, float scale, int* dev_status,
+                                    void* stream);
 
 /* Human-readable name of a pa_status value (static storage). */
 PA_API const char* pa_status_string(int status);

@@ -30,12 +30,16 @@ _lib.pa_decode.restype = _ci
 _lib.pa_prefill_chunk.argtypes = [_vp, _vp, _i32p, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci, _ci,
                                   ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
 _lib.pa_prefill_chunk.restype = _ci
+_lib.pa_decode_static_scratch.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
+                                          ctypes.c_float, _vp, _vp]
+_lib.pa_decode_static_scratch.restype = _ci
 _lib.pa_status_string.argtypes = [_ci]
 _lib.pa_status_string.restype = ctypes.c_char_p
 
 PA_OK = 0
 PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE = -1, -2, -3, -4
 PA_ERR_RANGE, PA_ERR_CUDA, PA_ERR_TIMEOUT = -5, -6, -7
+STATIC_SCRATCH_BYTES = 64 * 1024 * 1024  # PA_STATIC_SCRATCH_BYTES of include/pa.h
 
 
 def status_bit(code: int) -> int:
@@ -44,9 +48,10 @@ def status_bit(code: int) -> int:
 
 
 class PAError(RuntimeError):
-    def __init__(self, code: int):
+    def __init__(self, code: int, detail: str | None = None):
         self.code = code
-        super().__init__(pa_status_string(code))
+        msg = pa_status_string(code)
+        super().__init__(f"{msg} ({detail})" if detail else msg)
 
 
 def pa_status_string(code: int) -> str:
@@ -158,5 +163,36 @@ def pa_prefill_chunk(out, q, query_start, k_cache, v_cache, block_tables, contex
                                  _status_ptr(dev_status), _stream_ptr(stream)))
 
 
+def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale, dev_status=None,
+                             stream=None) -> None:
+    """pa_decode without a workspace argument, for callers that cannot allocate
+    device memory when they launch: the library's own per-device scratch array
+    (STATIC_SCRATCH_BYTES) is used instead.  Overlapping calls on one device
+    race on that array; make the first call on a device before any stream
+    capture.  See include/pa.h."""
+    op = _dev(out, "out", torch.bfloat16, 3)
+    qp = _dev(q, "q", torch.bfloat16, 3)
+    kc = _dev(k_cache, "k_cache", torch.bfloat16, 4)
+    vc = _dev(v_cache, "v_cache", torch.bfloat16, 4)
+    bt = _dev(block_tables, "block_tables", torch.int32, 2)
+    cl = _dev(context_lens, "context_lens", torch.int32, 1)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    if v_cache.shape != k_cache.shape or k_cache.shape[3] != q.shape[2]:
+        raise ValueError("k_cache/v_cache must be [num_blocks, Hkv, block_size, d] with q's d")
+    if block_tables.shape[0] != context_lens.shape[0] or q.shape[0] != context_lens.shape[0]:
+        raise ValueError("one query row, one block-table row and one length per sequence")
+    nb, hkv, bs, d = k_cache.shape
+    rc = _lib.pa_decode_static_scratch(op, qp, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0],
+                                       q.shape[1], hkv, d, bs, nb, float(scale), _status_ptr(dev_status),
+                                       _stream_ptr(stream))
+    if rc == PA_ERR_WORKSPACE:
+        need = int(_lib.pa_workspace_bytes(context_lens.shape[0], q.shape[1], hkv, d, block_tables.shape[1], bs))
+        raise PAError(rc, f"this batch needs {need} bytes of scratch, more than the {STATIC_SCRATCH_BYTES}-byte "
+                          "static array: use pa_decode with a workspace")
+    _check(rc)
+
+
 def exported_symbols() -> list[str]:
-    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_prefill_chunk", "pa_status_string"]
+    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_prefill_chunk", "pa_decode_static_scratch",
+            "pa_status_string"]

@@ -82,7 +82,7 @@ static size_t workspace_needed(int num_query_tokens, int num_q_heads, int num_kv
   return rows_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, num_sms);
 }
 
-static int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache,
+int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache,
                          const void* v_cache, const int32_t* block_tables, int max_blocks,
                          const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,

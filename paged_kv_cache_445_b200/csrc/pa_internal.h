@@ -88,5 +88,12 @@ int rows_supported(int group, int head_dim);
 int chunk_supported(int group, int head_dim);
 int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const void* v_cache, int total_q_tokens,
                  cudaStream_t stream, int num_sms);
+// Argument checks, tensor maps and kernel dispatch shared by the attention
+// entry points (query_start == nullptr: one query row per sequence).
+int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,
+                  const int32_t* block_tables, int max_blocks, const int32_t* context_lens, int num_seqs,
+                  int total_q_tokens, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                  int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
+                  void* stream);
 
 }  // namespace pa

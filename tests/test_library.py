@@ -85,3 +85,10 @@ def test_python_binding_imports_on_cpu():
     import paged_kv_cache_445_b200 as pa
     assert pa.pa_status_string(-4).startswith("PA_ERR_WORKSPACE")
     assert pa.status_bit(-5) == 32
+
+
+def test_static_scratch_size_matches_the_header():
+    from paged_kv_cache_445_b200 import _binding
+    m = re.search(r"#define\s+PA_STATIC_SCRATCH_BYTES\s+\((\d+)u\s*\*\s*(\d+)u\s*\*\s*(\d+)u\)", open(HEADER).read())
+    assert m, "PA_STATIC_SCRATCH_BYTES not found"
+    assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == _binding.STATIC_SCRATCH_BYTES
