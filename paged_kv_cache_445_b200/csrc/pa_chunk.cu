@@ -10,22 +10,30 @@
 //
 // How (B200):
 //  * M-tile = 128 query rows = 128/G consecutive tokens x the G query heads of
-//    one KV head (GQA packing: every K/V tile feeds all G heads).  Q comes in
-//    with one 3-D TMA box per head-dim half (128 rows x 128 bytes, 128-byte
-//    swizzle) -- a K-major UMMA operand as it lands.
+//    one KV head (GQA packing: every K/V tile feeds all G heads).  A work item
+//    is a PAIR of consecutive M-tiles (A and B) of one KV head: both multiply
+//    the same K/V tiles, so each tile crosses L2 -> shared memory once per
+//    256 query rows.  Q comes in with one 3-D TMA box per head-dim half and
+//    M-tile (128 rows x 128 bytes, 128-byte swizzle) -- a K-major UMMA operand
+//    as it lands.
 //  * N-tile = 128 keys: 128/block_size blocks, each fetched with 16-row TMA
 //    boxes straight into K-major SW128 panels (K for S = Q K^T) and the same
 //    panels serve as the MN-major B operand of O += P V.
-//  * Warp roles (6 warps): warp 0 issues TMA; warp 1 allocates tensor memory
-//    and issues tcgen05.mma from one thread; warps 2-5 (128 threads, thread =
-//    TMEM lane = query row) run the softmax.  S is double-buffered in TMEM so
-//    QK^T of tile j+1 overlaps the softmax of tile j; O (128 fp32 columns)
-//    stays in TMEM for the whole M-tile.
+//  * Warp roles (12 warps, 3 warpgroups): warp 0 issues TMA; warp 1 allocates
+//    tensor memory and issues tcgen05.mma from one thread; warpgroup 1 runs
+//    the softmax of M-tile A, warpgroup 2 that of M-tile B (thread = TMEM lane
+//    = query row).  Warpgroup 0 gives registers to the two softmax
+//    warpgroups (setmaxnreg).  Tensor memory: S_A, S_B (128 fp32 columns
+//    each; P overwrites the first 64 columns of its S as bf16 pairs and is
+//    the A operand of P V straight from tensor memory) and O_A, O_B (128
+//    columns each).  The MMA issue order QK_A(j), QK_B(j), PV_A(j), QK_A(j+1),
+//    PV_B(j), QK_B(j+1), ... lets the tensor cores work on one M-tile while the
+//    softmax of the other runs.
 //  * Softmax: row max and exp2 on the thread's own row (no shuffles), causal
 //    mask on diagonal tiles only, O is rescaled in TMEM only when the running
 //    maximum rises by more than 2^8 (between rescales the stale maximum is an
-//    exact reference point).  P goes to shared memory as a K-major SW128 A
-//    operand.  Key rows past the context are zeroed in V before P V.
+//    exact reference point).  Key rows past the context are zeroed in V
+//    before P V.
 //  * Every wait is bounded; on a timeout the CTA raises PA_ERR_TIMEOUT, stops
 //    all roles through a shared abort flag, drains its tensor-core work and
 //    frees its tensor memory.
@@ -38,23 +46,28 @@ namespace pa {
 
 namespace {
 
-constexpr int CH_THREADS = 192;
+constexpr int CH_THREADS = 384;
 constexpr int CH_D = 128;
 constexpr int CH_M = 128;                   // query rows per M-tile
 constexpr int CH_N = 128;                   // keys per N-tile
 constexpr int PANEL = CH_M * 128;           // one 128-row x 128-byte swizzled panel (16 KB)
-constexpr int Q_BYTES = 2 * PANEL;          // [2 head-dim halves][128 rows][128 B]
+constexpr int Q_BYTES = 2 * PANEL;          // one M-tile of Q: [2 head-dim halves][128 rows][128 B]
 constexpr int KV_BYTES = 2 * PANEL;         // one K (or V) tile
-constexpr int KST = 3;                      // K stages (a K tile is free once its QK^T is done)
-constexpr int VST = 2;                      // V stages (a V tile is free once its PV is done)
-constexpr int SMEM_Q = 0;
-constexpr int SMEM_K = SMEM_Q + Q_BYTES;
+constexpr int KST = 3;                      // K stages (a K tile is free once QK_B of it is done)
+constexpr int VST = 2;                      // V stages (a V tile is free once PV_B of it is done)
+constexpr int SMEM_Q = 0;                   // Q_A, Q_B
+constexpr int SMEM_K = SMEM_Q + 2 * Q_BYTES;
 constexpr int SMEM_V = SMEM_K + KST * KV_BYTES;
-constexpr int SMEM_P = SMEM_V + VST * KV_BYTES;
-constexpr int SMEM_TOTAL = SMEM_P + Q_BYTES;                  // + P (same shape as Q): 224 KB
-constexpr uint32_t TMEM_COLS = 512;                           // S0 [0,128), S1 [128,256), O [256,384)
-constexpr uint32_t TMEM_O = 256;
+constexpr int SMEM_TOTAL = SMEM_V + VST * KV_BYTES;           // 224 KB
+constexpr uint32_t TMEM_COLS = 512;                           // S_A, S_B, O_A, O_B: 128 columns each
+constexpr uint32_t TMEM_O = 256;                              // O of M-tile w at TMEM_O + 128 w
 constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when the max rises by > 2^8
+// Register split (setmaxnreg): the launch gives 168 per thread (65,536 / 384,
+// rounded down to 8); warpgroup 0 drops to 80, the softmax warpgroups rise to
+// 208: 128 x 80 + 256 x 208 = 63,488 <= 384 x 168 = 64,512, the launch's total
+// (a larger sum would make setmaxnreg.inc wait forever).
+constexpr int REGS_LAUNCH = 168, REGS_PRODUCER = 80, REGS_SOFTMAX = 208;
+static_assert(128 * REGS_PRODUCER + 256 * REGS_SOFTMAX <= CH_THREADS * REGS_LAUNCH, "register split");
 
 // ---- tcgen05 / UMMA helpers
 __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -77,6 +90,17 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
+// Same MMA with the A operand (M x 16, K-major, 2 bf16 per 32-bit column) read
+// from tensor memory at column address a_tmem.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -118,6 +142,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]),
+      "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -125,14 +160,13 @@ struct Item {
   int s;           // sequence
   int q0, qlen;    // its query rows
   int p0, ctx;     // position of its first row, its key count
-  int tb, kvh;     // token block (of 128/G tokens) and KV head
+  int tp, kvh;     // pair of token blocks (2 x 128/G tokens) and KV head
 };
 
 struct Shared {
-  uint64_t q_full, q_empty, o_empty, pv_done, drain;
-  uint64_t s_full[2], s_empty[2];
+  uint64_t q_full, q_empty, drain;
+  uint64_t s_full[2], p_full[2], pv_done[2], o_empty[2];
   uint64_t k_full[KST], k_empty[KST], v_full[VST], v_empty[VST];
-  uint64_t p_full;
   uint32_t tmem_base;
   int abort;
   long long total;
@@ -140,10 +174,11 @@ struct Shared {
 
 }  // namespace
 
-// Items = (multi-row sequence, token block, KV head), numbered sequence by
-// sequence; every CTA walks items blockIdx.x, + gridDim.x, ...  The batch is
-// scanned from global memory by each role (it is small and L1-resident).
-__device__ __forceinline__ bool chunk_item(const ChunkParams& p, int tok, long long idx, Item& it) {
+// Items = (multi-row sequence, pair of token blocks, KV head), numbered
+// sequence by sequence; every CTA walks items blockIdx.x, + gridDim.x, ...
+// The batch is scanned from global memory by each role (it is small and
+// L1-resident).
+__device__ __forceinline__ bool chunk_item(const ChunkParams& p, int pair_tok, long long idx, Item& it) {
   long long base = 0;
   for (int s = 0; s < p.num_seqs; ++s) {
     const int q0 = __ldg(p.query_start + s), qlen = __ldg(p.query_start + s + 1) - q0;
@@ -151,8 +186,8 @@ __device__ __forceinline__ bool chunk_item(const ChunkParams& p, int tok, long l
     int ctx = __ldg(p.context_lens + s);
     const int cap = p.max_blocks * p.block_size;
     if (ctx > cap) ctx = cap;
-    const int nblk = (qlen + tok - 1) / tok;
-    const long long n = static_cast<long long>(nblk) * p.num_kv_heads;
+    const int npair = (qlen + pair_tok - 1) / pair_tok;
+    const long long n = static_cast<long long>(npair) * p.num_kv_heads;
     if (idx < base + n) {
       const int r = static_cast<int>(idx - base);
       it.s = s;
@@ -160,7 +195,7 @@ __device__ __forceinline__ bool chunk_item(const ChunkParams& p, int tok, long l
       it.qlen = qlen;
       it.ctx = ctx;
       it.p0 = ctx - qlen;
-      it.tb = r / p.num_kv_heads;
+      it.tp = r / p.num_kv_heads;
       it.kvh = r % p.num_kv_heads;
       return true;
     }
@@ -169,18 +204,19 @@ __device__ __forceinline__ bool chunk_item(const ChunkParams& p, int tok, long l
   return false;
 }
 
-__device__ __forceinline__ long long chunk_total(const ChunkParams& p, int tok) {
+__device__ __forceinline__ long long chunk_total(const ChunkParams& p, int pair_tok) {
   long long n = 0;
   for (int s = 0; s < p.num_seqs; ++s) {
     const int qlen = __ldg(p.query_start + s + 1) - __ldg(p.query_start + s);
-    if (qlen > 1) n += static_cast<long long>((qlen + tok - 1) / tok) * p.num_kv_heads;
+    if (qlen > 1) n += static_cast<long long>((qlen + pair_tok - 1) / pair_tok) * p.num_kv_heads;
   }
   return n;
 }
 
-// Keys an item needs: up to the last position of its token block (capped at the context).
-__device__ __forceinline__ int item_tiles(const Item& it, int tok) {
-  int last = it.p0 + min((it.tb + 1) * tok, it.qlen) - 1;  // last visible key of the block's last row
+// Key tiles an item needs: up to the last position of its pair's last row
+// (capped at the context).  M-tile A may see fewer; its extra keys are masked.
+__device__ __forceinline__ int item_tiles(const Item& it, int pair_tok) {
+  int last = it.p0 + min((it.tp + 1) * pair_tok, it.qlen) - 1;
   if (last >= it.ctx) last = it.ctx - 1;
   return last < 0 ? 0 : last / CH_N + 1;
 }
@@ -201,11 +237,21 @@ __device__ __forceinline__ bool ch_wait(Shared& sh, uint64_t* bar, uint32_t phas
   }
 }
 
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 template <int G>
 __global__ void __launch_bounds__(CH_THREADS, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, const ChunkParams p) {
   constexpr int TOK = CH_M / G;  // tokens per M-tile
+  constexpr int PAIR = 2 * TOK;  // tokens per item
   extern __shared__ uint8_t smem_raw[];
   __shared__ Shared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -214,13 +260,12 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(&sh.q_full, 1);
     mbar_init(&sh.q_empty, 1);
-    mbar_init(&sh.o_empty, 128);
-    mbar_init(&sh.pv_done, 1);
     mbar_init(&sh.drain, 1);
-    mbar_init(&sh.p_full, 128);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sh.s_full[b], 1);
-      mbar_init(&sh.s_empty[b], 128);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&sh.s_full[w], 1);
+      mbar_init(&sh.p_full[w], 128);
+      mbar_init(&sh.pv_done[w], 1);
+      mbar_init(&sh.o_empty[w], 128);
     }
     for (int b = 0; b < KST; ++b) {
       mbar_init(&sh.k_full[b], 1);
@@ -231,10 +276,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       mbar_init(&sh.v_empty[b], 1);
     }
     sh.abort = 0;
-    sh.total = chunk_total(p, TOK);
+    sh.total = chunk_total(p, PAIR);
     fence_mbar_init();
   }
-  if (warp == 1) {  // tensor memory: S0, S1, O
+  if (warp == 1) {  // tensor memory: S_A, S_B, O_A, O_B
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh.tmem_base)),
                  "r"(TMEM_COLS)
                  : "memory");
@@ -247,19 +292,22 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
   grid_dependency_wait();  // the cache may still be being appended by the kernel before this one
 
   const long long total = sh.total;
-  if (warp == 0) {
+  if (warp < 4) {
+    // ================================================================ warpgroup 0
+    regs_dec<REGS_PRODUCER>();
+    if (warp == 0) {
     // ================================================================ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmq);
       prefetch_tmap(&tmk);
       prefetch_tmap(&tmv);
     }
-    const uint64_t pol = policy_evict_last();  // a chunk's K/V is re-read by every M-tile of the chunk
+    const uint64_t pol = policy_evict_last();  // a chunk's K/V is re-read by every item of the chunk
     uint32_t items = 0, tcount = 0;  // tiles issued over all items (stage and phase bookkeeping)
     for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x, ++items) {
       Item it;
-      if (!chunk_item(p, TOK, idx, it)) break;
-      const int nt = item_tiles(it, TOK);
+      if (!chunk_item(p, PAIR, idx, it)) break;
+      const int nt = item_tiles(it, PAIR);
       const int nblk_ctx = (it.ctx + p.block_size - 1) / p.block_size;
       const int32_t* table = p.block_tables + static_cast<long long>(it.s) * p.max_blocks;
       // lane b < 8 owns the b-th 16-key group of a tile: block id and row offset in the block
@@ -276,12 +324,15 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       int blk_cur, y_cur, blk_prev = -1, y_prev = 0, blk_next, y_next;
       tile_ids(0, blk_cur, y_cur);
       tile_ids(1, blk_next, y_next);
-      // the previous item's last QK^T has read Q
+      // the previous item's last QK^T has read both Q tiles
       if (items > 0 && !ch_wait(sh, &sh.q_empty, (items - 1) & 1, p.status)) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&sh.q_full, Q_BYTES);
-        tma_load_3d(smem + SMEM_Q, &tmq, &sh.q_full, 0, it.kvh * G, it.q0 + it.tb * TOK);
-        tma_load_3d(smem + SMEM_Q + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, it.q0 + it.tb * TOK);
+        const int t0 = it.q0 + it.tp * PAIR;
+        mbar_arrive_expect_tx(&sh.q_full, 2 * Q_BYTES);
+        tma_load_3d(smem + SMEM_Q, &tmq, &sh.q_full, 0, it.kvh * G, t0);
+        tma_load_3d(smem + SMEM_Q + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0);
+        tma_load_3d(smem + SMEM_Q + Q_BYTES, &tmq, &sh.q_full, 0, it.kvh * G, t0 + TOK);
+        tma_load_3d(smem + SMEM_Q + Q_BYTES + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0 + TOK);
       }
       auto load_tile = [&](const CUtensorMap* tm, uint64_t* bars_full, uint64_t* bars_empty, int nst, int base_off,
                            uint32_t t, int blk, int y) -> bool {
@@ -327,106 +378,121 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
     // ================================================================ MMA issuer
     const uint32_t idesc_qk = umma_idesc(CH_M, CH_N, 0, 0);
     const uint32_t idesc_pv = umma_idesc(CH_M, CH_D, 0, 1);
-    const uint32_t sq = smem_u32(smem + SMEM_Q), sp = smem_u32(smem + SMEM_P);
-    uint32_t q_phase = 0, p_phase = 0, o_phase = 0, s_use[2] = {0, 0}, kv_count = 0;
+    const uint32_t sq = smem_u32(smem + SMEM_Q);
+    uint32_t q_phase = 0, p_phase[2] = {0, 0}, o_phase = 0, kv_count = 0;
     bool first_item = true;
     for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x) {
       Item it;
-      if (!chunk_item(p, TOK, idx, it)) break;
-      const int nt = item_tiles(it, TOK);
+      if (!chunk_item(p, PAIR, idx, it)) break;
+      const int nt = item_tiles(it, PAIR);
       if (!ch_wait(sh, &sh.q_full, q_phase, p.status)) break;
       q_phase ^= 1;
-      if (!first_item) {  // the epilogue of the previous item has read O
-        if (!ch_wait(sh, &sh.o_empty, o_phase, p.status)) break;
+      if (!first_item) {  // both epilogues of the previous item have read O
+        if (!ch_wait(sh, &sh.o_empty[0], o_phase, p.status) || !ch_wait(sh, &sh.o_empty[1], o_phase, p.status))
+          break;
         o_phase ^= 1;
       }
       first_item = false;
-      bool ok = true;
-      auto qk = [&](int j) -> bool {
+      if (nt == 0) {  // nothing to multiply: Q is free, and each epilogue gets its one P V completion
+        if (lane == 0) {
+          umma_commit(&sh.q_empty);
+          umma_commit(&sh.pv_done[0]);
+          umma_commit(&sh.pv_done[1]);
+        }
+        __syncwarp();
+        continue;
+      }
+      // S_w(j) = Q_w K(j)^T.  S_w last held P_w(j - 1), which P V_w(j - 1)
+      // read: that MMA was issued before this one, and the MMAs of one CTA run
+      // in issue order.
+      auto qk = [&](int w, int j) -> bool {
         const int stage = (kv_count + j) % KST;
-        const uint32_t use = (kv_count + j) / KST;
-        if (!ch_wait(sh, &sh.k_full[stage], use & 1, p.status)) return false;
-        const int sb = j & 1;
-        if (s_use[sb] > 0 && !ch_wait(sh, &sh.s_empty[sb], (s_use[sb] - 1) & 1, p.status)) return false;
-        ++s_use[sb];
+        if (w == 0 && !ch_wait(sh, &sh.k_full[stage], ((kv_count + j) / KST) & 1, p.status)) return false;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sk = smem_u32(smem + SMEM_K + stage * KV_BYTES);
+          const uint32_t qw = sq + w * Q_BYTES;
 #pragma unroll
           for (int kk = 0; kk < CH_D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
-            umma_f16(tmem + sb * CH_N, umma_desc(sq + off, 16, 1024), umma_desc(sk + off, 16, 1024), idesc_qk,
+            umma_f16(tmem + w * CH_N, umma_desc(qw + off, 16, 1024), umma_desc(sk + off, 16, 1024), idesc_qk,
                      kk > 0);
           }
-          umma_commit(&sh.s_full[sb]);
-          umma_commit(&sh.k_empty[stage]);
-          if (j == nt - 1) umma_commit(&sh.q_empty);
+          umma_commit(&sh.s_full[w]);
+          if (w == 1) {
+            umma_commit(&sh.k_empty[stage]);
+            if (j == nt - 1) umma_commit(&sh.q_empty);
+          }
         }
         __syncwarp();
         return true;
       };
-      auto pv = [&](int j) -> bool {
-        if (!ch_wait(sh, &sh.p_full, p_phase, p.status)) return false;
-        p_phase ^= 1;
+      // O_w += P_w(j) V(j), P_w(j) in the first 64 columns of S_w
+      auto pv = [&](int w, int j) -> bool {
+        if (!ch_wait(sh, &sh.p_full[w], p_phase[w], p.status)) return false;
+        p_phase[w] ^= 1;
         const int stage = (kv_count + j) % VST;
-        if (!ch_wait(sh, &sh.v_full[stage], ((kv_count + j) / VST) & 1, p.status)) return false;
+        if (w == 0 && !ch_wait(sh, &sh.v_full[stage], ((kv_count + j) / VST) & 1, p.status)) return false;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sv = smem_u32(smem + SMEM_V + stage * KV_BYTES);
+          const uint32_t pt = tmem + w * CH_N;
 #pragma unroll
-          for (int kk = 0; kk < CH_N / 16; ++kk) {
-            // A = P (K-major, keys 16kk..), B = V (MN-major: 16 key rows from row 16kk, both head-dim panels)
-            umma_f16(tmem + TMEM_O, umma_desc(sp + (kk >> 2) * PANEL + (kk & 3) * 32, 16, 1024),
-                     umma_desc(sv + kk * 16 * 128, PANEL, 1024), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&sh.pv_done);
-          umma_commit(&sh.v_empty[stage]);
+          for (int kk = 0; kk < CH_N / 16; ++kk)  // keys 16kk.. = P columns 8kk..; V rows 16kk.., both panels
+            umma_f16_ts(tmem + TMEM_O + w * CH_N, pt + 8 * kk, umma_desc(sv + kk * 16 * 128, PANEL, 1024),
+                        idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&sh.pv_done[w]);
+          if (w == 1) umma_commit(&sh.v_empty[stage]);
         }
         __syncwarp();
         return true;
       };
-      if (nt > 0) ok = qk(0);
-      for (int j = 1; ok && j < nt; ++j) ok = qk(j) && pv(j - 1);
-      if (ok && nt > 0) ok = pv(nt - 1);
+      bool ok = qk(0, 0) && qk(1, 0);
+      for (int j = 1; ok && j < nt; ++j) ok = pv(0, j - 1) && qk(0, j) && pv(1, j - 1) && qk(1, j);
+      if (ok) ok = pv(0, nt - 1) && pv(1, nt - 1);
       kv_count += nt;
       if (!ok) break;
     }
+    }
   } else {
-    // ================================================================ softmax warpgroup
+    // ================================================================ softmax warpgroups
+    regs_inc<REGS_SOFTMAX>();
+    const int w = (warp >> 2) - 1;        // 0: M-tile A, 1: M-tile B
     const int quad = warp & 3;            // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;     // query row of the M-tile = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t s_col = tmem + lane_addr + w * CH_N, o_col = tmem + lane_addr + TMEM_O + w * CH_N;
     const int tok_in_tile = row / G, head_in_group = row % G;
-    uint32_t s_phase[2] = {0, 0}, pv_phase = 0, kv_count = 0;
-    uint8_t* pbuf = smem + SMEM_P;
+    // kv_count: key tiles of earlier items (V stages); pv_count: completions
+    // of pv_done[w] so far (one per tile, one for an item without tiles)
+    uint32_t s_phase = 0, kv_count = 0, pv_count = 0;
     for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x) {
       Item it;
-      if (!chunk_item(p, TOK, idx, it)) break;
-      const int nt = item_tiles(it, TOK);
-      const int tok = it.tb * TOK + tok_in_tile;       // row's token within the chunk
-      const int last_key = it.p0 + tok;                // causal limit (inclusive)
+      if (!chunk_item(p, PAIR, idx, it)) break;
+      const int nt = item_tiles(it, PAIR);
+      const int tok = it.tp * PAIR + w * TOK + tok_in_tile;  // row's token within the chunk
+      const int last_key = it.p0 + tok;                       // causal limit (inclusive)
       const bool row_valid = tok < it.qlen && last_key >= 0;
+      const int tile_last = it.p0 + it.tp * PAIR + w * TOK;   // first row of this M-tile: keys beyond it are
+                                                              // masked for some row of the tile
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < nt && ok; ++j) {
-        const int sb = j & 1;
-        if (!(ok = ch_wait(sh, &sh.s_full[sb], s_phase[sb], p.status))) break;
-        s_phase[sb] ^= 1;
+        if (!(ok = ch_wait(sh, &sh.s_full[w], s_phase, p.status))) break;
+        s_phase ^= 1;
         tc_fence_after();
         float s[CH_N];
 #pragma unroll
         for (int c = 0; c < CH_N / 32; ++c) {
           float v[32];
-          tmem_ld32(tmem + lane_addr + sb * CH_N + c * 32, v);
+          tmem_ld32(s_col + c * 32, v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[c * 32 + i] = v[i];
         }
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&sh.s_empty[sb]);
 
         const int key0 = j * CH_N;
-        const bool diag = key0 + CH_N - 1 > it.p0 + it.tb * TOK;  // some row of the tile stops inside it
+        const bool diag = key0 + CH_N - 1 > tile_last;  // some row of the tile stops inside (or before) it
         const float cs = p.scale_log2;
         // Off the diagonal every key is visible: take the max of the raw scores
         // and fold the scale into one FFMA per element below.  On a diagonal
@@ -450,75 +516,70 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
           if (!diag) mx *= cs;
         }
-        // Decide the reference maximum, compute P in registers (this overlaps the
-        // previous tile's P V on the tensor cores), and only then wait for that
-        // P V before P's shared memory is rewritten or O is rescaled.
         const bool rescale = mx > m_ref + RESCALE_LOG2 || m_ref == -INFINITY;
         const float m_new = rescale ? fmaxf(mx, m_ref) : m_ref;
-        uint32_t pk[CH_N / 2];
+        // P in bf16 pairs (keys 2c, 2c + 1 in column c), straight into S_w
+        const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;  // a row with no key yet: P = 0, not NaN
         float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const float neg_m = -m_new;
 #pragma unroll
-        for (int i = 0; i < CH_N / 2; ++i) {
-          const float x0 = s[2 * i], x1 = s[2 * i + 1];
-          const float a = fast_exp2(diag ? x0 + neg_m : fmaf(x0, cs, neg_m));
-          const float b = fast_exp2(diag ? x1 + neg_m : fmaf(x1, cs, neg_m));
-          l8[i & 7] += a + b;
-          pk[i] = pack_bf16x2(a, b);
+        for (int c = 0; c < CH_N / 64; ++c) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float x0 = s[64 * c + 2 * i], x1 = s[64 * c + 2 * i + 1];
+            const float a = fast_exp2(diag ? x0 + neg_m : fmaf(x0, cs, neg_m));
+            const float b = fast_exp2(diag ? x1 + neg_m : fmaf(x1, cs, neg_m));
+            l8[i & 7] += a + b;
+            pk[i] = pack_bf16x2(a, b);
+          }
+          tmem_st32u(s_col + 32 * c, pk);
         }
-        if (j > 0) {
-          if (!(ok = ch_wait(sh, &sh.pv_done, pv_phase, p.status))) break;
-          pv_phase ^= 1;
+        const bool resc = rescale && m_ref != -INFINITY;
+        const float alpha = resc ? fast_exp2(m_ref - m_new) : 1.f;
+        l = l * alpha + (((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7])));
+        m_ref = m_new;
+        // O holds tiles 0..j-1: wait for P V_w(j - 1), then scale O in tensor
+        // memory.  tcgen05.ld/st are warp-collective, so the whole warp takes
+        // this branch when any of its rows rescales (the others scale by 1).
+        if (j > 0 && __any_sync(FULL_MASK, resc)) {
+          // pv_done[w] completes once per tile; P V_w(j) cannot have completed
+          // (it waits for this thread's P), so the parity names the phase
+          if (!(ok = ch_wait(sh, &sh.pv_done[w], (pv_count + j - 1) & 1, p.status))) break;
           tc_fence_after();
-        }
-        if (rescale && m_ref != -INFINITY) {
-          const float alpha = fast_exp2(m_ref - m_new);
-          l *= alpha;
-          if (j > 0) {  // O holds tiles 0..j-1: scale it in tensor memory
 #pragma unroll
-            for (int c = 0; c < CH_D / 32; ++c) {
-              float v[32];
-              tmem_ld32(tmem + lane_addr + TMEM_O + c * 32, v);
-              tmem_wait_ld();
+          for (int c = 0; c < CH_D / 32; ++c) {
+            float v[32];
+            tmem_ld32(o_col + c * 32, v);
+            tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] *= alpha;
-              tmem_st32(tmem + lane_addr + TMEM_O + c * 32, v);
-            }
-            tmem_wait_st();
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tmem_st32(o_col + c * 32, v);
           }
         }
-        m_ref = m_new;
-        l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) + ((l8[4] + l8[5]) + (l8[6] + l8[7]));
-        // P (bf16), row `row` of the K-major SW128 A panels
-#pragma unroll
-        for (int c8 = 0; c8 < CH_N / 8; ++c8) {
-          uint8_t* dst = pbuf + (c8 >> 3) * PANEL + sw128(row, c8 & 7);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2], pk[4 * c8 + 3]);
-        }
+        tmem_wait_st();
         // keys past the context may hold anything (even NaN): zero their V rows
+        // (M-tile A's warpgroup does it; P V_B(j) is issued after P V_A(j))
         const int valid_keys = it.ctx - key0;
-        if (valid_keys < CH_N) {
+        if (w == 0 && valid_keys < CH_N) {
           const int stage = (kv_count + j) % VST;
           if (!(ok = ch_wait(sh, &sh.v_full[stage], ((kv_count + j) / VST) & 1, p.status))) break;
           uint8_t* vst = smem + SMEM_V + stage * KV_BYTES;
           const int nz = (CH_N - max(valid_keys, 0)) * 2 * 8;  // 16-byte chunks in both panels
-          for (int k = threadIdx.x - 64; k < nz; k += 128) {
+          for (int k = threadIdx.x - 128; k < nz; k += 128) {
             const int r = max(valid_keys, 0) + k / 16, rest = k % 16;
             *reinterpret_cast<uint4*>(vst + (rest >> 3) * PANEL + r * 128 + (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
           }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&sh.p_full);
+        mbar_arrive(&sh.p_full[w]);
       }
       kv_count += nt;
+      pv_count += nt > 0 ? nt : 1;
       if (!ok) break;
-      // ---- epilogue: O / l -> bf16 -> out
-      if (nt > 0) {
-        if (!ch_wait(sh, &sh.pv_done, pv_phase, p.status)) break;
-        pv_phase ^= 1;
-        tc_fence_after();
-      }
+      // ---- epilogue: O / l -> bf16 -> out (after the item's last pv_done completion)
+      if (!ch_wait(sh, &sh.pv_done[w], (pv_count - 1) & 1, p.status)) break;
+      tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
                             (static_cast<long long>(it.q0 + tok) * p.num_q_heads + it.kvh * G + head_in_group) * CH_D;
@@ -526,7 +587,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       for (int c = 0; c < CH_D / 32; ++c) {
         float v[32];
         if (nt > 0) {
-          tmem_ld32(tmem + lane_addr + TMEM_O + c * 32, v);
+          tmem_ld32(o_col + c * 32, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -535,17 +596,17 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         if (row_valid) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(v[i] * inv, v[i + 1] * inv);
-            w.y = pack_bf16x2(v[i + 2] * inv, v[i + 3] * inv);
-            w.z = pack_bf16x2(v[i + 4] * inv, v[i + 5] * inv);
-            w.w = pack_bf16x2(v[i + 6] * inv, v[i + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + i) = w;
+            uint4 u;
+            u.x = pack_bf16x2(v[i] * inv, v[i + 1] * inv);
+            u.y = pack_bf16x2(v[i + 2] * inv, v[i + 3] * inv);
+            u.z = pack_bf16x2(v[i + 4] * inv, v[i + 5] * inv);
+            u.w = pack_bf16x2(v[i + 6] * inv, v[i + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + i) = u;
           }
         }
       }
       tc_fence_before();
-      mbar_arrive(&sh.o_empty);
+      mbar_arrive(&sh.o_empty[w]);
     }
   }
 

@@ -122,6 +122,26 @@ def test_small_shapes_match_oracle(case):
     assert int(ds.status.item()) == 0
 
 
+def test_late_large_scores_rescale_some_rows_of_a_tile():
+    # one key deep in the prefix gets 40x the usual magnitude: for about half
+    # the query rows its score raises the running maximum far above the
+    # earlier tiles' (the others see a very negative score), so the rescale of
+    # O runs for some rows of a tile and not for others -- on the tensor-core
+    # chunk path (G 8) and on the rows path (G 6, head_dim 64)
+    from paged_kv_cache_445_b200.workloads import bf16_bits_to_f32, f32_to_bf16_bits
+    for prefix, qlen, hq, hkv, d, bs in (([870, 39], [130, 1], 16, 2, 128, 32), ([500, 20], [60, 1], 12, 2, 64, 16)):
+        w = workloads.custom(prefix, qlen, hq, hkv, d, bs, seed=12, poison=True)
+        pos = 300
+        blk, off = int(w.block_tables[0, pos // bs]), pos % bs
+        row = bf16_bits_to_f32(w.k_cache[blk, :, off, :]) * 40.0
+        w.k_cache[blk, :, off, :] = f32_to_bf16_bits(row)
+        ds = DeviceStep(w)
+        got = ds.step()
+        kc, vc = oracle_after_append(w)
+        compare(got, _attend_ref(w, kc, vc), f"large late score, d{d}")
+        assert int(ds.status.item()) == 0
+
+
 def test_varlen_entry_on_a_pure_decode_batch_matches_decode_entry():
     w = workloads.custom([30, 700, 4000], [1, 1, 1], 16, 2, 128, 16, seed=3, poison=True)
     a = DeviceStep(w).step()
@@ -154,6 +174,27 @@ def test_results_are_deterministic_and_workspace_is_reusable():
         outs.append(ds.out.float().cpu().numpy())
         compare(outs[-1], ref, "repeated call")
         assert int(ds.status.item()) == 0
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+
+
+def test_large_batch_with_claimed_tail_chunks_is_exact_and_deterministic():
+    # at least 16 tiles per launched warp: the last 3/16 of the tiles are
+    # handed out at run time in fixed chunks; whichever warp takes a chunk,
+    # the pieces and therefore the bits must be the same
+    ctx = [5000, 7000, 3000, 6000, 4500, 8000, 2500, 6500, 1, 17]
+    w = workloads.custom([c - 1 for c in ctx], [1] * len(ctx), 64, 8, 128, 16, seed=11, poison=True)
+    ds = DeviceStep(w)
+    ds.append()
+    kc, vc = oracle_after_append(w)
+    ref = _attend_ref(w, kc, vc)
+    outs = []
+    for _ in range(3):
+        ds.attend()
+        torch.cuda.synchronize()
+        assert int(ds.status.item()) == 0
+        outs.append(ds.out.float().cpu().numpy())
+    compare(outs[0], ref, "tail chunks")
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
 
