@@ -233,7 +233,11 @@ def step_bytes(w):
 
 
 class GpuStep:
-    def __init__(self, w, device):
+    """One workload resident on the GPU.  A decode batch runs its step as one
+    fused launch (pa_decode_append) unless fused=False; a mixed batch runs
+    pa_cache_append then pa_prefill_chunk."""
+
+    def __init__(self, w, device, fused=True):
         import torch
 
         import paged_kv_cache_445_b200 as pa
@@ -254,12 +258,25 @@ class GpuStep:
                                            w.block_tables.shape[1], w.block_size, device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.decode = w.is_decode
+        self.fused = self.decode and fused
+        self.launches = 1 if self.fused else step_launches(w)  # kernel launches per step
+        # host-to-device inputs of one step (what e2e copies)
+        self.inputs = ["q", "k_new", "v_new", "block_tables", "context_lens"]
+        if not self.fused:
+            self.inputs.append("slot_mapping")
+        if not self.decode:
+            self.inputs.append("query_start")
 
     def append(self):
+        if self.fused:
+            return  # part of the attention launch
         self.pa.pa_cache_append(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping, self.status)
 
     def attend(self):
-        if self.decode:
+        if self.fused:
+            self.pa.pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.k_cache, self.v_cache,
+                                     self.block_tables, self.context_lens, self.w.scale, self.workspace, self.status)
+        elif self.decode:
             self.pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
                               self.w.scale, self.workspace, self.status)
         else:
@@ -277,7 +294,7 @@ def run_ours(args, peaks):
     w = workloads.standard(args.workload, seed=rank_seed(args.workload, rank))
     log(f"[rank {rank}] workload {w.name}: {w.num_seqs} seqs, {w.num_query_tokens} query rows, "
         f"{int(w.context_lens.sum())} keys, pool {w.num_blocks} blocks ({time.time() - t0:.1f}s to generate)")
-    g = GpuStep(w, device)
+    g = GpuStep(w, device, fused=not args.separate_append)
     kv_bytes, attn_bytes, app_bytes, flops = step_bytes(w)
     stream = torch.cuda.current_stream()
 
@@ -312,16 +329,13 @@ def run_ours(args, peaks):
         raise SystemExit(f"device status {int(g.status.item())} after timing")
 
     # ---- end to end through the public calls with host buffers
-    pin = {name: getattr(g, name).cpu().pin_memory() for name in
-           ("q", "k_new", "v_new", "slot_mapping", "block_tables", "context_lens", "query_start")}
+    pin = {name: getattr(g, name).cpu().pin_memory() for name in g.inputs}
     out_host = torch.empty(g.out.shape, dtype=g.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for k, t in pin.items() if g.decode is False or k != "query_start")
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = out_host.numel() * out_host.element_size()
 
     def e2e_step():
         for k, t in pin.items():
-            if g.decode and k == "query_start":
-                continue
             getattr(g, k).copy_(t, non_blocking=True)
         g.append()
         g.attend()
@@ -350,7 +364,8 @@ def run_ours(args, peaks):
 
     clocks = sampler.summary()
     hbm, bf16_burst, bf16_sust, peak_src = peaks
-    achieved = attn_bytes / (attn_avg_ms * 1e-3) / 1e9
+    launch_bytes = attn_bytes + (app_bytes if g.fused else 0)  # the timed launch also appends when fused
+    achieved = launch_bytes / (attn_avg_ms * 1e-3) / 1e9
     traffic = profiled_traffic("pa_rows_kernel", w.name)
     line = {
         "metric": "paged-attn decode KV GB/s + seq-steps/s (70B layer, bs128); % of HBM peak",
@@ -375,17 +390,18 @@ def run_ours(args, peaks):
         "frac_of_hbm_peak": round(compose_value(total_kv, ms_step) / hbm / world, 4),
         "frac_of_8tbs_nominal": round(compose_value(total_kv, ms_step) / 8000.0 / world, 4),
         "roofline": {
-            "kernel": "pa_rows_kernel (attention)", "bound": "hbm",
+            "kernel": "pa_rows_kernel (append + attention, one launch)" if g.fused else "pa_rows_kernel (attention)",
+            "bound": "hbm",
             "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_src == "measured" else "fallback 6.65 TB/s",
-            "traffic": traffic, "algorithmic_bytes_per_launch": attn_bytes,
+            "traffic": traffic, "algorithmic_bytes_per_launch": launch_bytes,
             "avg_launch_ms": round(attn_avg_ms, 5),
         },
         "append": {"algorithmic_bytes": app_bytes},
         "e2e": {"value": round(compose_value(total_kv, e2e_ms), 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": step_launches(w) * args.steps,
+        "gpu_launches": g.launches * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
@@ -490,11 +506,13 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="decode batches: pa_cache_append + pa_decode instead of the fused pa_decode_append")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

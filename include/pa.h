@@ -130,6 +130,30 @@ PA_API int pa_decode(void* out, const void* q, const void* k_cache, const void* 
               void* stream);
 
 /*
+ * pa_decode_append -- pa_cache_append of this step's rows followed by
+ * pa_decode, in one launch.  Row s of k_new / v_new ([num_seqs, num_kv_heads,
+ * head_dim] bf16) is the newest token of sequence s; it is written to
+ * position context_lens[s] - 1 through the block table (the slot the host
+ * allocator hands out for that token), and the attention uses it as that
+ * position's key and value.  Output and cache contents are bit-identical to
+ * the two separate calls with slot_mapping[s] = that slot.
+ *
+ * The pages describe the step as one fused call over the batch ("vLLM serving
+ * internals", "What the scheduler looks like") and the cache update as part
+ * of attention ("Inference optimization", "Build it -- Step 2": the layer
+ * stores the new keys and values, then attends over the cache).  Fusing saves
+ * the append's launch and lets its stores overlap the attention's loads.
+ *
+ * k_cache / v_cache are written.  A block ID outside the pool skips that
+ * store and sets the RANGE bit; everything else as pa_decode.
+ */
+PA_API int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                            void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                            const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                            int head_dim, int block_size, int num_blocks, float scale, void* workspace,
+                            size_t workspace_bytes, int* dev_status, void* stream);
+
+/*
  * pa_prefill_chunk -- attention for a varlen batch that mixes prefill chunks
  * and decodes in one call.  Sequence s contributes qlen = query_start[s+1] -
  * query_start[s] query rows: the LAST qlen positions of its context_lens[s]

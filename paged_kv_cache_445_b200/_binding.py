@@ -30,6 +30,9 @@ _lib.pa_decode.restype = _ci
 _lib.pa_prefill_chunk.argtypes = [_vp, _vp, _i32p, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci, _ci,
                                   ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
 _lib.pa_prefill_chunk.restype = _ci
+_lib.pa_decode_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
+                                  ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
+_lib.pa_decode_append.restype = _ci
 _lib.pa_decode_static_scratch.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                           ctypes.c_float, _vp, _vp]
 _lib.pa_decode_static_scratch.restype = _ci
@@ -149,6 +152,24 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, works
                           bs, nb, float(scale), ws, workspace.numel(), _status_ptr(dev_status), _stream_ptr(stream)))
 
 
+def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, context_lens, scale, workspace,
+                     dev_status=None, stream=None) -> None:
+    """pa_cache_append of each sequence's newest row (k_new / v_new [B, Hkv, d],
+    written at position context_lens[s] - 1 through the block table) and
+    pa_decode, in one launch; see include/pa.h."""
+    op, qp, kc, vc, bt, cl, ws = _attention_args(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    kn = _dev(k_new, "k_new", torch.bfloat16, 3)
+    vn = _dev(v_new, "v_new", torch.bfloat16, 3)
+    nb, hkv, bs, d = k_cache.shape
+    if q.shape[0] != context_lens.shape[0]:
+        raise ValueError("pa_decode_append takes exactly one query row per sequence")
+    if k_new.shape != (context_lens.shape[0], hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("k_new / v_new must be [num_seqs, Hkv, d]")
+    _check(_lib.pa_decode_append(op, qp, kn, vn, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0],
+                                 q.shape[1], hkv, d, bs, nb, float(scale), ws, workspace.numel(),
+                                 _status_ptr(dev_status), _stream_ptr(stream)))
+
+
 def pa_prefill_chunk(out, q, query_start, k_cache, v_cache, block_tables, context_lens, scale, workspace,
                      dev_status=None, stream=None) -> None:
     """Varlen batch of prefill chunks and decodes: q/out [Tq, Hq, d],
@@ -194,5 +215,5 @@ def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_len
 
 
 def exported_symbols() -> list[str]:
-    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_prefill_chunk", "pa_decode_static_scratch",
-            "pa_status_string"]
+    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_decode_append", "pa_prefill_chunk",
+            "pa_decode_static_scratch", "pa_status_string"]

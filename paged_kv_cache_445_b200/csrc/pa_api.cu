@@ -86,8 +86,12 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                          const void* v_cache, const int32_t* block_tables, int max_blocks,
                          const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
-                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+                         void* workspace, size_t workspace_bytes, int* dev_status, void* stream,
+                         const void* k_new, const void* v_new) {
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace) return PA_ERR_NULL;
+  if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
+  if (k_new && query_start) return PA_ERR_UNSUPPORTED;  // the fused append serves one-row (decode) batches
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PA_ERR_SHAPE;
   int rc = check_attention_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks);
   if (rc != PA_OK) return rc;
   if (total_q_tokens < 0) return PA_ERR_SHAPE;
@@ -120,6 +124,10 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
   p.scale_log2 = scale * 1.4426950408889634f;
   rows_workspace_layout(workspace, total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms, &p);
   p.status = dev_status;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_cache = const_cast<void*>(k_cache);
+  p.v_cache = const_cast<void*>(v_cache);
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (query_start && chunk_supported(p.group, head_dim)) {
     // sequences with more than one query row run on the tcgen05 chunk kernel,
@@ -183,6 +191,16 @@ int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache
   return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                            num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                            workspace, workspace_bytes, dev_status, stream);
+}
+
+int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                     const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                     int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                     void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!k_new || !v_new) return PA_ERR_NULL;
+  return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                           num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                           workspace, workspace_bytes, dev_status, stream, k_new, v_new);
 }
 
 int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,

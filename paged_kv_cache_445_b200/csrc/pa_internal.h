@@ -39,6 +39,14 @@ struct RowsParams {
   int num_rows;                // query rows (Tq)
   int* status;      // optional device status word
   int total_warps;
+  // Fused cache append (decode only; nullptr: none).  Row s of k_new / v_new
+  // ([B, Hkv, D] bf16) is sequence s's newest token: the kernel writes it to
+  // position context_lens[s] - 1 through the block table and attends to it
+  // from these rows, not from the cache.
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
 };
 
 // Parameters of the tcgen05 chunk kernel (sequences with more than one query row).
@@ -94,6 +102,6 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                   const int32_t* block_tables, int max_blocks, const int32_t* context_lens, int num_seqs,
                   int total_q_tokens, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                   int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
-                  void* stream);
+                  void* stream, const void* k_new = nullptr, const void* v_new = nullptr);
 
 }  // namespace pa

@@ -319,6 +319,36 @@ __device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, 
   store_output<D, NT>(p, acc, ll, row, kvh, lane);
 }
 
+// Fused cache append (decode): write row s of k_new / v_new, sequence s's
+// newest token, to position context_lens[s] - 1 of its block table, every KV
+// head, 16-byte vectors over the whole grid.  The attention does not read
+// these bytes back (it takes the newest key from k_new / v_new), so nothing
+// waits for the stores.
+template <int D>
+__device__ __forceinline__ void fused_append(const RowsParams& p, long long tid, long long nthreads) {
+  constexpr int VEC = D / 8;
+  const long long n = static_cast<long long>(p.num_seqs) * p.num_kv_heads * VEC;
+  for (long long i = tid; i < n; i += nthreads) {
+    const int v = static_cast<int>(i % VEC);
+    const long long sh = i / VEC;
+    const int h = static_cast<int>(sh % p.num_kv_heads), s = static_cast<int>(sh / p.num_kv_heads);
+    const int ctx = __ldg(p.context_lens + s);
+    if (ctx < 1) continue;
+    const int pos = ctx - 1, lb = pos / p.block_size;
+    if (lb >= p.max_blocks) continue;  // reported by the attention's own length check
+    const int blk = __ldg(p.block_tables + static_cast<long long>(s) * p.max_blocks + lb);
+    if (blk < 0 || blk >= p.num_blocks) {
+      set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+      continue;
+    }
+    const long long src = sh * VEC + v;
+    const long long dst = ((static_cast<long long>(blk) * p.num_kv_heads + h) * p.block_size + pos % p.block_size) *
+                              VEC + v;
+    reinterpret_cast<uint4*>(p.k_cache)[dst] = __ldg(reinterpret_cast<const uint4*>(p.k_new) + src);
+    reinterpret_cast<uint4*>(p.v_cache)[dst] = __ldg(reinterpret_cast<const uint4*>(p.v_new) + src);
+  }
+}
+
 // What the consumer needs to know about the tile in a ring stage; written by
 // the issuing lane before the TMA, read by the warp after the stage completes.
 struct TileMeta {
@@ -453,9 +483,15 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
     };
 
     for (int k = 0; k < R && loading; ++k) issue(k);
+    // the first tiles are in flight: do this thread's share of the fused append meanwhile
+    if (p.k_new)
+      fused_append<D>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
+                      static_cast<long long>(gridDim.x) * ROWS_THREADS);
 
     float o[KT][NT][4];
     uint32_t qb[NT][KT][2];
+    constexpr int NEWV = (2 * D / 8 + 31) / 32;  // 16-byte vectors of the newest K and V row per lane
+    uint4 newkv[NEWV];
     float m[NT][2], l[NT][2];
     bool began = false;
     int piece_t0 = 0;
@@ -474,6 +510,17 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       if (tm.t == 0 || run_start) {  // a piece starts: load the G query rows of this KV head
         began = (tm.t == 0);
         piece_t0 = tm.t;
+        if (p.k_new) {  // fused append: the segment's newest key and value come from k_new / v_new
+#pragma unroll
+          for (int k = 0; k < NEWV; ++k) {
+            const int c = lane + 32 * k;
+            if (c < 2 * D / 8) {
+              const uint4* src = reinterpret_cast<const uint4*>(c < D / 8 ? p.k_new : p.v_new) +
+                                 (static_cast<long long>(tm.row) * p.num_kv_heads + tm.h) * (D / 8) + c % (D / 8);
+              newkv[k] = __ldg(src);
+            }
+          }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int head = nt * 8 + g;
@@ -496,6 +543,20 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       uint8_t* kt = ring + stage * S::STAGE_BYTES;
       uint8_t* vt = kt + S::HALF_BYTES;
       const int nvalid = min(TILE_KEYS, tm.nkeys - tm.t * TILE_KEYS);
+      if (p.k_new && tm.t == tm.n - 1) {
+        // the newest key is row nvalid - 1 of this tile: overwrite what the
+        // copy brought (the append of this very launch may not have landed)
+#pragma unroll
+        for (int k = 0; k < NEWV; ++k) {
+          const int c = lane + 32 * k;
+          if (c < 2 * D / 8) {
+            const int idx = c % (D / 8);
+            *reinterpret_cast<uint4*>((c < D / 8 ? kt : vt) + (idx >> 3) * 2048 + sw128(nvalid - 1, idx & 7)) =
+                newkv[k];
+          }
+        }
+        __syncwarp();
+      }
 
       // Pull the tile into registers (K as the A operand of S^T = K Q^T, V^T via
       // ldmatrix.trans as the A operand of O^T += V^T P^T) and hand the stage
@@ -659,6 +720,10 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       for (long long j = stopped_at + 1; j < issued; ++j) mbar_wait(&bar[j % R], static_cast<uint32_t>((j / R) & 1));
     }
   }
+
+  if (gw >= W && p.k_new)  // warps without tiles still take their share of the fused append
+    fused_append<D>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
+                    static_cast<long long>(gridDim.x) * ROWS_THREADS);
 
   // ---- grid barrier: every partial and table entry is stored before any merge reads it
   __syncwarp();

@@ -143,13 +143,18 @@ def _lengths(cfg: int, rng: np.random.Generator):
     if cfg == 5:
         ctx = rng.integers(256, 8192, size=127, endpoint=True)
         return (16384,) + tuple(ctx - 1), (512,) + (1,) * 127
+    if cfg == 6:  # the 70B-like length mix, each sequence verifying 4 draft tokens
+        ctx = np.clip(np.round(rng.lognormal(math.log(1500.0), 0.8, size=128)), 16, 8192).astype(np.int64)
+        return tuple(ctx - 4), (4,) * 128
     raise ValueError(f"unknown workload {cfg}")
 
 
 def standard_spec(cfg: int, seed: int | None = None) -> Spec:
-    """The five standard workloads (1 tiny decode, 2 Llama-3-8B-like decode,
+    """The standard workloads (1 tiny decode, 2 Llama-3-8B-like decode,
     3 Llama-3.3-70B-like decode at concurrency 128, 4 GRPO shared-prefix decode,
-    5 mixed 512-token prefill chunk + 127 decodes)."""
+    5 mixed 512-token prefill chunk + 127 decodes, 6 the workload-3 layer
+    verifying 4 draft tokens per sequence, as speculative decoding does --
+    "Inference optimization", section "Speculative decoding")."""
     seed = 445 + cfg if seed is None else seed
     rng = np.random.Generator(np.random.PCG64(seed))
     prefix, new = _lengths(cfg, rng)
@@ -163,7 +168,9 @@ def standard_spec(cfg: int, seed: int | None = None) -> Spec:
         groups = (tuple(range(16)), tuple(range(16, 32)))
         return Spec("grpo-shared-prefix-decode-2x16", 24, 4, 256, 32, prefix, new,
                     share=groups, share_tokens=2048)
-    return Spec("mixed-prefill512-plus-127-decodes", 64, 8, 128, 16, prefix, new)
+    if cfg == 5:
+        return Spec("mixed-prefill512-plus-127-decodes", 64, 8, 128, 16, prefix, new)
+    return Spec("llama3.3-70b-layer-verify4-b128", 64, 8, 128, 16, prefix, new, q_std=0.5)
 
 
 def build(spec: Spec, seed: int, poison: bool = False, max_blocks: int | None = None) -> Workload:

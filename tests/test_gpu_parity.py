@@ -30,7 +30,7 @@ def _attend_ref(w, kc, vc, only=None):
 
 # ------------------------------------------------------------------ append
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4, 5, 6])
 def test_append_is_bit_exact_on_the_standard_workloads(cfg):
     w = workloads.standard(cfg, poison=True)
     ds = DeviceStep(w)
@@ -91,6 +91,22 @@ def test_mixed_chunk_and_decodes_match_oracle():
     assert int(ds.status.item()) == 0
 
 
+def test_verify4_batch_matches_oracle_on_sampled_rows():
+    # 128 sequences of the 70B-like mix, 4 query rows each (speculative verification)
+    w = workloads.standard(6, poison=True)
+    ds = DeviceStep(w)
+    got = ds.step()
+    kc, vc = oracle_after_append(w)
+    rng = np.random.default_rng(6)
+    seqs = sorted({0, 1, 2, 127, *rng.integers(0, 128, 12).tolist()})
+    only = sorted({(t, h) for s in seqs for t in range(int(w.query_start[s]), int(w.query_start[s + 1]))
+                   for h in range(w.num_q_heads)})
+    ref = _attend_ref(w, kc, vc, only=np.array(only))
+    idx = tuple(np.array(only).T)
+    compare(got[idx], ref[idx], "verify-4 sampled rows")
+    assert int(ds.status.item()) == 0
+
+
 SMALL = [  # ctx list, qlen list, Hq, Hkv, d, bs
     ([1, 15, 16, 17, 33, 100, 257], [1] * 7, 8, 1, 128, 16),
     ([1, 31, 32, 33, 65, 300], [1] * 6, 8, 4, 64, 32),
@@ -140,6 +156,38 @@ def test_late_large_scores_rescale_some_rows_of_a_tile():
         kc, vc = oracle_after_append(w)
         compare(got, _attend_ref(w, kc, vc), f"large late score, d{d}")
         assert int(ds.status.item()) == 0
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+def test_fused_append_decode_equals_the_two_calls_bit_for_bit(cfg):
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.standard(cfg, poison=True)
+    two = DeviceStep(w)
+    two.step()
+    one = DeviceStep(w)
+    pa.pa_decode_append(one.out, one.q, one.k_new, one.v_new, one.k_cache, one.v_cache, one.block_tables,
+                        one.context_lens, w.scale, one.workspace, one.status)
+    torch.cuda.synchronize()
+    assert int(one.status.item()) == 0
+    assert torch.equal(one.out.view(torch.int16), two.out.view(torch.int16))
+    assert torch.equal(one.k_cache.view(torch.int16), two.k_cache.view(torch.int16))
+    assert torch.equal(one.v_cache.view(torch.int16), two.v_cache.view(torch.int16))
+    if cfg == 1:
+        kc, vc = oracle_after_append(w)
+        compare(one.out.float().cpu().numpy(), _attend_ref(w, kc, vc), "fused append, tiny")
+
+
+def test_fused_append_reports_a_bad_block_and_keeps_going():
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.custom([40, 60, 7], [1, 1, 1], 8, 2, 128, 16, seed=13)
+    ds = DeviceStep(w)
+    bt = w.block_tables.copy()
+    bt[1, 60 // 16] = w.num_blocks + 3  # the newest token's block is outside the pool
+    ds.block_tables = i32(bt)
+    pa.pa_decode_append(ds.out, ds.q, ds.k_new, ds.v_new, ds.k_cache, ds.v_cache, ds.block_tables,
+                        ds.context_lens, w.scale, ds.workspace, ds.status)
+    torch.cuda.synchronize()
+    assert int(ds.status.item()) & pa.status_bit(pa._binding.PA_ERR_RANGE)
 
 
 def test_varlen_entry_on_a_pure_decode_batch_matches_decode_entry():

@@ -159,7 +159,7 @@ def test_standard_tiny_workload_shape():
     assert w.scale == pytest.approx(1 / 8)
 
 
-@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5, 6])
 def test_standard_workload_specs(cfg):
     spec = workloads.standard_spec(cfg)
     ctx = np.array(spec.prefix) + np.array(spec.new)
@@ -174,6 +174,8 @@ def test_standard_workload_specs(cfg):
     if cfg == 5:
         assert spec.new[0] == 512 and spec.prefix[0] == 16384 and len(ctx) == 128
         assert (ctx[1:] >= 256).all() and (ctx[1:] <= 8192).all()
+    if cfg == 6:
+        assert len(ctx) == 128 and set(spec.new) == {4} and ctx.min() >= 16 and ctx.max() <= 8192
 
 
 def test_poisoned_workload_marks_every_invalid_slot():
