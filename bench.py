@@ -62,7 +62,7 @@ def measured_peaks():
 
 KERNEL_SOURCES = {  # the files whose text decides each kernel's code
     "pa_rows_kernel": ("pa_rows.cu", "pa_device.cuh"),
-    "pa_chunk_kernel": ("pa_chunk.cu", "pa_device.cuh"),
+    "pa_chunk_kernel": ("pa_chunk.cu", "pa_device.cuh", "pa_umma.cuh"),
 }
 
 
@@ -237,7 +237,7 @@ class GpuStep:
     fused launch (pa_decode_append) unless fused=False; a mixed batch runs
     pa_cache_append then pa_prefill_chunk."""
 
-    def __init__(self, w, device, fused=True):
+    def __init__(self, w, device, fused=True, cascade=True):
         import torch
 
         import paged_kv_cache_445_b200 as pa
@@ -254,12 +254,23 @@ class GpuStep:
         self.block_tables, self.context_lens = i32(w.block_tables), i32(w.context_lens)
         self.query_start, self.slot_mapping = i32(w.query_start), i32(w.slot_mapping)
         self.out = torch.empty_like(self.q)
-        self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim,
-                                           w.block_tables.shape[1], w.block_size, device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.decode = w.is_decode
         self.fused = self.decode and fused
-        self.launches = 1 if self.fused else step_launches(w)  # kernel launches per step
+        groups = w.prefix_groups() if self.decode and cascade else None
+        self.cascade = groups is not None
+        if self.cascade:  # shared prefixes read once per group (pa_decode_cascade)
+            self.group_start, self.group_prefix = i32(groups[0]), i32(groups[1])
+            self.workspace = pa.make_cascade_workspace(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                                       w.block_tables.shape[1], w.block_size, device)
+        else:
+            self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                               w.block_tables.shape[1], w.block_size, device)
+        # kernel launches per step
+        if self.cascade:
+            self.launches = 2 if self.fused else 3
+        else:
+            self.launches = 1 if self.fused else step_launches(w)
         # host-to-device inputs of one step (what e2e copies)
         self.inputs = ["q", "k_new", "v_new", "block_tables", "context_lens"]
         if not self.fused:
@@ -273,7 +284,12 @@ class GpuStep:
         self.pa.pa_cache_append(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping, self.status)
 
     def attend(self):
-        if self.fused:
+        if self.cascade:
+            self.pa.pa_decode_cascade(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
+                                      self.context_lens, self.w.scale, self.group_start, self.group_prefix,
+                                      self.workspace, k_new=self.k_new if self.fused else None,
+                                      v_new=self.v_new if self.fused else None, dev_status=self.status)
+        elif self.fused:
             self.pa.pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.k_cache, self.v_cache,
                                      self.block_tables, self.context_lens, self.w.scale, self.workspace, self.status)
         elif self.decode:
@@ -294,7 +310,7 @@ def run_ours(args, peaks):
     w = workloads.standard(args.workload, seed=rank_seed(args.workload, rank))
     log(f"[rank {rank}] workload {w.name}: {w.num_seqs} seqs, {w.num_query_tokens} query rows, "
         f"{int(w.context_lens.sum())} keys, pool {w.num_blocks} blocks ({time.time() - t0:.1f}s to generate)")
-    g = GpuStep(w, device, fused=not args.separate_append)
+    g = GpuStep(w, device, fused=not args.separate_append, cascade=args.cascade)
     kv_bytes, attn_bytes, app_bytes, flops = step_bytes(w)
     stream = torch.cuda.current_stream()
 
@@ -364,6 +380,10 @@ def run_ours(args, peaks):
 
     clocks = sampler.summary()
     hbm, bf16_burst, bf16_sust, peak_src = peaks
+    from paged_kv_cache_445_b200 import roofline as _rl
+    unique_kv = _rl.unique_kv_bytes(w.block_tables, w.context_lens, w.block_size, w.num_kv_heads, w.head_dim)
+    if g.cascade:  # a shared prefix crosses HBM once: the algorithmic bytes are the unique ones
+        attn_bytes = attn_bytes - kv_bytes + unique_kv
     launch_bytes = attn_bytes + (app_bytes if g.fused else 0)  # the timed launch also appends when fused
     achieved = launch_bytes / (attn_avg_ms * 1e-3) / 1e9
     traffic = profiled_traffic("pa_rows_kernel", w.name)
@@ -383,6 +403,7 @@ def run_ours(args, peaks):
             "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "block_size": w.block_size,
             "num_blocks": w.num_blocks, "query_rows": w.num_query_tokens,
             "context_tokens": int(w.context_lens.sum()), "kv_bytes_per_step": kv_bytes,
+            "unique_kv_bytes_per_step": unique_kv,
             "l2": f"no flush: every step reads {kv_bytes / 1e9:.2f} GB of KV, larger than the 126 MB L2",
             "parallelism": f"dp{world} (independent batch per GPU)",
         },
@@ -390,7 +411,9 @@ def run_ours(args, peaks):
         "frac_of_hbm_peak": round(compose_value(total_kv, ms_step) / hbm / world, 4),
         "frac_of_8tbs_nominal": round(compose_value(total_kv, ms_step) / 8000.0 / world, 4),
         "roofline": {
-            "kernel": "pa_rows_kernel (append + attention, one launch)" if g.fused else "pa_rows_kernel (attention)",
+            "kernel": ("pa_cascade_kernel + pa_rows_kernel (shared prefixes once, then the private keys)"
+                       if g.cascade else
+                       "pa_rows_kernel (append + attention, one launch)" if g.fused else "pa_rows_kernel (attention)"),
             "bound": "hbm",
             "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
@@ -511,6 +534,9 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cascade", action="store_true",
+                    help="shared-prefix batches: pa_decode_cascade (each shared prefix read once per group) "
+                         "instead of plain decode")
     ap.add_argument("--separate-append", action="store_true",
                     help="decode batches: pa_cache_append + pa_decode instead of the fused pa_decode_append")
     args = ap.parse_args(argv)

@@ -154,6 +154,41 @@ PA_API int pa_decode_append(void* out, const void* q, const void* k_new, const v
                             size_t workspace_bytes, int* dev_status, void* stream);
 
 /*
+ * pa_decode_cascade -- pa_decode (optionally fused with the append, as
+ * pa_decode_append) for a batch in which groups of sequences share a prefix of
+ * the KV cache, as copy-on-write forks of one prompt do ("vLLM serving
+ * internals", "PagedAttention as a virtual memory system": shared pages are
+ * stored once; "How vLLM gets real throughput on H100s", "PagedAttention
+ * borrows from operating systems": GRPO rollouts of one prompt share its
+ * pages).  The result equals pa_decode's up to rounding: softmax over keys
+ * 0..p splits exactly into the shared prefix and the rest.
+ *
+ * Groups: sequences group_start[g] .. group_start[g+1] - 1 (consecutive;
+ * group_start increasing, int32 [num_groups + 1], device) share their first
+ * group_prefix[g] tokens (int32 [num_groups], device): those entries of their
+ * block tables are identical.  Sequences outside [group_start[0],
+ * group_start[num_groups]) are plain decodes.  The first
+ * floor(group_prefix[g] / 64) * 64 keys of a group are read once for all its
+ * sequences and heads on the tcgen05 tensor cores; each sequence's remaining
+ * keys go through the decode kernel, which folds the prefix results in.  Each
+ * member's context must extend past that span (PA_ERR_RANGE on the device
+ * otherwise).  k_new / v_new: both NULL (append done elsewhere) or both set
+ * (fused append as in pa_decode_append).
+ *
+ * The workspace must hold pa_cascade_workspace_bytes() bytes, zero-filled
+ * once (contract of pa_workspace_bytes).  Supported: group <= 128 query heads
+ * per KV head, head_dim in {64, 128, 256}.
+ */
+PA_API size_t pa_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                         int max_blocks_per_seq, int block_size);
+PA_API int pa_decode_cascade(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                             void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                             int head_dim, int block_size, int num_blocks, float scale, const int32_t* group_start,
+                             const int32_t* group_prefix, int num_groups, void* workspace, size_t workspace_bytes,
+                             int* dev_status, void* stream);
+
+/*
  * pa_prefill_chunk -- attention for a varlen batch that mixes prefill chunks
  * and decodes in one call.  Sequence s contributes qlen = query_start[s+1] -
  * query_start[s] query rows: the LAST qlen positions of its context_lens[s]

@@ -33,6 +33,11 @@ _lib.pa_prefill_chunk.restype = _ci
 _lib.pa_decode_append.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                   ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
 _lib.pa_decode_append.restype = _ci
+_lib.pa_cascade_workspace_bytes.argtypes = [_ci, _ci, _ci, _ci, _ci, _ci]
+_lib.pa_cascade_workspace_bytes.restype = ctypes.c_size_t
+_lib.pa_decode_cascade.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
+                                   ctypes.c_float, _i32p, _i32p, _ci, _vp, ctypes.c_size_t, _vp, _vp]
+_lib.pa_decode_cascade.restype = _ci
 _lib.pa_decode_static_scratch.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                           ctypes.c_float, _vp, _vp]
 _lib.pa_decode_static_scratch.restype = _ci
@@ -170,6 +175,46 @@ def pa_decode_append(out, q, k_new, v_new, k_cache, v_cache, block_tables, conte
                                  _status_ptr(dev_status), _stream_ptr(stream)))
 
 
+def pa_cascade_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                               max_blocks_per_seq: int, block_size: int) -> int:
+    n = int(_lib.pa_cascade_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                                            block_size))
+    if n == 0:
+        raise PAError(PA_ERR_UNSUPPORTED)
+    return n
+
+
+def make_cascade_workspace(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                           max_blocks_per_seq: int, block_size: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace of pa_cascade_workspace_bytes() bytes."""
+    n = pa_cascade_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def pa_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens, scale, group_start, group_prefix,
+                      workspace, k_new=None, v_new=None, dev_status=None, stream=None) -> None:
+    """Decode attention for a batch with shared-prefix groups (sequences
+    group_start[g] .. group_start[g+1]-1 share their first group_prefix[g]
+    tokens); with k_new / v_new the step's append is fused in.  See include/pa.h."""
+    op, qp, kc, vc, bt, cl, ws = _attention_args(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    gs = _dev(group_start, "group_start", torch.int32, 1)
+    gp = _dev(group_prefix, "group_prefix", torch.int32, 1)
+    if group_start.shape[0] != group_prefix.shape[0] + 1:
+        raise ValueError("group_start must have one more entry than group_prefix")
+    nb, hkv, bs, d = k_cache.shape
+    if q.shape[0] != context_lens.shape[0]:
+        raise ValueError("pa_decode_cascade takes exactly one query row per sequence")
+    kn = vn = None
+    if k_new is not None or v_new is not None:
+        kn = _dev(k_new, "k_new", torch.bfloat16, 3)
+        vn = _dev(v_new, "v_new", torch.bfloat16, 3)
+        if k_new.shape != (context_lens.shape[0], hkv, d) or v_new.shape != k_new.shape:
+            raise ValueError("k_new / v_new must be [num_seqs, Hkv, d]")
+    _check(_lib.pa_decode_cascade(op, qp, kn, vn, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0],
+                                  q.shape[1], hkv, d, bs, nb, float(scale), gs, gp, group_prefix.shape[0], ws,
+                                  workspace.numel(), _status_ptr(dev_status), _stream_ptr(stream)))
+
+
 def pa_prefill_chunk(out, q, query_start, k_cache, v_cache, block_tables, context_lens, scale, workspace,
                      dev_status=None, stream=None) -> None:
     """Varlen batch of prefill chunks and decodes: q/out [Tq, Hq, d],
@@ -215,5 +260,5 @@ def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_len
 
 
 def exported_symbols() -> list[str]:
-    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_decode_append", "pa_prefill_chunk",
-            "pa_decode_static_scratch", "pa_status_string"]
+    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_decode_append", "pa_cascade_workspace_bytes",
+            "pa_decode_cascade", "pa_prefill_chunk", "pa_decode_static_scratch", "pa_status_string"]

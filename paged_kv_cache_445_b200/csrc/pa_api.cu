@@ -87,7 +87,8 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                          const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
                          void* workspace, size_t workspace_bytes, int* dev_status, void* stream,
-                         const void* k_new, const void* v_new) {
+                         const void* k_new, const void* v_new, const int32_t* group_start,
+                         const int32_t* group_prefix, int num_groups) {
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace) return PA_ERR_NULL;
   if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
   if (k_new && query_start) return PA_ERR_UNSUPPORTED;  // the fused append serves one-row (decode) batches
@@ -100,8 +101,16 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
   DeviceInfo di;
   if ((rc = device_info(&di)) != PA_OK) return rc;
   const long long max_keys = static_cast<long long>(max_blocks) * block_size;
-  if (workspace_bytes < workspace_needed(total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms))
-    return PA_ERR_WORKSPACE;
+  const size_t rows_bytes =
+      (workspace_needed(total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms) + 255) / 256 * 256;
+  if (num_groups < 0) return PA_ERR_SHAPE;
+  if (num_groups > 0) {  // shared-prefix groups: decode batches only
+    if (query_start) return PA_ERR_UNSUPPORTED;
+    if (!group_start || !group_prefix) return PA_ERR_NULL;
+    if (!cascade_supported(num_q_heads / num_kv_heads, head_dim)) return PA_ERR_UNSUPPORTED;
+  }
+  const size_t casc_bytes = num_groups > 0 ? cascade_partials_bytes(num_seqs, num_q_heads, head_dim) : 0;
+  if (workspace_bytes < rows_bytes + casc_bytes) return PA_ERR_WORKSPACE;
 
   CUtensorMap tmk, tmv;
   if ((rc = encode_kv_tmap(&tmk, k_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
@@ -128,7 +137,29 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
   p.v_new = v_new;
   p.k_cache = const_cast<void*>(k_cache);
   p.v_cache = const_cast<void*>(v_cache);
+  p.group_start = group_start;
+  p.group_prefix = group_prefix;
+  p.num_groups = num_groups;
+  p.casc_partials = num_groups > 0 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rows_bytes) : nullptr;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (num_groups > 0) {
+    // the shared prefixes first: per-slice partials that the rows kernel folds in
+    CascadeParams c{};
+    c.block_tables = block_tables;
+    c.max_blocks = max_blocks;
+    c.group_start = group_start;
+    c.group_prefix = group_prefix;
+    c.num_groups = num_groups;
+    c.num_q_heads = num_q_heads;
+    c.num_kv_heads = num_kv_heads;
+    c.group = p.group;
+    c.block_size = block_size;
+    c.num_blocks = num_blocks;
+    c.scale_log2 = p.scale_log2;
+    c.partials = const_cast<float*>(p.casc_partials);
+    c.status = dev_status;
+    if ((rc = launch_cascade(c, q, k_cache, v_cache, total_q_tokens, head_dim, st, di.num_sms)) != PA_OK) return rc;
+  }
   if (query_start && chunk_supported(p.group, head_dim)) {
     // sequences with more than one query row run on the tcgen05 chunk kernel,
     // the single rows (decodes) on the rows kernel right after it
@@ -201,6 +232,25 @@ int pa_decode_append(void* out, const void* q, const void* k_new, const void* v_
   return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                            num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                            workspace, workspace_bytes, dev_status, stream, k_new, v_new);
+}
+
+size_t pa_cascade_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int max_blocks_per_seq, int block_size) {
+  const size_t rows = pa_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size);
+  if (rows == 0 || !pa::cascade_supported(num_q_heads / num_kv_heads, head_dim)) return 0;
+  return (rows + 255) / 256 * 256 + pa::cascade_partials_bytes(num_seqs, num_q_heads, head_dim);
+}
+
+int pa_decode_cascade(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                      const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                      int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                      const int32_t* group_start, const int32_t* group_prefix, int num_groups, void* workspace,
+                      size_t workspace_bytes, int* dev_status, void* stream) {
+  if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
+  return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                           num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                           workspace, workspace_bytes, dev_status, stream, k_new, v_new, group_start, group_prefix,
+                           num_groups);
 }
 
 int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,

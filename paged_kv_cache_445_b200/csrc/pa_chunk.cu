@@ -41,6 +41,7 @@
 
 #include "pa_device.cuh"
 #include "pa_internal.h"
+#include "pa_umma.cuh"
 
 namespace pa {
 
@@ -68,93 +69,6 @@ constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when 
 // (a larger sum would make setmaxnreg.inc wait forever).
 constexpr int REGS_LAUNCH = 168, REGS_PRODUCER = 80, REGS_SOFTMAX = 208;
 static_assert(128 * REGS_PRODUCER + 256 * REGS_SOFTMAX <= CH_THREADS * REGS_LAUNCH, "register split");
-
-// ---- tcgen05 / UMMA helpers
-__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  // shared-memory matrix descriptor: start >> 4, LBO >> 4, SBO >> 4, version 1, 128-byte swizzle
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFF) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// kind::f16 instruction descriptor: bf16 x bf16 -> fp32, M x N, A/B major-ness
-__device__ __forceinline__ constexpr uint32_t umma_idesc(int m, int n, int a_mn_major, int b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
-         (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
-         (static_cast<uint32_t>(m >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
-}
-
-// Same MMA with the A operand (M x 16, K-major, 2 bf16 per 32-bit column) read
-// from tensor memory at column address a_tmem.
-__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-      ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])),
-      "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-      ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]),
-      "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 struct Item {
   int s;           // sequence
@@ -380,6 +294,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
     const uint32_t idesc_pv = umma_idesc(CH_M, CH_D, 0, 1);
     const uint32_t sq = smem_u32(smem + SMEM_Q);
     uint32_t q_phase = 0, p_phase[2] = {0, 0}, o_phase = 0, kv_count = 0;
+    uint32_t pv_commits[2] = {0, 0};  // completions committed to pv_done[w] so far
     bool first_item = true;
     for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x) {
       Item it;
@@ -400,14 +315,17 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           umma_commit(&sh.pv_done[1]);
         }
         __syncwarp();
+        ++pv_commits[0];
+        ++pv_commits[1];
         continue;
       }
-      // S_w(j) = Q_w K(j)^T.  S_w last held P_w(j - 1), which P V_w(j - 1)
-      // read: that MMA was issued before this one, and the MMAs of one CTA run
-      // in issue order.
+      // S_w(j) = Q_w K(j)^T.  S_w last held P_w(j - 1), the A operand of
+      // P V_w(j - 1): wait until that MMA has completed before overwriting it
+      // (for j = 0, the previous item's epilogue already waited for its last P V).
       auto qk = [&](int w, int j) -> bool {
         const int stage = (kv_count + j) % KST;
         if (w == 0 && !ch_wait(sh, &sh.k_full[stage], ((kv_count + j) / KST) & 1, p.status)) return false;
+        if (j > 0 && !ch_wait(sh, &sh.pv_done[w], (pv_commits[w] - 1) & 1, p.status)) return false;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sk = smem_u32(smem + SMEM_K + stage * KV_BYTES);
@@ -445,6 +363,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           if (w == 1) umma_commit(&sh.v_empty[stage]);
         }
         __syncwarp();
+        ++pv_commits[w];
         return true;
       };
       bool ok = qk(0, 0) && qk(1, 0);
@@ -509,11 +428,19 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           }
 #pragma unroll
           for (int k = 0; k < 8; ++k) m8[k] = s[k];
+          if (diag || cs >= 0.f) {
 #pragma unroll
-          for (int i = 8; i < CH_N; i += 8)
+            for (int i = 8; i < CH_N; i += 8)
 #pragma unroll
-            for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[i + k]);
-          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+              for (int k = 0; k < 8; ++k) m8[k] = fmaxf(m8[k], s[i + k]);
+            mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          } else {  // raw scores and a negative scale: the smallest raw score scales to the largest
+#pragma unroll
+            for (int i = 8; i < CH_N; i += 8)
+#pragma unroll
+              for (int k = 0; k < 8; ++k) m8[k] = fminf(m8[k], s[i + k]);
+            mx = fminf(fminf(fminf(m8[0], m8[1]), fminf(m8[2], m8[3])), fminf(fminf(m8[4], m8[5]), fminf(m8[6], m8[7])));
+          }
           if (!diag) mx *= cs;
         }
         const bool rescale = mx > m_ref + RESCALE_LOG2 || m_ref == -INFINITY;

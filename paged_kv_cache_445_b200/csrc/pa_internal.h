@@ -47,6 +47,58 @@ struct RowsParams {
   const void* v_new;
   void* k_cache;
   void* v_cache;
+  // Shared-prefix groups (decode only; num_groups = 0: none).  Sequences
+  // group_start[g] .. group_start[g+1]-1 share their first group_prefix[g]
+  // tokens; the cascade kernel has attended to the first cascade_span() of
+  // them and left per-slice partials in casc_partials, which this kernel folds
+  // in.  Its own segments start at that key.
+  const int32_t* group_start;
+  const int32_t* group_prefix;
+  int num_groups;
+  const float* casc_partials;  // [B][Hq][CASCADE_SPLITS + 1][D + 4]: O, m (log2 units), l; the last slot
+                               // holds this kernel's own unnormalised result of an unsplit segment
+};
+
+// Shared-prefix pass: prefix keys handled together, in tiles of 64, cut into at
+// most CASCADE_SPLITS slices per group.
+constexpr int CASCADE_SPLITS = 8;
+constexpr int CASCADE_TILE = 64;
+// one partial record: O[D], m, l, two floats of padding (16-byte aligned records)
+__host__ __device__ constexpr int cascade_record_floats(int head_dim) { return head_dim + 4; }
+__host__ __device__ __forceinline__ int cascade_span(int prefix_tokens) {
+  return prefix_tokens >= CASCADE_TILE ? prefix_tokens / CASCADE_TILE * CASCADE_TILE : 0;
+}
+__host__ __device__ __forceinline__ int cascade_splits(int span) {
+  const int tiles = span / CASCADE_TILE;
+  if (tiles <= 0) return 0;
+  const int n = tiles < CASCADE_SPLITS ? tiles : CASCADE_SPLITS;
+  const int per = (tiles + n - 1) / n;
+  return (tiles + per - 1) / per;  // no empty slice
+}
+
+// Sequences per M-tile of the shared-prefix pass: as many as fit in 128 rows
+// with a row count that is a multiple of 8 (whole 8-row swizzle atoms: a TMA
+// box of another height left the last rows of Q landing after the barrier).
+__host__ __device__ __forceinline__ int cascade_tokm(int group) {
+  int t = 128 / group;
+  while (t > 1 && (t * group) % 8 != 0) --t;
+  return t;
+}
+
+struct CascadeParams {
+  const int32_t* block_tables;
+  int max_blocks;
+  const int32_t* group_start;
+  const int32_t* group_prefix;
+  int num_groups;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;  // query heads per KV head
+  int block_size;
+  int num_blocks;
+  float scale_log2;
+  float* partials;
+  int* status;
 };
 
 // Parameters of the tcgen05 chunk kernel (sequences with more than one query row).
@@ -96,12 +148,17 @@ int rows_supported(int group, int head_dim);
 int chunk_supported(int group, int head_dim);
 int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const void* v_cache, int total_q_tokens,
                  cudaStream_t stream, int num_sms);
+int cascade_supported(int group, int head_dim);
+size_t cascade_partials_bytes(int num_seqs, int num_q_heads, int head_dim);
+int launch_cascade(const CascadeParams& p, const void* q, const void* k_cache, const void* v_cache,
+                   int total_q_tokens, int head_dim, cudaStream_t stream, int num_sms);
 // Argument checks, tensor maps and kernel dispatch shared by the attention
 // entry points (query_start == nullptr: one query row per sequence).
 int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,
                   const int32_t* block_tables, int max_blocks, const int32_t* context_lens, int num_seqs,
                   int total_q_tokens, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                   int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
-                  void* stream, const void* k_new = nullptr, const void* v_new = nullptr);
+                  void* stream, const void* k_new = nullptr, const void* v_new = nullptr,
+                  const int32_t* group_start = nullptr, const int32_t* group_prefix = nullptr, int num_groups = 0);
 
 }  // namespace pa

@@ -73,8 +73,24 @@ __device__ __forceinline__ long long warp_incl_scan64(long long v, int lane) {
 }
 
 struct SeqInfo {
-  int ctx, qlen, q0;
+  int ctx, qlen, q0;  // ctx: keys this kernel attends to, from key k0 on
+  int k0;             // keys before k0 came from the shared-prefix pass
 };
+
+// First key this kernel attends to for sequence s: the shared-prefix span of
+// its group, if it belongs to one (binary search over the group boundaries).
+__device__ __forceinline__ int cascade_key0(const RowsParams& p, int s) {
+  if (p.num_groups <= 0 || s < __ldg(p.group_start) || s >= __ldg(p.group_start + p.num_groups)) return 0;
+  int lo = 0, hi = p.num_groups - 1;  // last g with group_start[g] <= s
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.group_start + mid) <= s)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return cascade_span(__ldg(p.group_prefix + lo));
+}
 
 __device__ __forceinline__ SeqInfo seq_info(const RowsParams& p, int s) {
   SeqInfo si;
@@ -93,6 +109,16 @@ __device__ __forceinline__ SeqInfo seq_info(const RowsParams& p, int s) {
   }
   si.ctx = ctx < 0 ? 0 : ctx;
   if (si.qlen < 0) si.qlen = 0;
+  si.k0 = 0;
+  if (p.num_groups > 0) {
+    const int k0 = cascade_key0(p, s);
+    if (k0 > 0 && si.qlen == 1 && si.ctx > k0) {
+      si.k0 = k0;
+      si.ctx -= k0;
+    } else if (k0 > 0) {  // the newest token must lie after the shared prefix
+      set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+    }
+  }
   return si;
 }
 
@@ -107,6 +133,7 @@ struct Cursor {
   int s, i, h, t;  // sequence, row within it, KV head, tile within the segment
   int n, nkeys;    // tiles and keys of the current segment
   int p0, qlen, q0;
+  int k0;          // first key of the segments (after a shared prefix handled elsewhere)
   long long u;     // global unit index
 };
 
@@ -116,6 +143,7 @@ __device__ __forceinline__ bool enter_seq(const RowsParams& p, Cursor& c, int s)
   c.s = s;
   c.qlen = si.qlen;
   c.q0 = si.q0;
+  c.k0 = si.k0;
   c.p0 = si.ctx - si.qlen;
   c.i = c.p0 < 0 ? -c.p0 : 0;  // first row that has a key
   c.h = 0;
@@ -247,6 +275,7 @@ __device__ __forceinline__ void seek(const RowsParams& p, const long long* pfx, 
   cc.s = s_found;
   cc.qlen = si.qlen;
   cc.q0 = si.q0;
+  cc.k0 = si.k0;
   cc.p0 = si.ctx - si.qlen;
   const int i0 = cc.p0 < 0 ? -cc.p0 : 0;
   const long long o = a - seq_base;
@@ -266,6 +295,65 @@ __device__ __forceinline__ void seek(const RowsParams& p, const long long* pfx, 
   cc.h = static_cast<int>(rem / cc.n);
   cc.t = static_cast<int>(rem % cc.n);
   cc.u = a;
+}
+
+// Fold the shared-prefix partials of (sequence seq, KV head kvh) into the state
+// of its segment: per query head, O <- O e^(m - m') + O_k e^(m_k - m'),
+// l likewise, m' = max(m, m_k), over the prefix slices k.
+template <int D, int NT>
+__device__ __forceinline__ void fold_prefix(const RowsParams& p, int k_begin, int k_end, float (&o)[D / 16][NT][4],
+                                            float (&m)[NT][2], float (&l)[NT][2], int seq, int kvh, int lane) {
+  const int g = lane >> 2, c = lane & 3;
+  for (int k = k_begin; k < k_end; ++k) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int head = nt * 8 + 2 * c + e;
+        if (head >= p.group) continue;
+        const float* src = p.casc_partials +
+                           ((static_cast<long long>(seq) * p.num_q_heads + kvh * p.group + head) * (CASCADE_SPLITS + 1) +
+                            k) * cascade_record_floats(D);
+        const float mk = __ldcg(src + D), lk = __ldcg(src + D + 1);
+        const float mn = fmaxf(m[nt][e], mk);
+        const float f = fast_exp2(m[nt][e] - mn), w = fast_exp2(mk - mn);
+        m[nt][e] = mn;
+        l[nt][e] = l[nt][e] * f + w * lk;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {  // accumulator rows: head dim 16 mt + g and 16 mt + g + 8
+          o[mt][nt][e] = o[mt][nt][e] * f + w * __ldcg(src + 16 * mt + g);
+          o[mt][nt][2 + e] = o[mt][nt][2 + e] * f + w * __ldcg(src + 16 * mt + g + 8);
+        }
+      }
+  }
+}
+
+// Store the unnormalised state of a whole private segment in the shared-prefix
+// buffer's last slot (index CASCADE_SPLITS), row-major per query head.
+template <int D, int NT>
+__device__ __forceinline__ void store_own_partial(const RowsParams& p, const float (&o)[D / 16][NT][4],
+                                                  const float (&m)[NT][2], const float (&l)[NT][2], int seq, int kvh,
+                                                  int lane) {
+  const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int head = nt * 8 + 2 * c + e;
+      if (head >= p.group) continue;
+      float* dst = const_cast<float*>(p.casc_partials) +
+                   ((static_cast<long long>(seq) * p.num_q_heads + kvh * p.group + head) * (CASCADE_SPLITS + 1) +
+                    CASCADE_SPLITS) * cascade_record_floats(D);
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        dst[16 * mt + g] = o[mt][nt][e];
+        dst[16 * mt + g + 8] = o[mt][nt][2 + e];
+      }
+      if (g == 0) {
+        dst[D] = m[nt][e];
+        dst[D + 1] = l[nt][e];
+      }
+    }
 }
 
 // Merge the partial (m, l, O) results of the pieces of segment [segA, segA + n)
@@ -314,6 +402,14 @@ __device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, 
         acc[mt][nt][2] = acc[mt][nt][2] * f[0] + gk[0] * v.z;
         acc[mt][nt][3] = acc[mt][nt][3] * f[1] + gk[1] * v.w;
       }
+    }
+  }
+  if (p.num_groups > 0) {
+    const int span = seq_info(p, row).k0;  // decode: row = sequence; 0 if its keys were not split
+    if (span > 0) {
+      // n == 0: the private part was one piece, kept in the last slot; then the prefix slices
+      if (n == 0) fold_prefix<D, NT>(p, CASCADE_SPLITS, CASCADE_SPLITS + 1, acc, mm, ll, row, kvh, lane);
+      fold_prefix<D, NT>(p, 0, cascade_splits(span), acc, mm, ll, row, kvh, lane);
     }
   }
   store_output<D, NT>(p, acc, ll, row, kvh, lane);
@@ -442,7 +538,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
 
     auto issue = [&](int stage) {
       const bool first = lc.u == a, last = lc.u == e - 1;
-      const int key0 = lc.t * TILE_KEYS;
+      const int key0 = lc.k0 + lc.t * TILE_KEYS;
       const int lb = key0 / p.block_size, y = key0 - lb * p.block_size;
       const int blk = bt_lookup(p, win, lc.s, lb, lane);
       if (lc.t == 0 || first) {
@@ -682,7 +778,13 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
             v += __shfl_xor_sync(FULL_MASK, v, 16);
             l[nt][q2] = v;
           }
-        if (began && tm.t == tm.n - 1) {
+        if (began && tm.t == tm.n - 1 && p.num_groups > 0 && seq_info(p, tm.row).k0 > 0) {
+          // the whole private part of a shared-prefix segment: keep it unnormalised
+          // for the merge phase, which folds in the prefix (decode: row = sequence)
+          store_own_partial<D, NT>(p, o, m, l, tm.row, tm.h, lane);
+          if (lane == 0)
+            p.seginfo[static_cast<long long>(tm.row) * p.num_kv_heads + tm.h] = (tm.u - tm.t) + 1;  // no pieces
+        } else if (began && tm.t == tm.n - 1) {
           store_output<D, NT>(p, o, l, tm.row, tm.h, lane);
         } else if (nslots < ROWS_SLOTS_PER_WARP) {
           const long long slot = static_cast<long long>(gw) * ROWS_SLOTS_PER_WARP + nslots++;

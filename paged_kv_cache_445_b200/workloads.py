@@ -88,6 +88,7 @@ class Workload:
     query_start: np.ndarray
     slot_mapping: np.ndarray
     shared_prefix_tokens: int = 0
+    shared_groups: tuple = ()  # (first sequence, end sequence) of each copy-on-write group
 
     @property
     def num_seqs(self) -> int:
@@ -104,6 +105,23 @@ class Workload:
     @property
     def is_decode(self) -> bool:
         return bool(np.all(self.query_lens == 1))
+
+    def prefix_groups(self):
+        """(group_start int32 [G + 1], group_prefix int32 [G]) describing the
+        shared-prefix groups as consecutive sequence ranges (gaps between
+        groups become groups with prefix 0), or None when nothing is shared."""
+        if not self.shared_groups or self.shared_prefix_tokens <= 0:
+            return None
+        start, prefix, pos = [], [], None
+        for lo, hi in sorted(self.shared_groups):
+            if pos is not None and lo > pos:  # sequences between two groups share nothing
+                start.append(pos)
+                prefix.append(0)
+            start.append(lo)
+            prefix.append(self.shared_prefix_tokens)
+            pos = hi
+        start.append(pos)
+        return np.asarray(start, dtype=np.int32), np.asarray(prefix, dtype=np.int32)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -228,9 +246,15 @@ def build(spec: Spec, seed: int, poison: bool = False, max_blocks: int | None = 
         k_cache.transpose(0, 2, 1, 3)[bad] = BF16_NAN  # views: writes land in the caches
         v_cache.transpose(0, 2, 1, 3)[bad] = BF16_NAN
 
+    groups = []
+    for g in spec.share:
+        members = sorted(g)
+        if members != list(range(members[0], members[-1] + 1)):
+            raise AssertionError("copy-on-write groups are consecutive sequences")
+        groups.append((members[0], members[-1] + 1))
     return Workload(spec.name, hq, hkv, d, bs, nb, 1.0 / math.sqrt(d), q, k_new, v_new,
                     k_cache, v_cache, block_tables, context_lens, query_start, slot_mapping,
-                    spec.share_tokens)
+                    spec.share_tokens, tuple(groups))
 
 
 def standard(cfg: int, seed: int | None = None, poison: bool = False) -> Workload:
