@@ -50,6 +50,11 @@ PINS = {
     ],
     "cache_append": ["test_append_is_a_byte_copy", "test_append_then_attend_reads_new_row"],
     "slot_mapping": ["test_slot_mapping_closed_form", "test_allocator_slots_match_oracle"],
+    "e4m3_to_f64": ["test_e4m3_values_from_the_definition"],
+    "f32_to_e4m3": ["test_e4m3_round_trip_and_monotone", "test_e4m3_ties_to_even_and_saturation"],
+    "cache_append_fp8": ["test_fp8_append_writes_codes_of_the_scaled_rows"],
+    "paged_attention_fp8": ["test_fp8_attention_equals_bf16_attention_on_exact_values",
+                            "test_fp8_scales_factor_out"],
 }
 
 
@@ -83,6 +88,18 @@ def _bind(lib):
         f64p, u16p, u16p, u16p, i32p, ci, i32p, i32p, ci, ci, ci, ci, ci, ci,
         ctypes.c_double, ctypes.c_void_p, ci]
     lib.oracle_paged_attention.restype = ci
+    u8p = np.ctypeslib.ndpointer(np.uint8, flags="C_CONTIGUOUS")
+    lib.oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_f64.restype = ctypes.c_double
+    lib.oracle_f32_to_e4m3.argtypes = [ctypes.c_float]
+    lib.oracle_f32_to_e4m3.restype = ctypes.c_uint8
+    lib.oracle_cache_append_fp8.argtypes = [u16p, u16p, u8p, u8p, i32p, ci, ci, ci, ci, ci, ctypes.c_float,
+                                            ctypes.c_float]
+    lib.oracle_cache_append_fp8.restype = ci
+    lib.oracle_paged_attention_fp8.argtypes = [
+        f64p, u16p, u8p, u8p, i32p, ci, i32p, i32p, ci, ci, ci, ci, ci, ci,
+        ctypes.c_double, ctypes.c_double, ctypes.c_double, ctypes.c_void_p, ci]
+    lib.oracle_paged_attention_fp8.restype = ci
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ci
     return lib
@@ -159,6 +176,66 @@ def paged_attention(q, k_cache, v_cache, block_tables, context_lens, query_start
                                     bs, nb, float(scale), ptr, n_only)
     if rc != 0:
         raise ValueError(f"oracle_paged_attention failed: {rc}")
+    return out
+
+
+def e4m3_to_f64(codes, lib=None) -> np.ndarray:
+    """Values of E4M3 codes (OCP 8-bit float, "FN" variant)."""
+    lib = lib or load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_to_f64(int(x)) for x in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def f32_to_e4m3(x, lib=None) -> np.ndarray:
+    """E4M3 codes of binary32 values: round to nearest-even, saturate to +-448."""
+    lib = lib or load()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([lib.oracle_f32_to_e4m3(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def inv_scale(scale: float) -> float:
+    """The binary32 reciprocal the append multiplies by: fl32(1 / fl32(scale))."""
+    return float(np.float32(1.0) / np.float32(scale))
+
+
+def cache_append_fp8(k_new, v_new, k_cache, v_cache, slot_map, k_scale, v_scale, lib=None):
+    """In-place E4M3 append: code = E4M3(bf16 value * fl32(1 / scale)), product in binary32."""
+    lib = lib or load()
+    assert k_cache.dtype == np.uint8 and k_cache.flags.c_contiguous
+    assert v_cache.dtype == np.uint8 and v_cache.flags.c_contiguous
+    nb, hkv, bs, d = k_cache.shape
+    kn = _c(k_new, np.uint16)
+    vn = _c(v_new, np.uint16)
+    sm = _c(slot_map, np.int32)
+    rc = lib.oracle_cache_append_fp8(kn, vn, k_cache, v_cache, sm, len(sm), nb, hkv, d, bs,
+                                     inv_scale(k_scale), inv_scale(v_scale))
+    if rc != 0:
+        raise ValueError(f"oracle_cache_append_fp8 failed: {rc}")
+
+
+def paged_attention_fp8(q, k_cache, v_cache, block_tables, context_lens, query_start, scale, k_scale, v_scale,
+                        only=None, lib=None):
+    """paged_attention over E4M3 caches (uint8 codes) with per-tensor scales."""
+    lib = lib or load()
+    q = _c(q, np.uint16)
+    kc = _c(k_cache, np.uint8)
+    vc = _c(v_cache, np.uint8)
+    bt = _c(block_tables, np.int32)
+    cl = _c(context_lens, np.int32)
+    qs = _c(query_start, np.int32)
+    t, hq, d = q.shape
+    nb, hkv, bs, d2 = kc.shape
+    assert d == d2 and int(qs[-1]) == t
+    out = np.zeros((t, hq, d), dtype=np.float64)
+    if only is not None:
+        only_arr = _c(only, np.int32).reshape(-1, 2)
+        ptr, n_only = only_arr.ctypes.data, len(only_arr)
+    else:
+        only_arr, ptr, n_only = None, None, 0
+    rc = lib.oracle_paged_attention_fp8(out, q, kc, vc, bt, bt.shape[1], cl, qs, len(cl), hq, hkv, d, bs, nb,
+                                        float(scale), float(k_scale), float(v_scale), ptr, n_only)
+    if rc != 0:
+        raise ValueError(f"oracle_paged_attention_fp8 failed: {rc}")
     return out
 
 

@@ -292,6 +292,190 @@ int oracle_paged_attention(double *out, const uint16_t *q, const uint16_t *k_cac
     return status;
 }
 
+/*
+ * ---- FP8 KV cache -------------------------------------------------------
+ *
+ * The pages serve Llama 3.3 70B in FP8 ("vLLM serving internals",
+ * introduction and "Numbers to remember"; "How vLLM gets real throughput on
+ * H100s", "Hopper-specific tunings") without fixing a format.  The reading
+ * taken here: the cache stores E4M3 codes of the OCP 8-bit floating point
+ * specification ("FN" variant: sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits, no infinities, S.1111.111 = NaN, largest finite 1.75 * 2^8 = 448,
+ * subnormals m/8 * 2^-6) with one scale per tensor: code = E4M3(x * (1/scale))
+ * rounded to nearest-even and saturated to +-448, value = E4M3value * scale.
+ */
+double oracle_e4m3_to_f64(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    double v = (e == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+uint8_t oracle_f32_to_e4m3(float xf)
+{
+    double x = xf; /* exact */
+    if (isnan(x))
+        return 0x7F;
+    uint8_t sgn = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (isinf(a))
+        return (uint8_t)(sgn | 0x7E);
+    if (a == 0.0)
+        return sgn;
+    int e2;
+    frexp(a, &e2);           /* a = f * 2^e2, f in [0.5, 1): floor(log2 a) = e2 - 1 */
+    int ex = e2 - 1;
+    double quantum = ex < -6 ? ldexp(1.0, -9) : ldexp(1.0, ex - 3);
+    double r = nearbyint(a / quantum) * quantum; /* a / quantum is exact; ties to even */
+    if (r > 448.0)
+        r = 448.0; /* saturate to the largest finite value */
+    if (r == 0.0)
+        return sgn;
+    frexp(r, &e2);
+    ex = e2 - 1;
+    if (ex < -6) /* subnormal: exponent field 0, r = m * 2^-9 */
+        return (uint8_t)(sgn | (uint8_t)(r / ldexp(1.0, -9)));
+    int m = (int)((r / ldexp(1.0, ex) - 1.0) * 8.0);
+    return (uint8_t)(sgn | (uint8_t)((ex + 7) << 3) | (uint8_t)m);
+}
+
+/*
+ * FP8 cache append [KV]: for every token with slot >= 0 and every KV head,
+ * code = E4M3(bf16 value * inv_scale), the product taken in binary32.
+ */
+int oracle_cache_append_fp8(const uint16_t *k_new, const uint16_t *v_new, uint8_t *k_cache, uint8_t *v_cache,
+                            const int32_t *slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                            int head_dim, int block_size, float k_inv_scale, float v_inv_scale)
+{
+    long long num_slots = (long long)num_blocks * block_size;
+    for (int t = 0; t < num_tokens; ++t) {
+        long long slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        if (slot >= num_slots)
+            return ORACLE_ERR_RANGE;
+        long long blk = slot / block_size, off = slot % block_size;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            long long dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
+            long long src = ((long long)t * num_kv_heads + h) * head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                float kx = (float)bf16_bits_to_double(k_new[src + d]) * k_inv_scale;
+                float vx = (float)bf16_bits_to_double(v_new[src + d]) * v_inv_scale;
+                k_cache[dst + d] = oracle_f32_to_e4m3(kx);
+                v_cache[dst + d] = oracle_f32_to_e4m3(vx);
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* One output row [SDPA] over an FP8 cache: K_j = E4M3value * k_scale, V_j likewise. */
+static int attend_one_fp8(double *out, const uint16_t *q_row, const uint8_t *k_cache, const uint8_t *v_cache,
+                          const int32_t *block_tables, int max_blocks, int s, int last_key, int kvh,
+                          int num_kv_heads, int head_dim, int block_size, int num_blocks, double scale,
+                          double k_scale, double v_scale, double *scores, double *acc)
+{
+    int nkeys = last_key + 1;
+    for (int d = 0; d < head_dim; ++d)
+        acc[d] = 0.0;
+    if (nkeys <= 0) {
+        memcpy(out, acc, sizeof(double) * (size_t)head_dim);
+        return ORACLE_OK;
+    }
+    double m = -INFINITY;
+    for (int j = 0; j < nkeys; ++j) {
+        long long row = physical_row(block_tables, max_blocks, s, j, block_size, num_blocks);
+        if (row < 0)
+            return ORACLE_ERR_RANGE;
+        long long blk = row / block_size, off = row % block_size;
+        const uint8_t *krow = k_cache + ((blk * num_kv_heads + kvh) * block_size + off) * head_dim;
+        double dot = 0.0;
+        for (int d = 0; d < head_dim; ++d)
+            dot += bf16_bits_to_double(q_row[d]) * (oracle_e4m3_to_f64(krow[d]) * k_scale);
+        scores[j] = scale * dot;
+        if (scores[j] > m)
+            m = scores[j];
+    }
+    double denom = 0.0;
+    for (int j = 0; j < nkeys; ++j) {
+        double w = exp(scores[j] - m);
+        long long row = physical_row(block_tables, max_blocks, s, j, block_size, num_blocks);
+        long long blk = row / block_size, off = row % block_size;
+        const uint8_t *vrow = v_cache + ((blk * num_kv_heads + kvh) * block_size + off) * head_dim;
+        for (int d = 0; d < head_dim; ++d)
+            acc[d] += w * (oracle_e4m3_to_f64(vrow[d]) * v_scale);
+        denom += w;
+    }
+    for (int d = 0; d < head_dim; ++d)
+        acc[d] /= denom;
+    memcpy(out, acc, sizeof(double) * (size_t)head_dim);
+    return ORACLE_OK;
+}
+
+/* oracle_paged_attention over an FP8 cache (same conventions). */
+int oracle_paged_attention_fp8(double *out, const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                               const int32_t *block_tables, int max_blocks, const int32_t *context_lens,
+                               const int32_t *query_start, int num_seqs, int num_q_heads, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, double scale, double k_scale,
+                               double v_scale, const int32_t *only_rows, int n_only)
+{
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+        return ORACLE_ERR_SHAPE;
+    int group = num_q_heads / num_kv_heads;
+    int num_tokens = query_start[num_seqs];
+    int max_ctx = 0;
+    for (int s = 0; s < num_seqs; ++s)
+        if (context_lens[s] > max_ctx)
+            max_ctx = context_lens[s];
+    int32_t *seq_of = (int32_t *)malloc(sizeof(int32_t) * (size_t)(num_tokens > 0 ? num_tokens : 1));
+    if (!seq_of)
+        return ORACLE_ERR_NOMEM;
+    for (int s = 0; s < num_seqs; ++s)
+        for (int t = query_start[s]; t < query_start[s + 1]; ++t)
+            seq_of[t] = s;
+    long long n_items = only_rows ? n_only : (long long)num_tokens * num_q_heads;
+    int status = ORACLE_OK;
+#pragma omp parallel
+    {
+        double *scores = (double *)malloc(sizeof(double) * (size_t)(max_ctx > 0 ? max_ctx : 1));
+        double *acc = (double *)malloc(sizeof(double) * (size_t)head_dim);
+        if (!scores || !acc) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long long it = 0; it < n_items; ++it) {
+            if (!scores || !acc)
+                continue;
+            int t, h;
+            if (only_rows) {
+                t = only_rows[2 * it];
+                h = only_rows[2 * it + 1];
+            } else {
+                t = (int)(it / num_q_heads);
+                h = (int)(it % num_q_heads);
+            }
+            int s = seq_of[t];
+            int qlen = query_start[s + 1] - query_start[s];
+            int pos = context_lens[s] - qlen + (t - query_start[s]);
+            int rc = attend_one_fp8(out + ((long long)t * num_q_heads + h) * head_dim,
+                                    q + ((long long)t * num_q_heads + h) * head_dim, k_cache, v_cache, block_tables,
+                                    max_blocks, s, pos, h / group, num_kv_heads, head_dim, block_size, num_blocks,
+                                    scale, k_scale, v_scale, scores, acc);
+            if (rc != ORACLE_OK) {
+#pragma omp atomic write
+                status = rc;
+            }
+        }
+        free(scores);
+        free(acc);
+    }
+    free(seq_of);
+    return status;
+}
+
 int oracle_num_threads(void)
 {
     int n = 1;
