@@ -321,6 +321,18 @@ def run_ours(args, peaks):
     if int(g.status.item()) != 0:
         raise SystemExit(f"device status {int(g.status.item())} after warm-up")
 
+    graph = None
+    if args.graph:  # the whole step (all its launches) as one CUDA graph, replayed per step
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            g.append()
+            g.attend()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        if int(g.status.item()) != 0:
+            raise SystemExit(f"device status {int(g.status.item())} after graph warm-up")
+
     # ---- device-timed region
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -330,6 +342,11 @@ def run_ours(args, peaks):
     with sampler:
         start.record(stream)
         for i in range(args.steps):
+            if graph is not None:  # append + attention inside one replay: the events bracket both
+                ev[i][0].record(stream)
+                graph.replay()
+                ev[i][1].record(stream)
+                continue
             g.append()
             ev[i][0].record(stream)
             g.attend()
@@ -384,7 +401,8 @@ def run_ours(args, peaks):
     unique_kv = _rl.unique_kv_bytes(w.block_tables, w.context_lens, w.block_size, w.num_kv_heads, w.head_dim)
     if g.cascade:  # a shared prefix crosses HBM once: the algorithmic bytes are the unique ones
         attn_bytes = attn_bytes - kv_bytes + unique_kv
-    launch_bytes = attn_bytes + (app_bytes if g.fused else 0)  # the timed launch also appends when fused
+    # the timed launch (or replay) also appends when fused or replayed as a graph
+    launch_bytes = attn_bytes + (app_bytes if (g.fused or graph is not None) else 0)
     achieved = launch_bytes / (attn_avg_ms * 1e-3) / 1e9
     traffic = profiled_traffic("pa_rows_kernel", w.name)
     line = {
@@ -406,6 +424,7 @@ def run_ours(args, peaks):
             "unique_kv_bytes_per_step": unique_kv,
             "l2": f"no flush: every step reads {kv_bytes / 1e9:.2f} GB of KV, larger than the 126 MB L2",
             "parallelism": f"dp{world} (independent batch per GPU)",
+            "cuda_graph": graph is not None,
         },
         "seq_steps_per_s": round(total_seqs / (ms_step * 1e-3), 1),
         "frac_of_hbm_peak": round(compose_value(total_kv, ms_step) / hbm / world, 4),
@@ -534,6 +553,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step (all its launches) in a CUDA graph and time its replays")
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix batches: pa_decode_cascade (each shared prefix read once per group) "
                          "instead of plain decode")

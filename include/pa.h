@@ -154,6 +154,40 @@ PA_API int pa_decode_append(void* out, const void* q, const void* k_new, const v
                             size_t workspace_bytes, int* dev_status, void* stream);
 
 /*
+ * FP8 (E4M3) KV cache.  The pages serve the 70B model in FP8 ("vLLM serving
+ * internals", introduction and "Numbers to remember"; "How vLLM gets real
+ * throughput on H100s", "Hopper-specific tunings") without fixing a format;
+ * the cache here stores codes of the OCP 8-bit floating point E4M3 format
+ * ("FN" variant: no infinities, largest finite 448) with one scale per
+ * tensor: code = E4M3(x * fl32(1 / scale)) (binary32 product, nearest-even,
+ * saturated to +-448), value = E4M3value * scale.  k_cache / v_cache are
+ * uint8 [num_blocks, num_kv_heads, block_size, head_dim]: half the bytes of
+ * bf16, so a decode step reads half the bytes.
+ *
+ * pa_cache_append_fp8 -- pa_cache_append into an FP8 cache (quantising).
+ * Scales must be positive and finite (PA_ERR_SHAPE otherwise).
+ */
+PA_API int pa_cache_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                               const int32_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                               int head_dim, int block_size, float k_scale, float v_scale, int* dev_status,
+                               void* stream);
+
+/*
+ * pa_decode_fp8 -- pa_decode over an FP8 cache; with k_new / v_new set (both
+ * or neither) the step's append is fused in, as in pa_decode_append (the new
+ * rows are quantised exactly as pa_cache_append_fp8 does).  q and out stay
+ * bf16.  Keys and values enter the tensor cores as f16 (exact for E4M3
+ * values) with q converted to f16; accumulation is fp32.  Supported:
+ * head_dim 128 or 256 (PA_ERR_UNSUPPORTED otherwise); same workspace as
+ * pa_decode.
+ */
+PA_API int pa_decode_fp8(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache,
+                         void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                         const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                         int block_size, int num_blocks, float scale, float k_scale, float v_scale, void* workspace,
+                         size_t workspace_bytes, int* dev_status, void* stream);
+
+/*
  * pa_decode_cascade -- pa_decode (optionally fused with the append, as
  * pa_decode_append) for a batch in which groups of sequences share a prefix of
  * the KV cache, as copy-on-write forks of one prompt do ("vLLM serving

@@ -10,7 +10,8 @@ the import raises: there is no CPU fallback.
 from __future__ import annotations
 
 __all__ = [
-    "pa_cache_append", "pa_decode", "pa_decode_append", "pa_decode_cascade", "pa_cascade_workspace_bytes",
+    "pa_cache_append", "pa_decode", "pa_decode_append", "pa_cache_append_fp8", "pa_decode_fp8",
+    "pa_decode_cascade", "pa_cascade_workspace_bytes",
     "make_cascade_workspace", "pa_prefill_chunk", "pa_workspace_bytes", "pa_decode_static_scratch",
     "pa_status_string", "PAError", "library_path", "make_workspace", "status_bit",
 ]

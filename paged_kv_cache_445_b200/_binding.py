@@ -38,6 +38,12 @@ _lib.pa_cascade_workspace_bytes.restype = ctypes.c_size_t
 _lib.pa_decode_cascade.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                    ctypes.c_float, _i32p, _i32p, _ci, _vp, ctypes.c_size_t, _vp, _vp]
 _lib.pa_decode_cascade.restype = _ci
+_lib.pa_cache_append_fp8.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _ci, _ci, _ci, _ci, ctypes.c_float,
+                                     ctypes.c_float, _vp, _vp]
+_lib.pa_cache_append_fp8.restype = _ci
+_lib.pa_decode_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
+                               ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
+_lib.pa_decode_fp8.restype = _ci
 _lib.pa_decode_static_scratch.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                           ctypes.c_float, _vp, _vp]
 _lib.pa_decode_static_scratch.restype = _ci
@@ -215,6 +221,47 @@ def pa_decode_cascade(out, q, k_cache, v_cache, block_tables, context_lens, scal
                                   workspace.numel(), _status_ptr(dev_status), _stream_ptr(stream)))
 
 
+def pa_cache_append_fp8(k_new, v_new, k_cache, v_cache, slot_mapping, k_scale, v_scale, dev_status=None,
+                        stream=None) -> None:
+    """Append into an FP8 (E4M3 codes, uint8) cache with per-tensor scales; see include/pa.h."""
+    kp = _dev(k_new, "k_new", torch.bfloat16, 3)
+    vp = _dev(v_new, "v_new", torch.bfloat16, 3)
+    kc = _dev(k_cache, "k_cache", torch.uint8, 4)
+    vc = _dev(v_cache, "v_cache", torch.uint8, 4)
+    sm = _dev(slot_mapping, "slot_mapping", torch.int32, 1)
+    nb, hkv, bs, d = k_cache.shape
+    if v_cache.shape != k_cache.shape or k_new.shape[1:] != (hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("k_new/v_new [T, Hkv, d] and caches [num_blocks, Hkv, block_size, d] must agree")
+    _check(_lib.pa_cache_append_fp8(kp, vp, kc, vc, sm, k_new.shape[0], nb, hkv, d, bs, float(k_scale),
+                                    float(v_scale), _status_ptr(dev_status), _stream_ptr(stream)))
+
+
+def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale, workspace,
+                  k_new=None, v_new=None, dev_status=None, stream=None) -> None:
+    """Decode over an FP8 cache; with k_new / v_new the step's append is fused in.  See include/pa.h."""
+    op = _dev(out, "out", torch.bfloat16, 3)
+    qp = _dev(q, "q", torch.bfloat16, 3)
+    kc = _dev(k_cache, "k_cache", torch.uint8, 4)
+    vc = _dev(v_cache, "v_cache", torch.uint8, 4)
+    bt = _dev(block_tables, "block_tables", torch.int32, 2)
+    cl = _dev(context_lens, "context_lens", torch.int32, 1)
+    ws = _dev(workspace, "workspace", torch.uint8, 1)
+    nb, hkv, bs, d = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or q.shape[2] != d:
+        raise ValueError("out/q [B, Hq, d] and caches [num_blocks, Hkv, block_size, d] must agree")
+    if q.shape[0] != context_lens.shape[0] or block_tables.shape[0] != context_lens.shape[0]:
+        raise ValueError("one query row, one block-table row and one length per sequence")
+    kn = vn = None
+    if k_new is not None or v_new is not None:
+        kn = _dev(k_new, "k_new", torch.bfloat16, 3)
+        vn = _dev(v_new, "v_new", torch.bfloat16, 3)
+        if k_new.shape != (context_lens.shape[0], hkv, d) or v_new.shape != k_new.shape:
+            raise ValueError("k_new / v_new must be [num_seqs, Hkv, d]")
+    _check(_lib.pa_decode_fp8(op, qp, kn, vn, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0],
+                              q.shape[1], hkv, d, bs, nb, float(scale), float(k_scale), float(v_scale), ws,
+                              workspace.numel(), _status_ptr(dev_status), _stream_ptr(stream)))
+
+
 def pa_prefill_chunk(out, q, query_start, k_cache, v_cache, block_tables, context_lens, scale, workspace,
                      dev_status=None, stream=None) -> None:
     """Varlen batch of prefill chunks and decodes: q/out [Tq, Hq, d],
@@ -260,5 +307,6 @@ def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_len
 
 
 def exported_symbols() -> list[str]:
-    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_decode_append", "pa_cascade_workspace_bytes",
-            "pa_decode_cascade", "pa_prefill_chunk", "pa_decode_static_scratch", "pa_status_string"]
+    return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_decode_append", "pa_cache_append_fp8",
+            "pa_decode_fp8", "pa_cascade_workspace_bytes", "pa_decode_cascade", "pa_prefill_chunk",
+            "pa_decode_static_scratch", "pa_status_string"]

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "pa_internal.h"
@@ -66,6 +67,26 @@ int encode_kv_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_
   return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
 
+// FP8 cache [num_blocks, Hkv, block_size, D] bytes viewed as (128, block_size,
+// D/128, Hkv, num_blocks): one box brings a 16-key tile of one (block, head) as
+// D/128 swizzled [16 x 128-byte] panels, the same smem layout as bf16 at half
+// the head dim.
+static int encode_kv_tmap_fp8(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads,
+                              int block_size, int head_dim) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return PA_ERR_CUDA;
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim);
+  const cuuint64_t dims[5] = {128, static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(head_dim / 128),
+                              static_cast<cuuint64_t>(num_kv_heads), static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t strides[4] = {row, 128, row * block_size, row * block_size * num_kv_heads};
+  const cuuint32_t box[5] = {128, 16, static_cast<cuuint32_t>(head_dim / 128), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(cache), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
 static int check_attention_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                                  int num_blocks, int max_blocks) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks <= 0)
@@ -88,10 +109,15 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
                          void* workspace, size_t workspace_bytes, int* dev_status, void* stream,
                          const void* k_new, const void* v_new, const int32_t* group_start,
-                         const int32_t* group_prefix, int num_groups) {
+                         const int32_t* group_prefix, int num_groups, int kv_fp8, float k_scale, float v_scale) {
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace) return PA_ERR_NULL;
   if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
   if (k_new && query_start) return PA_ERR_UNSUPPORTED;  // the fused append serves one-row (decode) batches
+  if (kv_fp8) {  // E4M3 caches: head_dim 128 or 256, no shared-prefix pass, finite positive scales
+    if (head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+    if (num_groups > 0) return PA_ERR_UNSUPPORTED;
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !(k_scale < INFINITY) || !(v_scale < INFINITY)) return PA_ERR_SHAPE;
+  }
   if (k_new && (!aligned16(k_new) || !aligned16(v_new))) return PA_ERR_SHAPE;
   int rc = check_attention_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, max_blocks);
   if (rc != PA_OK) return rc;
@@ -113,8 +139,13 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
   if (workspace_bytes < rows_bytes + casc_bytes) return PA_ERR_WORKSPACE;
 
   CUtensorMap tmk, tmv;
-  if ((rc = encode_kv_tmap(&tmk, k_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
-  if ((rc = encode_kv_tmap(&tmv, v_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
+  if (kv_fp8) {
+    if ((rc = encode_kv_tmap_fp8(&tmk, k_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
+    if ((rc = encode_kv_tmap_fp8(&tmv, v_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
+  } else {
+    if ((rc = encode_kv_tmap(&tmk, k_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
+    if ((rc = encode_kv_tmap(&tmv, v_cache, num_blocks, num_kv_heads, block_size, head_dim)) != PA_OK) return rc;
+  }
 
   RowsParams p{};
   p.out = out;
@@ -131,6 +162,15 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
   p.num_blocks = num_blocks;
   p.skip_multi = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.kv_fp8 = kv_fp8;
+  p.v_scale = 1.f;
+  p.k_inv_scale = p.v_inv_scale = 1.f;
+  if (kv_fp8) {  // scores of codes times k_scale: fold it into the softmax scale
+    p.scale_log2 = scale * k_scale * 1.4426950408889634f;
+    p.v_scale = v_scale;
+    p.k_inv_scale = 1.f / k_scale;
+    p.v_inv_scale = 1.f / v_scale;
+  }
   rows_workspace_layout(workspace, total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms, &p);
   p.status = dev_status;
   p.k_new = k_new;
@@ -160,7 +200,7 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
     c.status = dev_status;
     if ((rc = launch_cascade(c, q, k_cache, v_cache, total_q_tokens, head_dim, st, di.num_sms)) != PA_OK) return rc;
   }
-  if (query_start && chunk_supported(p.group, head_dim)) {
+  if (query_start && !kv_fp8 && chunk_supported(p.group, head_dim)) {
     // sequences with more than one query row run on the tcgen05 chunk kernel,
     // the single rows (decodes) on the rows kernel right after it
     ChunkParams c{};
@@ -251,6 +291,37 @@ int pa_decode_cascade(void* out, const void* q, const void* k_new, const void* v
                            num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                            workspace, workspace_bytes, dev_status, stream, k_new, v_new, group_start, group_prefix,
                            num_groups);
+}
+
+int pa_cache_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                        const int32_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads, int head_dim,
+                        int block_size, float k_scale, float v_scale, int* dev_status, void* stream) {
+  if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0) return PA_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PA_ERR_UNSUPPORTED;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  if (!(k_scale > 0.f) || !(v_scale > 0.f) || !(k_scale < INFINITY) || !(v_scale < INFINITY)) return PA_ERR_SHAPE;
+  if (num_tokens == 0) return PA_OK;
+  if (!k_new || !v_new || !k_cache || !v_cache || !slot_mapping) return PA_ERR_NULL;
+  if (!pa::aligned16(k_new) || !pa::aligned16(v_new) || !pa::aligned16(k_cache) || !pa::aligned16(v_cache))
+    return PA_ERR_SHAPE;
+  pa::DeviceInfo di;
+  int rc = pa::device_info(&di);
+  if (rc != PA_OK) return rc;
+  return pa::launch_append_fp8(k_new, v_new, k_cache, v_cache, slot_mapping, num_tokens, num_blocks, num_kv_heads,
+                               head_dim, block_size, 1.f / k_scale, 1.f / v_scale, dev_status,
+                               static_cast<cudaStream_t>(stream), di.num_sms);
+}
+
+int pa_decode_fp8(void* out, const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                  const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens, int num_seqs,
+                  int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                  float k_scale, float v_scale, void* workspace, size_t workspace_bytes, int* dev_status,
+                  void* stream) {
+  if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
+  return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                           num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                           workspace, workspace_bytes, dev_status, stream, k_new, v_new, nullptr, nullptr, 0, 1,
+                           k_scale, v_scale);
 }
 
 int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,

@@ -170,6 +170,48 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
+// D[16x8] += A[16x16] * B[16x8], f16 inputs, fp32 accumulators.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 codes (low and high 16 bits of x: bytes 0-1 or 2-3) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_lo_to_f16x2(uint32_t x) {
+  uint32_t y;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t x) {
+  uint32_t y;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, hi;\n\t}" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Bytes (b0, b1, b2, b3) of x -> (b0, b2, b1, b3): pairs the same byte of two 16-bit halves.
+__device__ __forceinline__ uint32_t pair_bytes(uint32_t x) {
+  uint32_t y;
+  asm("prmt.b32 %0, %1, 0, 0x3120;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Two binary32 values -> their E4M3 codes (nearest-even, saturated to +-448): lo in byte 0, hi in byte 1.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t y;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t y;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
 // D[16x8] += A[16x16] * B[16x8], bf16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {

@@ -55,6 +55,13 @@ struct RowsParams {
   const int32_t* group_start;
   const int32_t* group_prefix;
   int num_groups;
+  // FP8 (E4M3) cache: codes of value / scale.  The K scale is folded into
+  // scale_log2; v_scale multiplies the output; the inverse scales quantise the
+  // fused append.
+  int kv_fp8;
+  float v_scale;
+  float k_inv_scale;
+  float v_inv_scale;
   const float* casc_partials;  // [B][Hq][CASCADE_SPLITS + 1][D + 4]: O, m (log2 units), l; the last slot
                                // holds this kernel's own unnormalised result of an unsplit segment
 };
@@ -135,6 +142,9 @@ int encode_kv_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_
 int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache, const int32_t* slot_mapping,
                   int num_tokens, int num_blocks, int num_kv_heads, int head_dim, int block_size, int* dev_status,
                   cudaStream_t stream, int num_sms);
+int launch_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                      const int32_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads, int head_dim,
+                      int block_size, float k_inv, float v_inv, int* dev_status, cudaStream_t stream, int num_sms);
 int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
                 cudaStream_t stream, int num_sms);
 // Workspace of the rows kernel for at most num_rows query rows on a device with
@@ -159,6 +169,7 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                   int total_q_tokens, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                   int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
                   void* stream, const void* k_new = nullptr, const void* v_new = nullptr,
-                  const int32_t* group_start = nullptr, const int32_t* group_prefix = nullptr, int num_groups = 0);
+                  const int32_t* group_start = nullptr, const int32_t* group_prefix = nullptr, int num_groups = 0,
+                  int kv_fp8 = 0, float k_scale = 1.f, float v_scale = 1.f);
 
 }  // namespace pa

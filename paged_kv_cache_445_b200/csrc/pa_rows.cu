@@ -193,11 +193,10 @@ __device__ __forceinline__ int bt_lookup(const RowsParams& p, BtWindow& w, int s
 
 __device__ __forceinline__ long long range_start(long long w, long long T, long long W) { return T * w / W; }
 
-template <int D, int NT>
+template <int D, int NT, bool F8 = false>
 struct RowsShape {
   static constexpr int KT = D / 16;                    // k-steps of QK^T, m-tiles of PV
-  static constexpr int PIECES = D / 64;                // 64-column TMA boxes per row
-  static constexpr int HALF_BYTES = TILE_KEYS * D * 2; // K (or V) bytes of a tile
+  static constexpr int HALF_BYTES = TILE_KEYS * D * (F8 ? 1 : 2);  // K (or V) bytes of a tile
   static constexpr int STAGE_BYTES = 2 * HALF_BYTES;
   static constexpr int SLOT_O = KT * NT * 32 * 4;      // O^T fragment floats of a partial
   static constexpr int SLOT_M = SLOT_O;                // running maxima (8 NT floats)
@@ -207,10 +206,30 @@ struct RowsShape {
 };
 
 // Write normalised O for one segment: O^T fragments -> bf16 -> movmatrix -> rows of out.
-template <int D, int NT>
+// FP8 caches: the accumulator rows g and g + 8 of m-tile mt are head-dim
+// 16 mt + 2g and 16 mt + 2g + 1 (the order the E4M3 V fragments are built in),
+// so each lane stores its two heads' pairs directly; O also takes the V scale.
+template <int D, int NT, bool F8 = false>
 __device__ __forceinline__ void store_output(const RowsParams& p, const float (&o)[D / 16][NT][4],
                                              const float (&l)[NT][2], int row, int kvh, int lane) {
   const int g = lane >> 2, c = lane & 3;
+  if constexpr (F8) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int head = nt * 8 + 2 * c + e;
+        const float inv = p.v_scale / l[nt][e];
+        __nv_bfloat16* base = static_cast<__nv_bfloat16*>(p.out) +
+                              (static_cast<long long>(row) * p.num_q_heads + kvh * p.group + head) * D + 2 * g;
+        if (head < p.group) {
+#pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt)
+            *reinterpret_cast<uint32_t*>(base + 16 * mt) = pack_bf16x2(o[mt][nt][e] * inv, o[mt][nt][2 + e] * inv);
+        }
+      }
+    return;
+  }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const float inv0 = 1.f / l[nt][0], inv1 = 1.f / l[nt][1];
@@ -360,9 +379,9 @@ __device__ __forceinline__ void store_own_partial(const RowsParams& p, const flo
 // and write the normalised output row.  Piece k recorded (slot, tiles) at the
 // table entry of its first unit, so the walk visits the pieces in order; one
 // pass with a running maximum.
-template <int D, int NT>
+template <int D, int NT, bool F8>
 __device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, int n, int row, int kvh, int lane) {
-  using S = RowsShape<D, NT>;
+  using S = RowsShape<D, NT, F8>;
   constexpr int KT = S::KT;
   const int c = lane & 3;
   float mm[NT][2], acc[KT][NT][4], ll[NT][2];
@@ -412,7 +431,18 @@ __device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, 
       fold_prefix<D, NT>(p, 0, cascade_splits(span), acc, mm, ll, row, kvh, lane);
     }
   }
-  store_output<D, NT>(p, acc, ll, row, kvh, lane);
+  store_output<D, NT, F8>(p, acc, ll, row, kvh, lane);
+}
+
+// 8 bf16 (one 16-byte vector) -> 8 E4M3 codes of value * inv_scale (the
+// product in binary32, then nearest-even with saturation).
+__device__ __forceinline__ uint32_t bf16x2_bits_to_e4m3x2(uint32_t w, float inv) {
+  const float lo = __uint_as_float(w << 16) * inv, hi = __uint_as_float(w & 0xffff0000u) * inv;
+  return f32x2_to_e4m3x2(lo, hi);
+}
+__device__ __forceinline__ uint2 quantize8(uint4 x, float inv) {
+  return make_uint2(bf16x2_bits_to_e4m3x2(x.x, inv) | (bf16x2_bits_to_e4m3x2(x.y, inv) << 16),
+                    bf16x2_bits_to_e4m3x2(x.z, inv) | (bf16x2_bits_to_e4m3x2(x.w, inv) << 16));
 }
 
 // Fused cache append (decode): write row s of k_new / v_new, sequence s's
@@ -420,9 +450,9 @@ __device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, 
 // head, 16-byte vectors over the whole grid.  The attention does not read
 // these bytes back (it takes the newest key from k_new / v_new), so nothing
 // waits for the stores.
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ void fused_append(const RowsParams& p, long long tid, long long nthreads) {
-  constexpr int VEC = D / 8;
+  constexpr int VEC = D / 8;  // 16-byte vectors of a bf16 row
   const long long n = static_cast<long long>(p.num_seqs) * p.num_kv_heads * VEC;
   for (long long i = tid; i < n; i += nthreads) {
     const int v = static_cast<int>(i % VEC);
@@ -440,8 +470,15 @@ __device__ __forceinline__ void fused_append(const RowsParams& p, long long tid,
     const long long src = sh * VEC + v;
     const long long dst = ((static_cast<long long>(blk) * p.num_kv_heads + h) * p.block_size + pos % p.block_size) *
                               VEC + v;
-    reinterpret_cast<uint4*>(p.k_cache)[dst] = __ldg(reinterpret_cast<const uint4*>(p.k_new) + src);
-    reinterpret_cast<uint4*>(p.v_cache)[dst] = __ldg(reinterpret_cast<const uint4*>(p.v_new) + src);
+    const uint4 kx = __ldg(reinterpret_cast<const uint4*>(p.k_new) + src);
+    const uint4 vx = __ldg(reinterpret_cast<const uint4*>(p.v_new) + src);
+    if constexpr (F8) {  // 8 bf16 -> 8 E4M3 codes of value / scale (8 bytes)
+      reinterpret_cast<uint2*>(p.k_cache)[dst] = quantize8(kx, p.k_inv_scale);
+      reinterpret_cast<uint2*>(p.v_cache)[dst] = quantize8(vx, p.v_inv_scale);
+    } else {
+      reinterpret_cast<uint4*>(p.k_cache)[dst] = kx;
+      reinterpret_cast<uint4*>(p.v_cache)[dst] = vx;
+    }
   }
 }
 
@@ -453,11 +490,11 @@ struct TileMeta {
   int flags;  // bit 0: first tile of this warp's range, bit 1: last tile of it
 };
 
-template <int D, int NT, int R>
+template <int D, int NT, int R, bool F8>
 __global__ void __launch_bounds__(ROWS_THREADS, 1)
     rows_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 const RowsParams p) {
-  using S = RowsShape<D, NT>;
+  using S = RowsShape<D, NT, F8>;
   constexpr int KT = S::KT;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[ROWS_WARPS][R];
@@ -581,12 +618,14 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
     for (int k = 0; k < R && loading; ++k) issue(k);
     // the first tiles are in flight: do this thread's share of the fused append meanwhile
     if (p.k_new)
-      fused_append<D>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
+      fused_append<D, F8>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
                       static_cast<long long>(gridDim.x) * ROWS_THREADS);
 
     float o[KT][NT][4];
     uint32_t qb[NT][KT][2];
-    constexpr int NEWV = (2 * D / 8 + 31) / 32;  // 16-byte vectors of the newest K and V row per lane
+    // 16-byte chunks of the newest K and V row (as the cache stores them) per lane
+    constexpr int NCHUNK = F8 ? D / 16 : D / 8;
+    constexpr int NEWV = (2 * NCHUNK + 31) / 32;
     uint4 newkv[NEWV];
     float m[NT][2], l[NT][2];
     bool began = false;
@@ -609,11 +648,18 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
         if (p.k_new) {  // fused append: the segment's newest key and value come from k_new / v_new
 #pragma unroll
           for (int k = 0; k < NEWV; ++k) {
-            const int c = lane + 32 * k;
-            if (c < 2 * D / 8) {
-              const uint4* src = reinterpret_cast<const uint4*>(c < D / 8 ? p.k_new : p.v_new) +
-                                 (static_cast<long long>(tm.row) * p.num_kv_heads + tm.h) * (D / 8) + c % (D / 8);
-              newkv[k] = __ldg(src);
+            const int ch = lane + 32 * k;
+            if (ch < 2 * NCHUNK) {
+              const uint4* row = reinterpret_cast<const uint4*>(ch < NCHUNK ? p.k_new : p.v_new) +
+                                 (static_cast<long long>(tm.row) * p.num_kv_heads + tm.h) * (D / 8);
+              if constexpr (F8) {  // 16 bf16 -> 16 codes, quantised as the append quantises them
+                const float inv = ch < NCHUNK ? p.k_inv_scale : p.v_inv_scale;
+                const uint2 a = quantize8(__ldg(row + 2 * (ch % NCHUNK)), inv);
+                const uint2 b = quantize8(__ldg(row + 2 * (ch % NCHUNK) + 1), inv);
+                newkv[k] = make_uint4(a.x, a.y, b.x, b.y);
+              } else {
+                newkv[k] = __ldg(row + ch % NCHUNK);
+              }
             }
           }
         }
@@ -626,8 +672,16 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
               (static_cast<long long>(tm.row) * p.num_q_heads + tm.h * p.group + (ok ? head : 0)) * D);
 #pragma unroll
           for (int kk = 0; kk < KT; ++kk) {
-            qb[nt][kk][0] = ok ? __ldg(qp + 8 * kk + c) : 0u;
-            qb[nt][kk][1] = ok ? __ldg(qp + 8 * kk + 4 + c) : 0u;
+            if constexpr (F8) {
+              // f16 B fragment in the head-dim order of the E4M3 K fragments:
+              // k-step kk, lane column c covers head-dim 16 kk + 4c .. + 3
+              const uint2 w = ok ? __ldg(reinterpret_cast<const uint2*>(qp + 8 * kk + 2 * c)) : make_uint2(0u, 0u);
+              qb[nt][kk][0] = pack_f16x2(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+              qb[nt][kk][1] = pack_f16x2(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+            } else {
+              qb[nt][kk][0] = ok ? __ldg(qp + 8 * kk + c) : 0u;
+              qb[nt][kk][1] = ok ? __ldg(qp + 8 * kk + 4 + c) : 0u;
+            }
           }
           m[nt][0] = m[nt][1] = -INFINITY;
           l[nt][0] = l[nt][1] = 0.f;
@@ -644,10 +698,10 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
         // copy brought (the append of this very launch may not have landed)
 #pragma unroll
         for (int k = 0; k < NEWV; ++k) {
-          const int c = lane + 32 * k;
-          if (c < 2 * D / 8) {
-            const int idx = c % (D / 8);
-            *reinterpret_cast<uint4*>((c < D / 8 ? kt : vt) + (idx >> 3) * 2048 + sw128(nvalid - 1, idx & 7)) =
+          const int ch = lane + 32 * k;
+          if (ch < 2 * NCHUNK) {
+            const int idx = ch % NCHUNK;
+            *reinterpret_cast<uint4*>((ch < NCHUNK ? kt : vt) + (idx >> 3) * 2048 + sw128(nvalid - 1, idx & 7)) =
                 newkv[k];
           }
         }
@@ -664,11 +718,38 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       const int mi = lane >> 3;
       const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
       auto load_v = [&]() {
-        const int rv = (lane & 7) + (mi >> 1) * 8;
+        if constexpr (F8) {
+          // E4M3 V: one ldmatrix.trans of byte pairs covers m-tiles X, X + 1
+          // (16-byte chunks X, X + 1 = head-dim 16X .. 16X + 31) for keys 0-7
+          // and 8-15.  A lane receives keys 2c, 2c+1 at head-dim 2g, 2g+1 of
+          // the chunk; pairing the bytes by head-dim gives the f16 A rows
+          // g (head-dim 16X + 2g) and g + 8 (head-dim 16X + 2g + 1).
+          const int rv = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-        for (int mt = 0; mt < KT; ++mt) {
-          const int cg = 2 * mt + (mi & 1);
-          ldsm_x4_trans(vbase + (cg >> 3) * 2048 + sw128(rv, cg & 7), vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3]);
+          for (int x = 0; x < KT; x += 2) {
+            const int ch = x + (lane >> 4);
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_trans(vbase + (ch >> 3) * 2048 + sw128(rv, ch & 7), r0, r1, r2, r3);
+            r0 = pair_bytes(r0);
+            r1 = pair_bytes(r1);
+            r2 = pair_bytes(r2);
+            r3 = pair_bytes(r3);
+            vf[x][0] = e4m3x2_lo_to_f16x2(r0);
+            vf[x][1] = e4m3x2_hi_to_f16x2(r0);
+            vf[x][2] = e4m3x2_lo_to_f16x2(r1);
+            vf[x][3] = e4m3x2_hi_to_f16x2(r1);
+            vf[x + 1][0] = e4m3x2_lo_to_f16x2(r2);
+            vf[x + 1][1] = e4m3x2_hi_to_f16x2(r2);
+            vf[x + 1][2] = e4m3x2_lo_to_f16x2(r3);
+            vf[x + 1][3] = e4m3x2_hi_to_f16x2(r3);
+          }
+        } else {
+          const int rv = (lane & 7) + (mi >> 1) * 8;
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            const int cg = 2 * mt + (mi & 1);
+            ldsm_x4_trans(vbase + (cg >> 3) * 2048 + sw128(rv, cg & 7), vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3]);
+          }
         }
         if (nvalid < TILE_KEYS) {
           // keys past the context may hold anything (even NaN): their V rows must
@@ -692,7 +773,27 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
           issue(stage);
         }
       };
-      {
+      if constexpr (F8) {
+        // E4M3 K: one ldmatrix of byte pairs covers k-steps X, X + 1 (16-byte
+        // chunks X, X + 1) for keys 0-7 and 8-15.  A lane receives head-dim
+        // 4c .. 4c+3 of the chunk; its low pair is the f16 A column pair 2c, 2c+1
+        // of the k-step and its high pair the pair 2c+8, 2c+9 (Q uses the same order).
+        const int rk = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int x = 0; x < KT; x += 2) {
+          const int ch = x + (lane >> 4);
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(kbase + (ch >> 3) * 2048 + sw128(rk, ch & 7), r0, r1, r2, r3);
+          kf[x][0] = e4m3x2_lo_to_f16x2(r0);
+          kf[x][1] = e4m3x2_lo_to_f16x2(r1);
+          kf[x][2] = e4m3x2_hi_to_f16x2(r0);
+          kf[x][3] = e4m3x2_hi_to_f16x2(r1);
+          kf[x + 1][0] = e4m3x2_lo_to_f16x2(r2);
+          kf[x + 1][1] = e4m3x2_lo_to_f16x2(r3);
+          kf[x + 1][2] = e4m3x2_hi_to_f16x2(r2);
+          kf[x + 1][3] = e4m3x2_hi_to_f16x2(r3);
+        }
+      } else {
         const int rk = (lane & 7) + (mi & 1) * 8;
 #pragma unroll
         for (int kk = 0; kk < KT; ++kk)
@@ -710,8 +811,12 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       for (int nt = 0; nt < NT; ++nt) {
         sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
 #pragma unroll
-        for (int kk = 0; kk < KT; ++kk)
-          mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
+        for (int kk = 0; kk < KT; ++kk) {
+          if constexpr (F8)
+            mma_f16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
+          else
+            mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
+        }
       }
 
       // online softmax on the fragment: this lane holds keys g, g+8 of heads 2c, 2c+1
@@ -740,8 +845,13 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
         const float p1 = fast_exp2(s1 - mn1), p3 = fast_exp2(s3 - mn1);
         l[nt][0] = l[nt][0] * al[nt][0] + p0 + p2;
         l[nt][1] = l[nt][1] * al[nt][1] + p1 + p3;
-        pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
-        pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+        if constexpr (F8) {  // P in f16 for the f16 MMA
+          pb[nt][0] = movmatrix_trans(pack_f16x2(p0, p1));
+          pb[nt][1] = movmatrix_trans(pack_f16x2(p2, p3));
+        } else {
+          pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+          pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+        }
       }
       if (__any_sync(FULL_MASK, moved)) {  // rescale O only when some running maximum grew
 #pragma unroll
@@ -763,8 +873,12 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
 #pragma unroll
       for (int mt = 0; mt < KT; ++mt)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-          mma_bf16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          if constexpr (F8)
+            mma_f16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+          else
+            mma_bf16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+        }
 
       // ---- end of a piece: write the output, or a partial linked to its segment
       if (tm.t == tm.n - 1 || run_end) {
@@ -785,7 +899,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
           if (lane == 0)
             p.seginfo[static_cast<long long>(tm.row) * p.num_kv_heads + tm.h] = (tm.u - tm.t) + 1;  // no pieces
         } else if (began && tm.t == tm.n - 1) {
-          store_output<D, NT>(p, o, l, tm.row, tm.h, lane);
+          store_output<D, NT, F8>(p, o, l, tm.row, tm.h, lane);
         } else if (nslots < ROWS_SLOTS_PER_WARP) {
           const long long slot = static_cast<long long>(gw) * ROWS_SLOTS_PER_WARP + nslots++;
           float* ps = p.partials + slot * S::SLOT_FLOATS;
@@ -824,7 +938,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
   }
 
   if (gw >= W && p.k_new)  // warps without tiles still take their share of the fused append
-    fused_append<D>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
+    fused_append<D, F8>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
                     static_cast<long long>(gridDim.x) * ROWS_THREADS);
 
   // ---- grid barrier: every partial and table entry is stored before any merge reads it
@@ -848,7 +962,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
   for (long long seg = gw; seg < nseg; seg += p.total_warps) {
     const long long info = __ldcg(p.seginfo + seg);
     if (info == 0) continue;
-    merge_segment<D, NT>(p, (info & ((1ll << 40) - 1)) - 1, static_cast<int>(info >> 40),
+    merge_segment<D, NT, F8>(p, (info & ((1ll << 40) - 1)) - 1, static_cast<int>(info >> 40),
                          static_cast<int>(seg / p.num_kv_heads), static_cast<int>(seg % p.num_kv_heads), lane);
     if (lane == 0) p.seginfo[seg] = 0;
   }
@@ -866,12 +980,12 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
 
 // ------------------------------------------------------------------ host side
 
-template <int D, int NT, int R>
+template <int D, int NT, int R, bool F8 = false>
 static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream,
                          int num_sms) {
-  using S = RowsShape<D, NT>;
+  using S = RowsShape<D, NT, F8>;
   const int smem = ROWS_WARPS * R * S::STAGE_BYTES + 1024 + (ROWS_SMEM_SEQS + 1) * 8;
-  auto kern = rows_kernel<D, NT, R>;
+  auto kern = rows_kernel<D, NT, R, F8>;
   static int configured_dev = -1;
   static int blocks_per_sm = 1;
   int dev = 0;
@@ -961,6 +1075,17 @@ void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_h
 int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
                 cudaStream_t stream, int num_sms) {
   const bool two = p.group > 8;
+  if (p.kv_fp8) {  // E4M3 caches: a tile is half the bytes, so twice the stages
+    switch (head_dim) {
+      case 128:
+        return two ? launch_rows_t<128, 2, 6, true>(p, tmk, tmv, stream, num_sms)
+                   : launch_rows_t<128, 1, 6, true>(p, tmk, tmv, stream, num_sms);
+      case 256:
+        return launch_rows_t<256, 1, 3, true>(p, tmk, tmv, stream, num_sms);
+      default:
+        return PA_ERR_UNSUPPORTED;
+    }
+  }
   switch (head_dim) {
     case 64:
       return two ? launch_rows_t<64, 2, 8>(p, tmk, tmv, stream, num_sms)

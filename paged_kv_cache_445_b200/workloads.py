@@ -257,6 +257,36 @@ def build(spec: Spec, seed: int, poison: bool = False, max_blocks: int | None = 
                     spec.share_tokens, tuple(groups))
 
 
+E4M3_NAN = np.uint8(0x7F)
+
+
+def fp8_caches(w: Workload, seed: int, poison: bool = False):
+    """Synthetic contents of an FP8 (E4M3 code) cache of w's shape: codes with
+    a random sign, exponent field 3..9 and mantissa (values 2^-4 .. 3.75 before
+    the scale), and the per-tensor scales (0.5 for K, 0.25 for V).  With
+    ``poison`` every slot that does not hold a valid earlier token holds the
+    NaN code.  Returns (k_codes, v_codes, k_scale, v_scale)."""
+    out = []
+    for stream in (11, 12):
+        g = np.random.Generator(np.random.PCG64(seed).jumped(stream))
+        shape = w.k_cache.shape
+        sign = g.integers(0, 2, size=shape, dtype=np.uint8) << 7
+        exp = g.integers(3, 10, size=shape, dtype=np.uint8) << 3
+        man = g.integers(0, 8, size=shape, dtype=np.uint8)
+        out.append((sign | exp | man).astype(np.uint8))
+    kc, vc = out
+    if poison:
+        bad = np.ones((w.num_blocks, w.block_size), dtype=bool)
+        qs = w.query_start
+        for s in range(w.num_seqs):
+            prefix = int(w.context_lens[s]) - int(qs[s + 1] - qs[s])
+            pos = np.arange(prefix, dtype=np.int64)
+            bad[w.block_tables[s, pos // w.block_size], pos % w.block_size] = False
+        kc.transpose(0, 2, 1, 3)[bad] = E4M3_NAN
+        vc.transpose(0, 2, 1, 3)[bad] = E4M3_NAN
+    return kc, vc, 0.5, 0.25
+
+
 def standard(cfg: int, seed: int | None = None, poison: bool = False) -> Workload:
     seed = 445 + cfg if seed is None else seed
     return build(standard_spec(cfg, seed), seed, poison=poison)

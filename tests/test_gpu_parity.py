@@ -310,3 +310,36 @@ def test_small_workspace_is_rejected():
     with pytest.raises(pa.PAError) as e:
         ds.attend()
     assert e.value.code == pa._binding.PA_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("cfg", [3, 5])
+def test_a_captured_step_replays_bit_identically(cfg):
+    # the step's launches (cooperative, programmatic dependent launch) captured
+    # in a CUDA graph: replays give the eager result, bit for bit
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.standard(cfg)
+    ds = DeviceStep(w)
+    kc0, vc0 = ds.k_cache.clone(), ds.v_cache.clone()
+
+    def step():
+        if w.is_decode:
+            pa.pa_decode_append(ds.out, ds.q, ds.k_new, ds.v_new, ds.k_cache, ds.v_cache, ds.block_tables,
+                                ds.context_lens, w.scale, ds.workspace, ds.status)
+        else:
+            ds.append()
+            ds.attend()
+
+    step()
+    torch.cuda.synchronize()
+    eager = ds.out.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(2):
+        ds.out.fill_(0)
+        ds.k_cache.copy_(kc0)
+        ds.v_cache.copy_(vc0)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert int(ds.status.item()) == 0
+        assert torch.equal(ds.out.view(torch.int16), eager.view(torch.int16))
