@@ -237,7 +237,7 @@ class GpuStep:
     fused launch (pa_decode_append) unless fused=False; a mixed batch runs
     pa_cache_append then pa_prefill_chunk."""
 
-    def __init__(self, w, device, fused=True, cascade=True):
+    def __init__(self, w, device, fused=True, cascade=True, fp8=False):
         import torch
 
         import paged_kv_cache_445_b200 as pa
@@ -257,6 +257,12 @@ class GpuStep:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.decode = w.is_decode
         self.fused = self.decode and fused
+        self.fp8 = fp8
+        if fp8:  # E4M3 codes with per-tensor scales (decode batches only)
+            if not self.decode:
+                raise SystemExit("--kv-dtype fp8 is a decode path")
+            kc, vc, self.k_scale, self.v_scale = workloads_fp8_caches(w)
+            self.k_cache, self.v_cache = torch.from_numpy(kc).to(device), torch.from_numpy(vc).to(device)
         groups = w.prefix_groups() if self.decode and cascade else None
         self.cascade = groups is not None
         if self.cascade:  # shared prefixes read once per group (pa_decode_cascade)
@@ -281,10 +287,19 @@ class GpuStep:
     def append(self):
         if self.fused:
             return  # part of the attention launch
+        if self.fp8:
+            self.pa.pa_cache_append_fp8(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping,
+                                        self.k_scale, self.v_scale, self.status)
+            return
         self.pa.pa_cache_append(self.k_new, self.v_new, self.k_cache, self.v_cache, self.slot_mapping, self.status)
 
     def attend(self):
-        if self.cascade:
+        if self.fp8:
+            self.pa.pa_decode_fp8(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
+                                  self.w.scale, self.k_scale, self.v_scale, self.workspace,
+                                  k_new=self.k_new if self.fused else None, v_new=self.v_new if self.fused else None,
+                                  dev_status=self.status)
+        elif self.cascade:
             self.pa.pa_decode_cascade(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                                       self.context_lens, self.w.scale, self.group_start, self.group_prefix,
                                       self.workspace, k_new=self.k_new if self.fused else None,
@@ -300,6 +315,11 @@ class GpuStep:
                                      self.block_tables, self.context_lens, self.w.scale, self.workspace, self.status)
 
 
+def workloads_fp8_caches(w):
+    from paged_kv_cache_445_b200 import workloads
+    return workloads.fp8_caches(w, seed=445)
+
+
 def run_ours(args, peaks):
     import torch
 
@@ -310,8 +330,12 @@ def run_ours(args, peaks):
     w = workloads.standard(args.workload, seed=rank_seed(args.workload, rank))
     log(f"[rank {rank}] workload {w.name}: {w.num_seqs} seqs, {w.num_query_tokens} query rows, "
         f"{int(w.context_lens.sum())} keys, pool {w.num_blocks} blocks ({time.time() - t0:.1f}s to generate)")
-    g = GpuStep(w, device, fused=not args.separate_append, cascade=args.cascade)
+    g = GpuStep(w, device, fused=not args.separate_append, cascade=args.cascade, fp8=args.kv_dtype == "fp8")
     kv_bytes, attn_bytes, app_bytes, flops = step_bytes(w)
+    if g.fp8:  # one byte per cached element instead of two; the appended rows are written as bytes too
+        attn_bytes -= kv_bytes // 2
+        app_bytes -= len(w.slot_mapping) * w.num_kv_heads * w.head_dim * 2
+        kv_bytes //= 2
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
@@ -414,7 +438,7 @@ def run_ours(args, peaks):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "fp8-e4m3 cache, bf16 q/out" if g.fp8 else "bf16",
         "data": "synthetic (seeded PCG64, bf16 N(0,1) K/V, q N(0,0.5^2)); no weights",
         "config": {
             "workload": w.name, "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
@@ -430,7 +454,8 @@ def run_ours(args, peaks):
         "frac_of_hbm_peak": round(compose_value(total_kv, ms_step) / hbm / world, 4),
         "frac_of_8tbs_nominal": round(compose_value(total_kv, ms_step) / 8000.0 / world, 4),
         "roofline": {
-            "kernel": ("pa_cascade_kernel + pa_rows_kernel (shared prefixes once, then the private keys)"
+            "kernel": ("pa_rows_kernel, FP8 E4M3 cache (append + attention, one launch)" if g.fp8 else
+                       "pa_cascade_kernel + pa_rows_kernel (shared prefixes once, then the private keys)"
                        if g.cascade else
                        "pa_rows_kernel (append + attention, one launch)" if g.fused else "pa_rows_kernel (attention)"),
             "bound": "hbm",
@@ -553,6 +578,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-dtype", default="bf16", choices=["bf16", "fp8"],
+                    help="fp8: the cache holds E4M3 codes with per-tensor scales (decode workloads)")
     ap.add_argument("--graph", action="store_true",
                     help="capture one step (all its launches) in a CUDA graph and time its replays")
     ap.add_argument("--cascade", action="store_true",
