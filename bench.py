@@ -75,10 +75,10 @@ def kernel_source_hash(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str, workload: str):
+def profiled_traffic(kernel: str, workload: str, variant: str = ""):
     """dram read+write bytes per launch from a committed ncu summary, if it was
     taken on the current kernel sources; else None."""
-    path = os.path.join(PROFILE_DIR, f"{kernel}_{workload}.md")
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{workload}{variant}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -417,18 +417,20 @@ def run_ours(args, peaks):
     # ---- CPU baseline: the oracle on this host's cores, rank 0 at N = 1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_baseline(w, args.cpu_seconds)
+        cpu = oracle_baseline(w, args.cpu_seconds, fp8=g.fp8)
 
     clocks = sampler.summary()
     hbm, bf16_burst, bf16_sust, peak_src = peaks
     from paged_kv_cache_445_b200 import roofline as _rl
     unique_kv = _rl.unique_kv_bytes(w.block_tables, w.context_lens, w.block_size, w.num_kv_heads, w.head_dim)
+    if g.fp8:
+        unique_kv //= 2
     if g.cascade:  # a shared prefix crosses HBM once: the algorithmic bytes are the unique ones
         attn_bytes = attn_bytes - kv_bytes + unique_kv
     # the timed launch (or replay) also appends when fused or replayed as a graph
     launch_bytes = attn_bytes + (app_bytes if (g.fused or graph is not None) else 0)
     achieved = launch_bytes / (attn_avg_ms * 1e-3) / 1e9
-    traffic = profiled_traffic("pa_rows_kernel", w.name)
+    traffic = profiled_traffic("pa_rows_kernel", w.name, "-fp8" if g.fp8 else "")
     line = {
         "metric": "paged-attn decode KV GB/s + seq-steps/s (70B layer, bs128); % of HBM peak",
         "value": round(compose_value(total_kv, ms_step), 2),
@@ -500,18 +502,28 @@ def oracle_sample(w, max_rows: int):
     return oracle, only, seqs, roofline.kv_cache_bytes(1, w.num_kv_heads, w.head_dim, keys)
 
 
-def oracle_step(oracle, w, only, kc, vc):
+def oracle_step(oracle, w, only, kc, vc, scales=None):
     slots = oracle.slot_mapping(w.block_tables, w.context_lens, w.query_start, w.block_size, w.num_blocks)
+    if scales is not None:  # E4M3 cache: (k_scale, v_scale)
+        oracle.cache_append_fp8(w.k_new, w.v_new, kc, vc, slots, *scales)
+        oracle.paged_attention_fp8(w.q, kc, vc, w.block_tables, w.context_lens, w.query_start, w.scale, *scales,
+                                   only=only)
+        return
     oracle.cache_append(w.k_new, w.v_new, kc, vc, slots)
     oracle.paged_attention(w.q, kc, vc, w.block_tables, w.context_lens, w.query_start, w.scale, only=only)
 
 
-def oracle_baseline(w, seconds: float, max_rows: int = 16):
+def oracle_baseline(w, seconds: float, max_rows: int = 16, fp8: bool = False):
     oracle, only, seqs, sample_bytes = oracle_sample(w, max_rows)
-    kc, vc = w.k_cache, w.v_cache  # appended in place: the same rows every step
+    scales = None
+    if fp8:
+        kc, vc, k_scale, v_scale = workloads_fp8_caches(w)
+        scales, sample_bytes = (k_scale, v_scale), sample_bytes // 2
+    else:
+        kc, vc = w.k_cache, w.v_cache  # appended in place: the same rows every step
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(oracle, w, only, kc, vc)
+        oracle_step(oracle, w, only, kc, vc, scales)
         n += 1
         if time.perf_counter() - t0 >= seconds:
             break
