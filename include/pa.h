@@ -260,7 +260,7 @@ PA_API int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start
  * (64 MiB), part of the library's device image, so this call allocates
  * nothing.  A batch whose pa_workspace_bytes(num_seqs, ...) exceeds that size
  * is rejected with PA_ERR_WORKSPACE before any launch (for example, 8 query
- * heads per KV head at head_dim 128 on a 148-SM B200 fits about 1,700
+ * heads per KV head at head_dim 128 on a 148-SM B200 fits about 1,570
  * sequences with 512-block tables).
  *
  * Sharing: every call on a device uses the same array.  Calls that overlap in

@@ -43,6 +43,7 @@ constexpr int ROWS_WARPS = 4;
 constexpr int ROWS_THREADS = ROWS_WARPS * 32;
 constexpr int ROWS_SLOTS_PER_WARP = 2;  // a warp's range cuts at most its first and its last segment
 constexpr int ROWS_SMEM_SEQS = ROWS_SMEM_SEQS_HOST;  // sequences whose tile prefix sums live in shared memory
+constexpr int ROWS_MAX_CTAS_PER_SM = 3;  // the workspace holds partial slots for this many CTAs per SM
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -490,8 +491,16 @@ struct TileMeta {
   int flags;  // bit 0: first tile of this warp's range, bit 1: last tile of it
 };
 
+// CTAs per SM a variant is compiled for: the E4M3 kernel with one head tile
+// is bound by instruction latency (the code conversions), so it runs three
+// CTAs per SM (12 warps) in at most 168 registers; the others run two.
+template <int D, int NT, bool F8>
+constexpr int rows_ctas_per_sm() {
+  return (F8 && D == 128 && NT == 1) ? 3 : 2;
+}
+
 template <int D, int NT, int R, bool F8>
-__global__ void __launch_bounds__(ROWS_THREADS, 1)
+__global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() == 3 ? 3 : 1)
     rows_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 const RowsParams p) {
   using S = RowsShape<D, NT, F8>;
@@ -711,9 +720,10 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       // Pull the tile into registers (K as the A operand of S^T = K Q^T, V^T via
       // ldmatrix.trans as the A operand of O^T += V^T P^T) and hand the stage
       // back to TMA at once, so the ring never waits on the math.  With
-      // head_dim 256 both fragments would not fit in registers: V is read after
-      // the softmax and the stage is released then.
-      constexpr bool kEarly = D <= 128;
+      // head_dim 256 both bf16 fragments would not fit in registers: V is read
+      // after the softmax and the stage is released then (E4M3 codes, one byte
+      // each, fit).
+      constexpr bool kEarly = D <= 128 || F8;
       uint32_t kf[KT][4], vf[KT][4];
       const int mi = lane >> 3;
       const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
@@ -722,26 +732,15 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
           // E4M3 V: one ldmatrix.trans of byte pairs covers m-tiles X, X + 1
           // (16-byte chunks X, X + 1 = head-dim 16X .. 16X + 31) for keys 0-7
           // and 8-15.  A lane receives keys 2c, 2c+1 at head-dim 2g, 2g+1 of
-          // the chunk; pairing the bytes by head-dim gives the f16 A rows
-          // g (head-dim 16X + 2g) and g + 8 (head-dim 16X + 2g + 1).
+          // the chunk.  The bytes stay packed in vf[X / 2]; the product loop
+          // pairs them by head-dim into the f16 A rows g (head-dim 16X + 2g)
+          // and g + 8 (head-dim 16X + 2g + 1).
           const int rv = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
           for (int x = 0; x < KT; x += 2) {
             const int ch = x + (lane >> 4);
-            uint32_t r0, r1, r2, r3;
-            ldsm_x4_trans(vbase + (ch >> 3) * 2048 + sw128(rv, ch & 7), r0, r1, r2, r3);
-            r0 = pair_bytes(r0);
-            r1 = pair_bytes(r1);
-            r2 = pair_bytes(r2);
-            r3 = pair_bytes(r3);
-            vf[x][0] = e4m3x2_lo_to_f16x2(r0);
-            vf[x][1] = e4m3x2_hi_to_f16x2(r0);
-            vf[x][2] = e4m3x2_lo_to_f16x2(r1);
-            vf[x][3] = e4m3x2_hi_to_f16x2(r1);
-            vf[x + 1][0] = e4m3x2_lo_to_f16x2(r2);
-            vf[x + 1][1] = e4m3x2_hi_to_f16x2(r2);
-            vf[x + 1][2] = e4m3x2_lo_to_f16x2(r3);
-            vf[x + 1][3] = e4m3x2_hi_to_f16x2(r3);
+            ldsm_x4_trans(vbase + (ch >> 3) * 2048 + sw128(rv, ch & 7), vf[x / 2][0], vf[x / 2][1], vf[x / 2][2],
+                          vf[x / 2][3]);
           }
         } else {
           const int rv = (lane & 7) + (mi >> 1) * 8;
@@ -757,12 +756,22 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
           // 2c, 2c+1 (fragments 0, 1) and 8+2c, 9+2c (fragments 2, 3).
           const uint32_t lo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
           const uint32_t hi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+          if constexpr (F8) {  // packed codes: registers 0, 2 hold keys 2c, 2c+1 and 1, 3 keys 8+2c, 9+2c
 #pragma unroll
-          for (int mt = 0; mt < KT; ++mt) {
-            vf[mt][0] &= lo;
-            vf[mt][1] &= lo;
-            vf[mt][2] &= hi;
-            vf[mt][3] &= hi;
+            for (int x = 0; x < KT / 2; ++x) {
+              vf[x][0] &= lo;
+              vf[x][1] &= hi;
+              vf[x][2] &= lo;
+              vf[x][3] &= hi;
+            }
+          } else {
+#pragma unroll
+            for (int mt = 0; mt < KT; ++mt) {
+              vf[mt][0] &= lo;
+              vf[mt][1] &= lo;
+              vf[mt][2] &= hi;
+              vf[mt][3] &= hi;
+            }
           }
         }
       };
@@ -777,21 +786,14 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
         // E4M3 K: one ldmatrix of byte pairs covers k-steps X, X + 1 (16-byte
         // chunks X, X + 1) for keys 0-7 and 8-15.  A lane receives head-dim
         // 4c .. 4c+3 of the chunk; its low pair is the f16 A column pair 2c, 2c+1
-        // of the k-step and its high pair the pair 2c+8, 2c+9 (Q uses the same order).
+        // of the k-step and its high pair the pair 2c+8, 2c+9 (Q uses the same
+        // order).  The codes stay packed in kf[X / 2] until the product loop.
         const int rk = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
         for (int x = 0; x < KT; x += 2) {
           const int ch = x + (lane >> 4);
-          uint32_t r0, r1, r2, r3;
-          ldsm_x4(kbase + (ch >> 3) * 2048 + sw128(rk, ch & 7), r0, r1, r2, r3);
-          kf[x][0] = e4m3x2_lo_to_f16x2(r0);
-          kf[x][1] = e4m3x2_lo_to_f16x2(r1);
-          kf[x][2] = e4m3x2_hi_to_f16x2(r0);
-          kf[x][3] = e4m3x2_hi_to_f16x2(r1);
-          kf[x + 1][0] = e4m3x2_lo_to_f16x2(r2);
-          kf[x + 1][1] = e4m3x2_lo_to_f16x2(r3);
-          kf[x + 1][2] = e4m3x2_hi_to_f16x2(r2);
-          kf[x + 1][3] = e4m3x2_hi_to_f16x2(r3);
+          ldsm_x4(kbase + (ch >> 3) * 2048 + sw128(rk, ch & 7), kf[x / 2][0], kf[x / 2][1], kf[x / 2][2],
+                  kf[x / 2][3]);
         }
       } else {
         const int rk = (lane & 7) + (mi & 1) * 8;
@@ -808,15 +810,27 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
       // S^T[key, head] = K . Q^T
       float sacc[NT][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      if constexpr (F8) {  // E4M3 -> f16 just before each pair of k-steps
 #pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-          if constexpr (F8)
-            mma_f16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
-          else
-            mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
+        for (int x = 0; x < KT / 2; ++x) {
+          const uint32_t* r = kf[x];
+          const uint32_t a0 = e4m3x2_lo_to_f16x2(r[0]), a1 = e4m3x2_lo_to_f16x2(r[1]);
+          const uint32_t a2 = e4m3x2_hi_to_f16x2(r[0]), a3 = e4m3x2_hi_to_f16x2(r[1]);
+          const uint32_t b0 = e4m3x2_lo_to_f16x2(r[2]), b1 = e4m3x2_lo_to_f16x2(r[3]);
+          const uint32_t b2 = e4m3x2_hi_to_f16x2(r[2]), b3 = e4m3x2_hi_to_f16x2(r[3]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_f16_16816(sacc[nt], a0, a1, a2, a3, qb[nt][2 * x][0], qb[nt][2 * x][1]);
+            mma_f16_16816(sacc[nt], b0, b1, b2, b3, qb[nt][2 * x + 1][0], qb[nt][2 * x + 1][1]);
+          }
         }
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int kk = 0; kk < KT; ++kk)
+            mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
       }
 
       // online softmax on the fragment: this lane holds keys g, g+8 of heads 2c, 2c+1
@@ -870,15 +884,28 @@ __global__ void __launch_bounds__(ROWS_THREADS, 1)
         load_v();
         release();
       }
+      if constexpr (F8) {  // pair the codes by head-dim, E4M3 -> f16, two m-tiles per packed fragment
 #pragma unroll
-      for (int mt = 0; mt < KT; ++mt)
+        for (int x = 0; x < KT / 2; ++x) {
+          const uint32_t r0 = pair_bytes(vf[x][0]), r1 = pair_bytes(vf[x][1]);
+          const uint32_t r2 = pair_bytes(vf[x][2]), r3 = pair_bytes(vf[x][3]);
+          const uint32_t a0 = e4m3x2_lo_to_f16x2(r0), a1 = e4m3x2_hi_to_f16x2(r0);
+          const uint32_t a2 = e4m3x2_lo_to_f16x2(r1), a3 = e4m3x2_hi_to_f16x2(r1);
+          const uint32_t b0 = e4m3x2_lo_to_f16x2(r2), b1 = e4m3x2_hi_to_f16x2(r2);
+          const uint32_t b2 = e4m3x2_lo_to_f16x2(r3), b3 = e4m3x2_hi_to_f16x2(r3);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          if constexpr (F8)
-            mma_f16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
-          else
-            mma_bf16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_f16_16816(o[2 * x][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+            mma_f16_16816(o[2 * x + 1][nt], b0, b1, b2, b3, pb[nt][0], pb[nt][1]);
+          }
         }
+      } else {
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+      }
 
       // ---- end of a piece: write the output, or a partial linked to its segment
       if (tm.t == tm.n - 1 || run_end) {
@@ -996,7 +1023,8 @@ static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUt
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, ROWS_THREADS, smem) != cudaSuccess || nb < 1)
       return PA_ERR_CUDA;
-    blocks_per_sm = nb > 2 ? 2 : nb;
+    constexpr int cap = rows_ctas_per_sm<D, NT, F8>();
+    blocks_per_sm = nb > cap ? cap : nb;
     configured_dev = dev;
   }
   RowsParams p = p0;
@@ -1038,7 +1066,7 @@ size_t slot_bytes(int group, int head_dim) {
   const size_t o = static_cast<size_t>(head_dim / 16) * nt * 32 * 4;
   return (o + 16 * nt + 1 + 63) / 64 * 64 * sizeof(float);
 }
-size_t max_warps(int num_sms) { return static_cast<size_t>(num_sms) * 2 * ROWS_WARPS; }
+size_t max_warps(int num_sms) { return static_cast<size_t>(num_sms) * ROWS_MAX_CTAS_PER_SM * ROWS_WARPS; }
 }  // namespace
 
 namespace {
@@ -1075,11 +1103,11 @@ void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_h
 int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
                 cudaStream_t stream, int num_sms) {
   const bool two = p.group > 8;
-  if (p.kv_fp8) {  // E4M3 caches: a tile is half the bytes, so twice the stages
+  if (p.kv_fp8) {  // E4M3 caches: a tile is half the bytes, so more stages (or more CTAs) per SM
     switch (head_dim) {
       case 128:
         return two ? launch_rows_t<128, 2, 6, true>(p, tmk, tmv, stream, num_sms)
-                   : launch_rows_t<128, 1, 6, true>(p, tmk, tmv, stream, num_sms);
+                   : launch_rows_t<128, 1, 4, true>(p, tmk, tmv, stream, num_sms);
       case 256:
         return launch_rows_t<256, 1, 3, true>(p, tmk, tmv, stream, num_sms);
       default:
