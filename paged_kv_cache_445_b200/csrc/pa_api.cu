@@ -201,9 +201,31 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
     if ((rc = launch_cascade(c, q, k_cache, v_cache, total_q_tokens, head_dim, st, di.num_sms)) != PA_OK) return rc;
   }
   if (query_start && !kv_fp8 && chunk_supported(p.group, head_dim)) {
-    // sequences with more than one query row run on the tcgen05 chunk kernel,
-    // the single rows (decodes) on the rows kernel right after it
+    // sequences with 2 .. 64/G query rows run on the tcgen05 multi-row kernel,
+    // longer ones on the tcgen05 chunk kernel, the single rows (decodes) on the
+    // rows kernel after both
+    const bool verify = verify_supported(p.group, head_dim, num_seqs);
+    if (verify) {
+      VerifyParams v{};
+      v.out = out;
+      v.block_tables = block_tables;
+      v.context_lens = context_lens;
+      v.query_start = query_start;
+      v.num_seqs = num_seqs;
+      v.max_blocks = max_blocks;
+      v.num_q_heads = num_q_heads;
+      v.num_kv_heads = num_kv_heads;
+      v.group = p.group;
+      v.block_size = block_size;
+      v.num_blocks = num_blocks;
+      v.scale_log2 = p.scale_log2;
+      v.status = dev_status;
+      v.slots = p.partials;
+      v.counters = p.verify_counters;
+      if ((rc = launch_verify(v, q, k_cache, v_cache, total_q_tokens, st, di.num_sms)) != PA_OK) return rc;
+    }
     ChunkParams c{};
+    c.min_qlen = verify ? VERIFY_MAX_COLS / p.group + 1 : 2;
     c.out = out;
     c.block_tables = block_tables;
     c.context_lens = context_lens;

@@ -96,7 +96,7 @@ __device__ __forceinline__ bool chunk_item(const ChunkParams& p, int pair_tok, l
   long long base = 0;
   for (int s = 0; s < p.num_seqs; ++s) {
     const int q0 = __ldg(p.query_start + s), qlen = __ldg(p.query_start + s + 1) - q0;
-    if (qlen <= 1) continue;
+    if (qlen < p.min_qlen) continue;
     int ctx = __ldg(p.context_lens + s);
     const int cap = p.max_blocks * p.block_size;
     if (ctx > cap) ctx = cap;
@@ -122,7 +122,7 @@ __device__ __forceinline__ long long chunk_total(const ChunkParams& p, int pair_
   long long n = 0;
   for (int s = 0; s < p.num_seqs; ++s) {
     const int qlen = __ldg(p.query_start + s + 1) - __ldg(p.query_start + s);
-    if (qlen > 1) n += static_cast<long long>((qlen + pair_tok - 1) / pair_tok) * p.num_kv_heads;
+    if (qlen >= p.min_qlen) n += static_cast<long long>((qlen + pair_tok - 1) / pair_tok) * p.num_kv_heads;
   }
   return n;
 }
@@ -571,8 +571,8 @@ static int encode_q_tmap(CUtensorMap* map, const void* q, int total_q_tokens, in
 }
 
 // [num_blocks, Hkv, block_size, D] as a 4-D tensor; box = 64 columns x 16 rows of one (block, head).
-static int encode_kv16_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
-                            EncodeTiledFn fn) {
+int encode_kv16_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
+                     EncodeTiledFn fn) {
   const cuuint64_t row = CH_D * 2;
   const cuuint64_t dims[4] = {CH_D, static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_kv_heads),
                               static_cast<cuuint64_t>(num_blocks)};

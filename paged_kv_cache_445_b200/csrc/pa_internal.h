@@ -36,6 +36,7 @@ struct RowsParams {
   long long* table;            // workspace: (tiles << 32 | slot) of the piece that starts at each unit
   long long table_len;         // entries in table
   int* sched;                  // workspace: [warps at the barrier, warps done], zero between calls
+  int* verify_counters;        // workspace: one per SM for the multi-row kernel, zero between calls
   int num_rows;                // query rows (Tq)
   int* status;      // optional device status word
   int total_warps;
@@ -109,6 +110,36 @@ struct CascadeParams {
 };
 
 // Parameters of the tcgen05 chunk kernel (sequences with more than one query row).
+// Sequences with 2 .. 64/G query rows (multi-token verification) on the
+// tcgen05 kernel with the keys in M; the rest of a varlen batch goes to the
+// chunk and rows kernels.  head_dim 128, bf16 caches.
+constexpr int VERIFY_SMEM_SEQS = 1024;  // batches up to this many sequences
+__host__ __device__ constexpr int verify_slot_floats(int ncol) { return (ncol * 128 + 2 * ncol + 63) / 64 * 64; }
+constexpr int VERIFY_MAX_COLS = 64;
+
+struct VerifyParams {
+  void* out;                    // bf16 [Tq, Hq, 128]
+  const int32_t* block_tables;  // [B, max_blocks]
+  const int32_t* context_lens;  // [B]
+  const int32_t* query_start;   // [B + 1]
+  int num_seqs;
+  int max_blocks;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int block_size;
+  int num_blocks;
+  float scale_log2;
+  int* status;
+  float* slots;     // workspace: two (O, m, l) piece slots per CTA
+  int* counters;    // workspace: one per CTA, zero between calls
+  int ncol_lo, ncol_hi;  // set per launch: this kernel takes qlen * G in (ncol_lo, ncol_hi]
+};
+
+int verify_supported(int group, int head_dim, int num_seqs);
+int launch_verify(const VerifyParams& p, const void* q, const void* k_cache, const void* v_cache,
+                  int total_q_tokens, cudaStream_t stream, int num_sms);
+
 struct ChunkParams {
   void* out;                    // bf16 [Tq, Hq, 128]
   const int32_t* block_tables;  // [B, max_blocks]
@@ -123,12 +154,16 @@ struct ChunkParams {
   int num_blocks;
   float scale_log2;
   int* status;
+  int min_qlen;  // sequences with fewer query rows belong to the other kernels
 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encode_fn();
+// [num_blocks, Hkv, block_size, 128] bf16 as a 4-D tensor; box = 64 columns x 16 rows of one (block, head).
+int encode_kv16_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
+                     EncodeTiledFn fn);
 
 struct DeviceInfo {
   int num_sms;

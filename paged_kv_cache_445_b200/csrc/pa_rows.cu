@@ -1075,12 +1075,22 @@ size_t table_entries(int num_rows, int num_kv_heads, long long max_keys) {
 }
 }  // namespace
 
+// Partial-result area: the rows kernel's slots, which the multi-row kernel
+// (head_dim 128) also uses for its pieces (it runs to completion first).
+static size_t partials_bytes(int num_q_heads, int num_kv_heads, int head_dim, int num_sms) {
+  const size_t rows = max_warps(num_sms) * ROWS_SLOTS_PER_WARP * slot_bytes(num_q_heads / num_kv_heads, head_dim);
+  const size_t verify = static_cast<size_t>(num_sms) * 2 * verify_slot_floats(VERIFY_MAX_COLS) * sizeof(float);
+  return head_dim == 128 && verify > rows ? verify : rows;
+}
+
+static size_t verify_counter_bytes(int num_sms) { return round256(static_cast<size_t>(num_sms) * sizeof(int)); }
+
 size_t rows_workspace_bytes(int num_rows, int num_q_heads, int num_kv_heads, int head_dim, long long max_keys,
                             int num_sms) {
-  const size_t w = max_warps(num_sms);
-  return SCHED_BYTES + round256(static_cast<size_t>(num_rows) * num_kv_heads * sizeof(long long)) +
+  return SCHED_BYTES + verify_counter_bytes(num_sms) +
+         round256(static_cast<size_t>(num_rows) * num_kv_heads * sizeof(long long)) +
          round256(table_entries(num_rows, num_kv_heads, max_keys) * sizeof(long long)) +
-         w * ROWS_SLOTS_PER_WARP * slot_bytes(num_q_heads / num_kv_heads, head_dim);
+         partials_bytes(num_q_heads, num_kv_heads, head_dim, num_sms);
 }
 
 void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_heads, int head_dim,
@@ -1088,9 +1098,10 @@ void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_h
   (void)num_q_heads;
   (void)head_dim;
   uint8_t* b = static_cast<uint8_t*>(ws);
-  (void)num_sms;
   p->sched = reinterpret_cast<int*>(b);
   b += SCHED_BYTES;
+  p->verify_counters = reinterpret_cast<int*>(b);
+  b += verify_counter_bytes(num_sms);
   p->seginfo = reinterpret_cast<long long*>(b);
   b += round256(static_cast<size_t>(num_rows) * num_kv_heads * sizeof(long long));
   p->table = reinterpret_cast<long long*>(b);
