@@ -151,15 +151,6 @@ __device__ __forceinline__ bool ch_wait(Shared& sh, uint64_t* bar, uint32_t phas
   }
 }
 
-template <int N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 template <int G>
 __global__ void __launch_bounds__(CH_THREADS, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,

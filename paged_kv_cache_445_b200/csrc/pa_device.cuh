@@ -69,6 +69,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t phase) {
   return done != 0;
 }
 
+// Non-blocking test of the barrier's phase.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t phase) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return done != 0;
+}
+
 // Wait for the barrier's phase; false if it did not complete in time.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t phase) {
   if (mbar_try_wait(bar, phase)) return true;

@@ -1,8 +1,9 @@
 // pa_umma.cuh -- tcgen05 (5th-generation tensor core) helpers shared by the
 // kernels that keep their accumulators in tensor memory: shared-memory matrix
 // descriptors, the kind::f16 instruction descriptor, MMA issue with A from
-// shared or tensor memory, commits to mbarriers, fences, and tensor-memory
-// loads and stores of 32 columns (shape 32x32b: thread = lane = row).
+// shared or tensor memory, commits to mbarriers, fences, tensor-memory loads
+// and stores of 32 columns (shape 32x32b: thread = lane = row), and register
+// reallocation between warpgroups.
 #pragma once
 
 #include <cstdint>
@@ -92,6 +93,17 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
       "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]),
       "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
+}
+
+// Register reallocation between warpgroups (every thread of the warpgroup
+// executes it; the increases must fit in what the launch gave the block).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

@@ -45,7 +45,6 @@ namespace pa {
 
 namespace {
 
-constexpr int VF_THREADS = 256;
 constexpr int VF_D = 128;                  // head_dim
 constexpr int VF_N = 128;                  // keys per tile (the M of S^T)
 constexpr int VF_PANEL = VF_N * 128;       // 128 rows x 128 bytes (64 head-dim columns)
@@ -54,11 +53,13 @@ constexpr float VF_RESCALE_LOG2 = 8.f;
 constexpr uint32_t VF_TMEM_COLS = 512;     // S_0, S_1 at 0 / NCOL; O_0 at 128, O_1 at 256
 constexpr uint32_t VF_TMEM_O = 128;
 constexpr int VF_SOFTMAX_BAR = 1;          // named barrier of the four softmax warps
+constexpr int VF_THREADS = 256;            // warps 0, 2: TMA; 1: MMA; 3: idle; 4-7: softmax and epilogue
 
 template <int NCOL>
 struct VfLayout {
-  static constexpr int KST = NCOL == 32 ? 3 : 2;  // K stages
-  static constexpr int VST = 2;                   // V stages
+  // K is consumed by S one tile ahead of the softmax, V by P V after it: V gets the deeper ring
+  static constexpr int KST = 2;                   // K stages
+  static constexpr int VST = NCOL == 32 ? 3 : 2;  // V stages
   static constexpr int PP = NCOL * 128;           // one P panel: NCOL rows x 64 keys
   static constexpr int PBUF = 2 * PP;
   static constexpr int QP = NCOL * 128;           // one Q panel: NCOL rows x 64 head-dims
@@ -69,8 +70,11 @@ struct VfLayout {
   static constexpr int Q_OFF = P_OFF + 2 * PBUF;
   static constexpr int K_OFF = Q_OFF + 2 * QBUF;
   static constexpr int V_OFF = K_OFF + KST * VF_KV_BYTES;
-  static constexpr int RED_OFF = V_OFF + VST * VF_KV_BYTES;  // float red[2][4][NCOL], lred[4][NCOL], mv[4][NCOL], av[4][NCOL]
-  static constexpr int RED_FLOATS = 2 * 4 * NCOL + 3 * 4 * NCOL;
+  // red[2][4][NCOL] (column maxima of the 4 warps, double-buffered), lred[4][NCOL]
+  // (column sums), mv[4][NCOL] (-m per warp), av[4][NCOL] (rescale factors per
+  // warp), em[2][NCOL], el[2][NCOL] (m and l of the two items whose epilogue may be pending)
+  static constexpr int RED_OFF = V_OFF + VST * VF_KV_BYTES;
+  static constexpr int RED_FLOATS = 2 * 4 * NCOL + 3 * 4 * NCOL + 4 * NCOL;
   static constexpr int PFX_OFF = RED_OFF + RED_FLOATS * 4;   // long long pfx[VERIFY_SMEM_SEQS + 1]
   static constexpr int BYTES = PFX_OFF + (VERIFY_SMEM_SEQS + 1) * 8;
   static_assert(K_OFF % 1024 == 0 && V_OFF % 1024 == 0 && Q_OFF % 1024 == 0, "swizzled tiles need 1024-byte alignment");
@@ -81,7 +85,7 @@ struct VfLayout {
 struct VfShared {
   uint64_t q_full[2], q_empty[2], o_empty[2];
   uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
-  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+  uint64_t k_full[2], k_empty[2], v_full[3], v_empty[3];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -225,10 +229,6 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   long long* pfx = reinterpret_cast<long long*>(smem + L::PFX_OFF);
-  float* red = reinterpret_cast<float*>(smem + L::RED_OFF);  // [2][4][NCOL]
-  float* lred = red + 2 * 4 * NCOL;                          // [4][NCOL]
-  float* mvs = lred + 4 * NCOL;                              // [4][NCOL]
-  float* avs = mvs + 4 * NCOL;                               // [4][NCOL]
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
@@ -297,330 +297,224 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
     }
   }
 
-  if (warp == 0 && ua < ub) {
-    // ================================================================ TMA producer
+  if ((warp == 0 || warp == 2) && ua < ub) {
+    // ================================================================ TMA producers
+    // warp 0 loads Q (per item) and K tiles, warp 2 the V tiles: each ring
+    // refills as soon as its own stage is free
+    const bool is_k = warp == 0;
+    const int nst = is_k ? L::KST : L::VST;
+    uint64_t* full = is_k ? sh.k_full : sh.v_full;
+    uint64_t* empty = is_k ? sh.k_empty : sh.v_empty;
+    const CUtensorMap* tm = is_k ? &tmk : &tmv;
+    uint8_t* ring = smem + (is_k ? L::K_OFF : L::V_OFF);
     if (lane == 0) {
-      prefetch_tmap(&tmq);
-      prefetch_tmap(&tmk);
-      prefetch_tmap(&tmv);
+      if (is_k) prefetch_tmap(&tmq);
+      prefetch_tmap(tm);
     }
     const uint64_t pol = policy_evict_first();  // each K/V tile is read once
-    uint32_t g = 0, i = 0, vg = 0;              // K tiles issued, items, V tiles issued
-    int v_kvh = 0, v_blk = -1, v_y = 0;         // the V tile still to issue (one tile behind K)
-    bool v_pending = false, ok = true;
-    auto issue_v = [&]() -> bool {
-      const int vs = vg % L::VST;
-      if (vg >= L::VST && !vf_wait(sh, &sh.v_empty[vs], ((vg / L::VST) - 1) & 1, p.status)) return false;
-      if (lane == 0) mbar_arrive_expect_tx(&sh.v_full[vs], VF_KV_BYTES);
-      __syncwarp();
+    // lane b < 8: block and row offset of keys 128 j + 16 b .. + 15 of item x
+    auto tile_ids = [&](const VfItem& x, int j, int& blk, int& y) {
+      blk = -1;
+      y = 0;
       if (lane < VF_N / 16) {
-        uint8_t* dst = smem + L::V_OFF + vs * VF_KV_BYTES + lane * 2048;
-        tma_load_4d(dst, &tmv, &sh.v_full[vs], 0, v_y, v_kvh, v_blk, pol);
-        tma_load_4d(dst + VF_PANEL, &tmv, &sh.v_full[vs], 64, v_y, v_kvh, v_blk, pol);
+        const int key0 = j * VF_N + lane * 16;
+        const int lb = key0 / p.block_size;
+        y = key0 - lb * p.block_size;
+        if (lb < (x.ctx + p.block_size - 1) / p.block_size) {
+          blk = __ldg(p.block_tables + static_cast<long long>(x.s) * p.max_blocks + lb);
+          if (is_k && (blk < 0 || blk >= p.num_blocks)) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+        }
       }
-      ++vg;
-      return true;
     };
+    uint32_t g = 0, i = 0;  // tiles issued, items
+    bool ok = true;
     VfItem it;
     vf_seek(p, pfx, ua, ua, ub, it);
     do {
-      const int qb = i & 1;
-      if (i >= 2 && !(ok = vf_wait(sh, &sh.q_empty[qb], ((i >> 1) - 1) & 1, p.status))) break;
-      if (lane == 0) {
-        uint8_t* dq = smem + L::Q_OFF + qb * L::QBUF;
-        mbar_arrive_expect_tx(&sh.q_full[qb], L::QBUF);
-        tma_load_3d(dq, &tmq, &sh.q_full[qb], 0, it.kvh * p.group, it.q0);
-        tma_load_3d(dq + L::QP, &tmq, &sh.q_full[qb], 64, it.kvh * p.group, it.q0);
-      }
-      const int nblk_ctx = (it.ctx + p.block_size - 1) / p.block_size;
-      const int32_t* table = p.block_tables + static_cast<long long>(it.s) * p.max_blocks;
-      for (int j = it.t0; j < it.t1; ++j) {
-        // lane b < 8: block and row offset of keys 128 j + 16 b .. + 15
-        int blk = -1, y = 0;
-        if (lane < VF_N / 16) {
-          const int key0 = j * VF_N + lane * 16;
-          const int lb = key0 / p.block_size;
-          y = key0 - lb * p.block_size;
-          if (lb < nblk_ctx) {
-            blk = __ldg(table + lb);
-            if (blk < 0 || blk >= p.num_blocks) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
-          }
+      if (is_k) {
+        const int qb = i & 1;
+        if (i >= 2 && !(ok = vf_wait(sh, &sh.q_empty[qb], ((i >> 1) - 1) & 1, p.status))) break;
+        if (lane == 0) {
+          uint8_t* dq = smem + L::Q_OFF + qb * L::QBUF;
+          mbar_arrive_expect_tx(&sh.q_full[qb], L::QBUF);
+          tma_load_3d(dq, &tmq, &sh.q_full[qb], 0, it.kvh * p.group, it.q0);
+          tma_load_3d(dq + L::QP, &tmq, &sh.q_full[qb], 64, it.kvh * p.group, it.q0);
         }
-        const int ks = g % L::KST;
-        if (g >= static_cast<uint32_t>(L::KST) &&
-            !(ok = vf_wait(sh, &sh.k_empty[ks], ((g / L::KST) - 1) & 1, p.status)))
-          break;
-        if (lane == 0) mbar_arrive_expect_tx(&sh.k_full[ks], VF_KV_BYTES);
+      }
+      int blk, y;
+      tile_ids(it, it.t0, blk, y);
+      for (int j = it.t0; j < it.t1; ++j) {
+        int nblk = -1, ny = 0;
+        if (j + 1 < it.t1) tile_ids(it, j + 1, nblk, ny);  // the next tile's table entry loads during the wait
+        const int st = g % nst;
+        if (g >= static_cast<uint32_t>(nst) && !(ok = vf_wait(sh, &empty[st], ((g / nst) - 1) & 1, p.status))) break;
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], VF_KV_BYTES);
         __syncwarp();
         if (lane < VF_N / 16) {  // out-of-range block IDs read zeros (and were reported)
-          uint8_t* dst = smem + L::K_OFF + ks * VF_KV_BYTES + lane * 2048;
-          tma_load_4d(dst, &tmk, &sh.k_full[ks], 0, y, it.kvh, blk, pol);
-          tma_load_4d(dst + VF_PANEL, &tmk, &sh.k_full[ks], 64, y, it.kvh, blk, pol);
+          uint8_t* dst = ring + st * VF_KV_BYTES + lane * 2048;
+          tma_load_4d(dst, tm, &full[st], 0, y, it.kvh, blk, pol);
+          tma_load_4d(dst + VF_PANEL, tm, &full[st], 64, y, it.kvh, blk, pol);
         }
         ++g;
-        if (v_pending && !(ok = issue_v())) break;
-        v_pending = true;
-        v_kvh = it.kvh;
-        v_blk = blk;
-        v_y = y;
+        blk = nblk;
+        y = ny;
       }
       if (!ok) break;
       ++i;
     } while (!sh.abort && vf_next(p, pfx, ua, ub, it));
-    if (ok && v_pending) ok = issue_v();
-    if (sh.abort) {  // let this CTA's copies still in flight land before its shared memory goes away
-      for (int st = 0; st < L::KST; ++st) {
-        const uint32_t uses = g / L::KST + (static_cast<uint32_t>(st) < g % L::KST ? 1u : 0u);
-        if (uses > 0) mbar_wait(&sh.k_full[st], (uses - 1) & 1);
+    if (sh.abort) {  // let this warp's copies still in flight land before shared memory goes away
+      for (int st = 0; st < nst; ++st) {
+        const uint32_t uses = g / nst + (static_cast<uint32_t>(st) < g % nst ? 1u : 0u);
+        if (uses > 0) mbar_wait(&full[st], (uses - 1) & 1);
       }
-      for (int st = 0; st < L::VST; ++st) {
-        const uint32_t uses = vg / L::VST + (static_cast<uint32_t>(st) < vg % L::VST ? 1u : 0u);
-        if (uses > 0) mbar_wait(&sh.v_full[st], (uses - 1) & 1);
-      }
-      for (uint32_t b = 0; b < 2; ++b) {
-        const uint32_t uses = i / 2 + (b < i % 2 ? 1u : 0u);
-        if (uses > 0) mbar_wait(&sh.q_full[b], (uses - 1) & 1);
+      if (is_k) {
+        for (uint32_t b = 0; b < 2; ++b) {
+          const uint32_t uses = i / 2 + (b < i % 2 ? 1u : 0u);
+          if (uses > 0) mbar_wait(&sh.q_full[b], (uses - 1) & 1);
+        }
       }
     }
   } else if (warp == 1 && ua < ub) {
     // ================================================================ MMA issuer
+    // Issues S(g) and P V(g) as their inputs become ready (non-blocking
+    // tests), S running ahead of P V: the next tile's S is computed while the
+    // softmax works on the current one.  The warp gives up after WAIT_NS
+    // without progress.
     const uint32_t idesc_s = umma_idesc(VF_N, NCOL, 0, 0);  // S^T = K Q^T: M = keys, N = columns
     const uint32_t idesc_o = umma_idesc(128, VF_D, 0, 1);   // O = P V: M = columns (of 128), N = head_dim
     const uint32_t sbase = smem_u32(smem);
-    uint32_t g = 0, i = 0;
-    // the P V of the previous tile, issued after the next tile's S
-    uint32_t pv_g = 0, pv_i = 0;
-    bool pv_pending = false, pv_first = false, ok = true;
-    auto issue_pv = [&]() -> bool {
-      const int b = pv_g & 1, vs = pv_g % L::VST, ob = pv_i & 1;
-      if (!vf_wait(sh, &sh.p_full[b], (pv_g >> 1) & 1, p.status)) return false;
-      if (!vf_wait(sh, &sh.v_full[vs], (pv_g / L::VST) & 1, p.status)) return false;
-      if (pv_first && pv_i >= 2 && !vf_wait(sh, &sh.o_empty[ob], ((pv_i >> 1) - 1) & 1, p.status)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t sp = sbase + L::P_OFF + b * L::PBUF;
-        const uint32_t sv = sbase + L::V_OFF + vs * VF_KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < VF_N / 16; ++kk)  // keys 16 kk .. + 15: P columns of panel kk / 4, V rows 16 kk ..
-          umma_f16(tmem + VF_TMEM_O + ob * 128, umma_desc(sp + (kk >> 2) * L::PP + (kk & 3) * 32, 16, 1024),
-                   umma_desc(sv + kk * 16 * 128, VF_PANEL, 1024), idesc_o, (!pv_first || kk > 0) ? 1u : 0u);
-        umma_commit(&sh.pv_done[b]);
-        umma_commit(&sh.v_empty[vs]);
-      }
-      __syncwarp();
-      return true;
-    };
+    constexpr int RING = 4;           // tiles whose S is issued and P V is not
+    uint32_t job_item[RING];          // their item (its O slot and the o_empty phase)
+    bool job_first[RING];             // their P V starts the item's O
+    bool o_first = true;
+    uint32_t gs = 0, is = 0, gp = 0;  // next S tile, its item; next P V tile
     VfItem it;
     vf_seek(p, pfx, ua, ua, ub, it);
-    do {
-      const int qb = i & 1;
-      for (int j = it.t0; j < it.t1; ++j) {
-        const int ks = g % L::KST, b = g & 1;
-        if (j == it.t0 && !(ok = vf_wait(sh, &sh.q_full[qb], (i >> 1) & 1, p.status))) break;
-        if (!(ok = vf_wait(sh, &sh.k_full[ks], (g / L::KST) & 1, p.status))) break;
-        if (g >= 2 && !(ok = vf_wait(sh, &sh.s_empty[b], ((g >> 1) - 1) & 1, p.status))) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sk = sbase + L::K_OFF + ks * VF_KV_BYTES;
-          const uint32_t sq = sbase + L::Q_OFF + qb * L::QBUF;
+    int j = it.t0;
+    bool s_more = true;
+    uint64_t t_idle = globaltimer_ns();
+    uint32_t spins = 0;
+    while (true) {
+      bool prog = false;
+      if (s_more && gs - gp < static_cast<uint32_t>(RING)) {
+        const int ks = gs % L::KST, b = gs & 1, qb = is & 1;
+        bool rdy = (j != it.t0 || mbar_test_wait(&sh.q_full[qb], (is >> 1) & 1)) &&
+                   mbar_test_wait(&sh.k_full[ks], (gs / L::KST) & 1) &&
+                   (gs < 2 || mbar_test_wait(&sh.s_empty[b], ((gs >> 1) - 1) & 1));
+        rdy = __shfl_sync(FULL_MASK, rdy, 0);
+        if (rdy) {
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sk = sbase + L::K_OFF + ks * VF_KV_BYTES;
+            const uint32_t sq = sbase + L::Q_OFF + qb * L::QBUF;
 #pragma unroll
-          for (int kk = 0; kk < VF_D / 16; ++kk) {
-            const uint32_t ok_ = (kk >> 2) * VF_PANEL + (kk & 3) * 32, oq = (kk >> 2) * L::QP + (kk & 3) * 32;
-            umma_f16(tmem + b * NCOL, umma_desc(sk + ok_, 16, 1024), umma_desc(sq + oq, 16, 1024), idesc_s,
-                     kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < VF_D / 16; ++kk) {
+              const uint32_t offk = (kk >> 2) * VF_PANEL + (kk & 3) * 32, offq = (kk >> 2) * L::QP + (kk & 3) * 32;
+              umma_f16(tmem + b * NCOL, umma_desc(sk + offk, 16, 1024), umma_desc(sq + offq, 16, 1024), idesc_s,
+                       kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&sh.s_full[b]);
+            umma_commit(&sh.k_empty[ks]);
+            if (j == it.t1 - 1) umma_commit(&sh.q_empty[qb]);
           }
-          umma_commit(&sh.s_full[b]);
-          umma_commit(&sh.k_empty[ks]);
-          if (j == it.t1 - 1) umma_commit(&sh.q_empty[qb]);
+          __syncwarp();
+          job_item[gs % RING] = is;
+          job_first[gs % RING] = o_first;
+          o_first = false;
+          ++gs;
+          prog = true;
+          if (++j == it.t1) {
+            ++is;
+            if (vf_next(p, pfx, ua, ub, it)) {
+              j = it.t0;
+              o_first = true;
+            } else {
+              s_more = false;
+            }
+          }
         }
-        __syncwarp();
-        if (pv_pending && !(ok = issue_pv())) break;
-        pv_pending = true;
-        pv_g = g;
-        pv_i = i;
-        pv_first = j == it.t0;
-        ++g;
       }
-      if (!ok) break;
-      ++i;
-    } while (!sh.abort && vf_next(p, pfx, ua, ub, it));
-    if (ok && pv_pending) issue_pv();
+      if (gp < gs) {
+        const int b = gp & 1, vs = gp % L::VST;
+        const uint32_t ji = job_item[gp % RING];
+        const bool first = job_first[gp % RING];
+        const int os = ji & 1;  // O slot: one per item parity
+        bool rdy = mbar_test_wait(&sh.p_full[b], (gp >> 1) & 1) && mbar_test_wait(&sh.v_full[vs], (gp / L::VST) & 1);
+        // the item two back, which used this O, has had its epilogue
+        if (rdy && first && ji >= 2) rdy = mbar_test_wait(&sh.o_empty[os], ((ji >> 1) - 1) & 1);
+        rdy = __shfl_sync(FULL_MASK, rdy, 0);
+        if (rdy) {
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t sp = sbase + L::P_OFF + b * L::PBUF;
+            const uint32_t sv = sbase + L::V_OFF + vs * VF_KV_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < VF_N / 16; ++kk)  // keys 16 kk .. + 15: P columns of panel kk / 4, V rows 16 kk ..
+              umma_f16(tmem + VF_TMEM_O + os * 128, umma_desc(sp + (kk >> 2) * L::PP + (kk & 3) * 32, 16, 1024),
+                       umma_desc(sv + kk * 16 * 128, VF_PANEL, 1024), idesc_o, (!first || kk > 0) ? 1u : 0u);
+            umma_commit(&sh.pv_done[b]);
+            umma_commit(&sh.v_empty[vs]);
+          }
+          __syncwarp();
+          ++gp;
+          prog = true;
+        }
+      }
+      if (!s_more && gp == gs) break;
+      if (prog) {
+        spins = 0;
+        t_idle = globaltimer_ns();
+      } else if ((++spins & 63) == 0) {
+        if (*reinterpret_cast<volatile int*>(&sh.abort)) break;
+        if (globaltimer_ns() - t_idle > WAIT_NS) {
+          sh.abort = 1;
+          set_status(p.status, PA_STATUS_BIT(PA_ERR_TIMEOUT));
+          break;
+        }
+      }
+    }
   } else if (warp >= 4 && ua < ub) {
     // ================================================================ softmax + epilogue
-    // These four warps meet at named barriers, which cannot time out: none of
+    // The four warps meet at a named barrier, which cannot time out: none of
     // them leaves the item loop early.  A failed wait only records itself (the
     // first one raises the abort flag, after which every wait returns at once)
     // and the loop runs on over the remaining items without merging pieces.
     const int quad = warp & 3;                // TMEM lane quadrant of this warp
     const int t = quad * 32 + lane;           // key of the tile = TMEM lane of S^T; column of O
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + L::RED_OFF);  // [2][4][NCOL]
+    float* lred = red + 2 * 4 * NCOL;                          // [4][NCOL]
+    float* mvs = lred + 4 * NCOL;                              // [4][NCOL]: -m (0 for a column with no key yet)
+    float* avs = mvs + 4 * NCOL;                               // [4][NCOL]
+    float* em = avs + 4 * NCOL;                                // [2][NCOL]
+    float* el = em + 2 * NCOL;                                 // [2][NCOL]
     const float cs = p.scale_log2;
     const int G = p.group;
     uint32_t g = 0, i = 0;
     bool ok = true;
-    VfItem it;
-    vf_seek(p, pfx, ua, ua, ub, it);
-    do {
-      const int ob = i & 1;
-      const int p0 = it.ctx - it.qlen;
-      float mr[NC32];       // running reference maxima of columns lane + 32 k (the same in every warp)
-      float lp[NCOL];       // this key lane's share of each column's sum
-#pragma unroll
-      for (int k = 0; k < NC32; ++k) mr[k] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < NCOL; ++c) lp[c] = 0.f;
-      uint32_t g_last = g;
-      for (int j = it.t0; j < it.t1; ++j) {
-        const int b = g & 1;
-        const uint32_t s_addr = tmem + lane_base + b * NCOL;
-        ok = vf_wait(sh, &sh.s_full[b], (g >> 1) & 1, p.status) && ok;
-        tc_fence_after();
-        // column c is visible to this key iff c >= cthr (rows i >= key - p0; keys past the context: none)
-        const int key = j * VF_N + t, kr = key - p0;
-        const int cthr = kr <= 0 ? 0 : (kr < it.qlen ? kr * G : NCOL);
-        const bool diag = j * VF_N + VF_N - 1 - p0 > 0;
-        auto load_scaled = [&](float (&x)[NCOL]) {
-#pragma unroll
-          for (int k = 0; k < NC32; ++k) {
-            float v[32];
-            tmem_ld32(s_addr + 32 * k, v);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) x[32 * k + c] = v[c];
-          }
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < NCOL; ++c) {
-            const float y = x[c] * cs;
-            x[c] = (diag && c < cthr) ? -INFINITY : y;
-          }
-        };
-        // ---- column maxima: reduce-scatter in the warp, then across the four warps
-        {
-          float x[NCOL];
-          load_scaled(x);
-#pragma unroll
-          for (int k = 0; k < NC32; ++k) {
-            float v[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = x[32 * k + c];
-            red[(b * 4 + quad) * NCOL + 32 * k + lane] = vf_reduce_scatter32<true>(v, lane);
-          }
-        }
-        softmax_bar();
-        bool moved = false;
-#pragma unroll
-        for (int k = 0; k < NC32; ++k) {
-          const int c = 32 * k + lane;
-          const float tm = fmaxf(fmaxf(red[(b * 4 + 0) * NCOL + c], red[(b * 4 + 1) * NCOL + c]),
-                                 fmaxf(red[(b * 4 + 2) * NCOL + c], red[(b * 4 + 3) * NCOL + c]));
-          const float mo = mr[k];
-          const float mn = (tm > mo + VF_RESCALE_LOG2 || mo == -INFINITY) ? fmaxf(tm, mo) : mo;
-          avs[quad * NCOL + c] = (mo == -INFINITY || mn == mo) ? 1.f : fast_exp2(mo - mn);
-          moved |= mn != mo;
-          mr[k] = mn;
-          mvs[quad * NCOL + c] = mn;
-        }
-        const bool resc = __any_sync(FULL_MASK, moved);  // the same in every warp: a CTA-wide decision
-        __syncwarp();
-        // ---- P = exp2(S - m): reload S (the registers went to the reduction)
-        float x[NCOL];
-        load_scaled(x);
-        tc_fence_before();
-        mbar_arrive(&sh.s_empty[b]);  // S_b may now take tile g + 2
-        if (resc) {
-#pragma unroll
-          for (int c = 0; c < NCOL; c += 4) {
-            const float4 a = *reinterpret_cast<const float4*>(avs + quad * NCOL + c);
-            lp[c] *= a.x;
-            lp[c + 1] *= a.y;
-            lp[c + 2] *= a.z;
-            lp[c + 3] *= a.w;
-          }
-          // O holds tiles t0 .. j-1 of this item: wait for P V(g - 1), then scale
-          // row t of O (column t) in tensor memory
-          if (j > it.t0) {
-            ok = vf_wait(sh, &sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, p.status) && ok;
-            tc_fence_after();
-            if (quad < NC32) {
-              const float a = avs[quad * NCOL + t];
-              const uint32_t o_addr = tmem + lane_base + VF_TMEM_O + ob * 128;
-#pragma unroll
-              for (int k = 0; k < VF_D / 32; ++k) {
-                float v[32];
-                tmem_ld32(o_addr + 32 * k, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] *= a;
-                tmem_st32(o_addr + 32 * k, v);
-              }
-              tmem_wait_st();
-            }
-          }
-        }
-        float pr[NCOL];
-#pragma unroll
-        for (int c = 0; c < NCOL; c += 4) {
-          const float4 m4 = *reinterpret_cast<const float4*>(mvs + quad * NCOL + c);
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float neg = mm[e] == -INFINITY ? 0.f : -mm[e];  // a column with no key yet: P = 0
-            pr[c + e] = fast_exp2(x[c + e] + neg);
-            lp[c + e] += pr[c + e];
-          }
-        }
-        // P_b last fed P V(g - 2): wait for it before overwriting
-        if (g >= 2) ok = vf_wait(sh, &sh.pv_done[b], ((g >> 1) - 1) & 1, p.status) && ok;
-        {
-          uint8_t* pb = smem + L::P_OFF + b * L::PBUF + (t >> 6) * L::PP;
-          const int kc = (t & 63) >> 3, ke = (t & 7) * 2;
-#pragma unroll
-          for (int c = 0; c < NCOL; ++c)
-            *reinterpret_cast<__nv_bfloat16*>(pb + c * 128 + ((kc ^ (c & 7)) << 4) + ke) = __float2bfloat16_rn(pr[c]);
-        }
-        // keys past the context may hold anything (even NaN): zero their V rows
-        const int valid = it.ctx - j * VF_N;
-        if (valid < VF_N) {
-          const int vs = g % L::VST;
-          ok = vf_wait(sh, &sh.v_full[vs], (g / L::VST) & 1, p.status) && ok;
-          if (t >= valid) {
-            uint8_t* vrow = smem + L::V_OFF + vs * VF_KV_BYTES + t * 128;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              *reinterpret_cast<uint4*>(vrow + k * 16) = make_uint4(0, 0, 0, 0);
-              *reinterpret_cast<uint4*>(vrow + VF_PANEL + k * 16) = make_uint4(0, 0, 0, 0);
-            }
-          }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&sh.p_full[b]);
-        g_last = g;
-        ++g;
-      }
 
-      // ---- epilogue: column sums, then O / l (or a piece of a cut item)
-#pragma unroll
-      for (int k = 0; k < NC32; ++k) {
-        float v[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) v[c] = lp[32 * k + c];
-        lred[quad * NCOL + 32 * k + lane] = vf_reduce_scatter32<false>(v, lane);
-      }
-      softmax_bar();
-      const bool cut = it.t0 > 0 || it.t1 < it.nt;
-      const int ncolv = it.qlen * G;
-      const int b0 = vf_cta_of(it.base, T, nct), b1 = vf_cta_of(it.base + it.nt - 1, T, nct);
-      ok = vf_wait(sh, &sh.pv_done[g_last & 1], (g_last >> 1) & 1, p.status) && ok;
+    // An item's epilogue runs once its last P V has completed: after the
+    // softmax of the tile two past it has waited for that P V (so the item's
+    // end never stalls the next item's tiles), or earlier with a wait of its
+    // own when the next item ends first, or at the end of the range.
+    VfItem pend;
+    uint32_t pend_g = 0, pend_i = 0;
+    bool pending = false;
+    auto finish = [&](bool wait) {
+      if (wait) ok = vf_wait(sh, &sh.pv_done[pend_g & 1], (pend_g >> 1) & 1, p.status) && ok;
       tc_fence_after();
+      const int ps = pend_i & 1;
+      const bool cut = pend.t0 > 0 || pend.t1 < pend.nt;
+      const int ncolv = pend.qlen * G;
+      const int b0 = vf_cta_of(pend.base, T, nct), b1 = vf_cta_of(pend.base + pend.nt - 1, T, nct);
       if (quad < NC32) {  // thread t owns column t of O
-        const float lsum = (lred[t] + lred[NCOL + t]) + (lred[2 * NCOL + t] + lred[3 * NCOL + t]);
-        const float mcol = (NC32 == 1 || quad == 0) ? mr[0] : mr[NC32 - 1];  // column t = lane + 32 quad
-        const uint32_t o_addr = tmem + lane_base + VF_TMEM_O + ob * 128;
+        const float mcol = em[ps * NCOL + t], lsum = el[ps * NCOL + t];
+        const uint32_t o_addr = tmem + lane_base + VF_TMEM_O + ps * 128;
         if (!cut) {
           const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                                (static_cast<long long>(it.q0 + t / G) * p.num_q_heads + it.kvh * G + t % G) * VF_D;
+          __nv_bfloat16* orow =
+              static_cast<__nv_bfloat16*>(p.out) +
+              (static_cast<long long>(pend.q0 + t / G) * p.num_q_heads + pend.kvh * G + t % G) * VF_D;
 #pragma unroll
           for (int k = 0; k < VF_D / 32; ++k) {
             float v[32];
@@ -640,8 +534,8 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
           }
         } else {
           // this CTA's piece: its first item goes to slot 0, its last to slot 1
-          const int slot = it.base <= ua ? 0 : 1;
-          float* ps = p.slots + (static_cast<long long>(blockIdx.x) * 2 + slot) * verify_slot_floats(NCOL);
+          const int slot = pend.base <= ua ? 0 : 1;
+          float* ps_ = p.slots + (static_cast<long long>(blockIdx.x) * 2 + slot) * verify_slot_floats(NCOL);
 #pragma unroll
           for (int k = 0; k < VF_D / 32; ++k) {
             float v[32];
@@ -649,14 +543,14 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; c += 4)
-              *reinterpret_cast<float4*>(ps + t * VF_D + 32 * k + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+              *reinterpret_cast<float4*>(ps_ + t * VF_D + 32 * k + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
           }
-          ps[NCOL * VF_D + t] = mcol;
-          ps[NCOL * VF_D + NCOL + t] = lsum;
+          ps_[NCOL * VF_D + t] = mcol;
+          ps_[NCOL * VF_D + NCOL + t] = lsum;
         }
       }
       tc_fence_before();
-      mbar_arrive(&sh.o_empty[ob]);
+      mbar_arrive(&sh.o_empty[ps]);
       if (cut) {
         // the CTA that lands the last piece of the item merges all of them, in CTA order
         __threadfence();
@@ -676,31 +570,210 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
             float mx = -INFINITY;
             for (int bb = b0; bb <= b1; ++bb) {
               if (vf_range_start(bb + 1, T, nct) == vf_range_start(bb, T, nct)) continue;  // empty range
-              const int sl = (bb == b0 && it.base != vf_range_start(b0, T, nct)) ? 1 : 0;
-              const float* ps = p.slots + (static_cast<long long>(bb) * 2 + sl) * verify_slot_floats(NCOL);
-              mx = fmaxf(mx, __ldcg(ps + NCOL * VF_D + c));
+              const int sl = (bb == b0 && pend.base != vf_range_start(b0, T, nct)) ? 1 : 0;
+              const float* q = p.slots + (static_cast<long long>(bb) * 2 + sl) * verify_slot_floats(NCOL);
+              mx = fmaxf(mx, __ldcg(q + NCOL * VF_D + c));
             }
-            float acc = 0.f, lsum = 0.f;
+            float acc = 0.f, lt = 0.f;
             for (int bb = b0; bb <= b1; ++bb) {
               if (vf_range_start(bb + 1, T, nct) == vf_range_start(bb, T, nct)) continue;
-              const int sl = (bb == b0 && it.base != vf_range_start(b0, T, nct)) ? 1 : 0;
-              const float* ps = p.slots + (static_cast<long long>(bb) * 2 + sl) * verify_slot_floats(NCOL);
-              const float m = __ldcg(ps + NCOL * VF_D + c);
-              const float w = m == -INFINITY ? 0.f : fast_exp2(m - mx);
-              lsum += __ldcg(ps + NCOL * VF_D + NCOL + c) * w;
-              acc += __ldcg(ps + c * VF_D + t) * w;
+              const int sl = (bb == b0 && pend.base != vf_range_start(b0, T, nct)) ? 1 : 0;
+              const float* q = p.slots + (static_cast<long long>(bb) * 2 + sl) * verify_slot_floats(NCOL);
+              const float m = __ldcg(q + NCOL * VF_D + c);
+              const float wgt = m == -INFINITY ? 0.f : fast_exp2(m - mx);
+              lt += __ldcg(q + NCOL * VF_D + NCOL + c) * wgt;
+              acc += __ldcg(q + c * VF_D + t) * wgt;
             }
-            __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                                  (static_cast<long long>(it.q0 + c / G) * p.num_q_heads + it.kvh * G + c % G) * VF_D;
-            orow[t] = __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
+            __nv_bfloat16* orow =
+                static_cast<__nv_bfloat16*>(p.out) +
+                (static_cast<long long>(pend.q0 + c / G) * p.num_q_heads + pend.kvh * G + c % G) * VF_D;
+            orow[t] = __float2bfloat16_rn(lt > 0.f ? acc / lt : 0.f);
           }
           if (t == 0) p.counters[b1] = 0;  // back to zero for the next call
         }
         softmax_bar();
         if (t == 0) sh.merge = 0;
       }
+      pending = false;
+    };
+
+    VfItem it;
+    vf_seek(p, pfx, ua, ua, ub, it);
+    do {
+      const uint32_t o_addr = tmem + lane_base + VF_TMEM_O + (i & 1) * 128;  // this item's O
+      const int p0 = it.ctx - it.qlen;
+      float mr[NC32];  // running reference maxima of columns lane + 32 k (the same in every warp)
+      float lp[NCOL];  // this key lane's share of each column's sum
+#pragma unroll
+      for (int k = 0; k < NC32; ++k) mr[k] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < NCOL; ++c) lp[c] = 0.f;
+      uint32_t g_last = 0;
+      for (int j = it.t0; j < it.t1; ++j, ++g) {
+        const int b = g & 1;
+        const uint32_t s_addr = tmem + lane_base + b * NCOL;
+        ok = vf_wait(sh, &sh.s_full[b], (g >> 1) & 1, p.status) && ok;
+        tc_fence_after();
+        // column c is visible to this key iff c >= cthr (rows i >= key - p0; keys past the context: none)
+        const int key = j * VF_N + t, kr = key - p0;
+        const int cthr = kr <= 0 ? 0 : (kr < it.qlen ? kr * G : NCOL);
+        const bool diag = j * VF_N + VF_N - 1 - p0 > 0;
+        // ---- column maxima: reduce-scatter in the warp, then across the four warps
+        constexpr bool kReload = NCOL > 32;  // 64 columns: the registers go to the reduction, S is read again
+        float x[NCOL];
+        auto load_scaled = [&]() {
+#pragma unroll
+          for (int k = 0; k < NC32; ++k) {
+            float v[32];
+            tmem_ld32(s_addr + 32 * k, v);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) x[32 * k + c] = v[c] * cs;
+          }
+          tmem_wait_ld();
+          if (diag) {
+#pragma unroll
+            for (int c = 0; c < NCOL; ++c) x[c] = c < cthr ? -INFINITY : x[c];
+          }
+        };
+        if constexpr (kReload) {
+#pragma unroll
+          for (int k = 0; k < NC32; ++k) {
+            float v[32];
+            tmem_ld32(s_addr + 32 * k, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] *= cs;
+            if (diag) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) v[c] = 32 * k + c < cthr ? -INFINITY : v[c];
+            }
+            red[(b * 4 + quad) * NCOL + 32 * k + lane] = vf_reduce_scatter32<true>(v, lane);
+          }
+        } else {
+          load_scaled();
+          tc_fence_before();
+          mbar_arrive(&sh.s_empty[b]);  // S_b may now take tile g + 2
+          float v[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) v[c] = x[c];
+          red[(b * 4 + quad) * NCOL + lane] = vf_reduce_scatter32<true>(v, lane);
+        }
+        softmax_bar();
+        bool moved = false;
+#pragma unroll
+        for (int k = 0; k < NC32; ++k) {
+          const int c = 32 * k + lane;
+          const float tm = fmaxf(fmaxf(red[(b * 4 + 0) * NCOL + c], red[(b * 4 + 1) * NCOL + c]),
+                                 fmaxf(red[(b * 4 + 2) * NCOL + c], red[(b * 4 + 3) * NCOL + c]));
+          const float mo = mr[k];
+          const float mn = (tm > mo + VF_RESCALE_LOG2 || mo == -INFINITY) ? fmaxf(tm, mo) : mo;
+          avs[quad * NCOL + c] = (mo == -INFINITY || mn == mo) ? 1.f : fast_exp2(mo - mn);
+          moved |= mn != mo;
+          mr[k] = mn;
+          mvs[quad * NCOL + c] = mn == -INFINITY ? 0.f : -mn;  // a column with no key yet: P = 0
+        }
+        const bool resc = __any_sync(FULL_MASK, moved);  // the same in every warp
+        __syncwarp();
+        if constexpr (kReload) {
+          load_scaled();
+          tc_fence_before();
+          mbar_arrive(&sh.s_empty[b]);
+        }
+        const bool had = j > it.t0;  // O already holds earlier tiles of this item
+        if (resc) {
+#pragma unroll
+          for (int c = 0; c < NCOL; c += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(avs + quad * NCOL + c);
+            lp[c] *= a.x;
+            lp[c + 1] *= a.y;
+            lp[c + 2] *= a.z;
+            lp[c + 3] *= a.w;
+          }
+        }
+        float pr[NCOL];
+#pragma unroll
+        for (int c = 0; c < NCOL; c += 4) {
+          const float4 nm = *reinterpret_cast<const float4*>(mvs + quad * NCOL + c);
+          pr[c] = fast_exp2(x[c] + nm.x);
+          pr[c + 1] = fast_exp2(x[c + 1] + nm.y);
+          pr[c + 2] = fast_exp2(x[c + 2] + nm.z);
+          pr[c + 3] = fast_exp2(x[c + 3] + nm.w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) lp[c + e] += pr[c + e];
+        }
+        // P_b last fed P V(g - 2): wait for it before overwriting
+        if (g >= 2) ok = vf_wait(sh, &sh.pv_done[b], ((g >> 1) - 1) & 1, p.status) && ok;
+        {
+          uint8_t* pb = smem + L::P_OFF + b * L::PBUF + (t >> 6) * L::PP;
+          const int kc = (t & 63) >> 3, ke = (t & 7) * 2;
+#pragma unroll
+          for (int c = 0; c < NCOL; ++c)
+            *reinterpret_cast<__nv_bfloat16*>(pb + c * 128 + ((kc ^ (c & 7)) << 4) + ke) = __float2bfloat16_rn(pr[c]);
+        }
+        // keys past the context may hold anything (even NaN): zero their V rows
+        const int valid = it.ctx - j * VF_N;
+        if (valid < VF_N) {
+          const int vs = g % L::VST;
+          ok = vf_wait(sh, &sh.v_full[vs], (g / L::VST) & 1, p.status) && ok;
+          if (t >= valid) {  // chunks in a lane-rotated order: the 32 lanes spread over the banks
+            uint8_t* vrow = smem + L::V_OFF + vs * VF_KV_BYTES + t * 128;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int ch = (k + t) & 7;
+              *reinterpret_cast<uint4*>(vrow + ch * 16) = make_uint4(0, 0, 0, 0);
+              *reinterpret_cast<uint4*>(vrow + VF_PANEL + ch * 16) = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+        if (resc && had) {
+          // O holds this item's earlier tiles: wait for the last P V into it
+          // (tile g - 1), then scale row t of O (column t) before P V(g) adds to it
+          ok = vf_wait(sh, &sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, p.status) && ok;
+          tc_fence_after();
+          if (quad < NC32) {
+            const float a = avs[quad * NCOL + t];
+#pragma unroll
+            for (int k = 0; k < VF_D / 32; ++k) {
+              float v[32];
+              tmem_ld32(o_addr + 32 * k, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) v[c] *= a;
+              tmem_st32(o_addr + 32 * k, v);
+            }
+            tmem_wait_st();
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.p_full[b]);
+        g_last = g;
+        // the P-buffer wait above covered P V(g - 2): the epilogue of an item
+        // that ended there can run now without waiting
+        if (pending && g == pend_g + 2) finish(false);
+      }
+
+      // ---- end of the item: column sums now, the rest of the epilogue deferred
+#pragma unroll
+      for (int k = 0; k < NC32; ++k) {
+        float v[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) v[c] = lp[32 * k + c];
+        lred[quad * NCOL + 32 * k + lane] = vf_reduce_scatter32<false>(v, lane);
+      }
+      softmax_bar();
+      if (pending) finish(true);  // the previous item ended one tile ago: its last P V needs a wait
+      if (t < NCOL) {
+        em[(i & 1) * NCOL + t] = (NC32 == 1 || quad == 0) ? mr[0] : mr[NC32 - 1];  // column t = lane + 32 quad
+        el[(i & 1) * NCOL + t] = (lred[t] + lred[NCOL + t]) + (lred[2 * NCOL + t] + lred[3 * NCOL + t]);
+      }
+      pend = it;
+      pend_g = g_last;
+      pend_i = i;
+      pending = true;
       ++i;
     } while (vf_next(p, pfx, ua, ub, it));  // every softmax warp walks every item: the named barriers stay matched
+    if (pending) finish(true);
   }
 
   // ---- teardown: drain this CTA's tensor-core work, then free tensor memory
