@@ -967,6 +967,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
   if (gw >= W && p.k_new)  // warps without tiles still take their share of the fused append
     fused_append<D, F8>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
                     static_cast<long long>(gridDim.x) * ROWS_THREADS);
+  if (T == 0) return;  // no tile anywhere (every CTA sees the same T): nothing to merge, no barrier
 
   // ---- grid barrier: every partial and table entry is stored before any merge reads it
   __syncwarp();

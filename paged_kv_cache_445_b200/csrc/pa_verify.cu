@@ -253,18 +253,10 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
     sh.merge = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh.tmem_base)),
-                 "r"(VF_TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
   // units per sequence, their prefix sums (batch metadata only)
   for (int s = threadIdx.x; s < p.num_seqs; s += VF_THREADS) pfx[s + 1] = vf_units(p, s);
   if (threadIdx.x == 0) pfx[0] = 0;
-  tc_fence_before();
   __syncthreads();
-  tc_fence_after();
   if (warp == 0) {
     long long carry = 0;
     for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
@@ -280,7 +272,6 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
     }
   }
   __syncthreads();
-  const uint32_t tmem = sh.tmem_base;
   const long long T = pfx[p.num_seqs];
   const int nct = gridDim.x;
   const long long ua = vf_range_start(blockIdx.x, T, nct), ub = vf_range_start(blockIdx.x + 1, T, nct);
@@ -296,8 +287,19 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
       for (int k = threadIdx.x; k < n; k += VF_THREADS) o[k] = make_uint4(0, 0, 0, 0);
     }
   }
+  if (ua >= ub) return;  // no unit for this CTA: leave before taking tensor memory
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sh.tmem_base)),
+                 "r"(VF_TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
 
-  if ((warp == 0 || warp == 2) && ua < ub) {
+  if (warp == 0 || warp == 2) {
     // ================================================================ TMA producers
     // warp 0 loads Q (per item) and K tiles, warp 2 the V tiles: each ring
     // refills as soon as its own stage is free
@@ -374,7 +376,7 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         }
       }
     }
-  } else if (warp == 1 && ua < ub) {
+  } else if (warp == 1) {
     // ================================================================ MMA issuer
     // Issues S(g) and P V(g) as their inputs become ready (non-blocking
     // tests), S running ahead of P V: the next tile's S is computed while the
@@ -473,7 +475,7 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         }
       }
     }
-  } else if (warp >= 4 && ua < ub) {
+  } else if (warp >= 4) {
     // ================================================================ softmax + epilogue
     // The four warps meet at a named barrier, which cannot time out: none of
     // them leaves the item loop early.  A failed wait only records itself (the
