@@ -113,7 +113,7 @@ struct CascadeParams {
 // Sequences with 2 .. 64/G query rows (multi-token verification) on the
 // tcgen05 kernel with the keys in M; the rest of a varlen batch goes to the
 // chunk and rows kernels.  head_dim 128, bf16 caches.
-constexpr int VERIFY_SMEM_SEQS = 1024;  // batches up to this many sequences
+constexpr int VERIFY_SMEM_SEQS = 512;   // batches up to this many sequences
 __host__ __device__ constexpr int verify_slot_floats(int ncol) { return (ncol * 128 + 2 * ncol + 63) / 64 * 64; }
 constexpr int VERIFY_MAX_COLS = 64;
 

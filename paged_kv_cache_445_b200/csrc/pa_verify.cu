@@ -57,9 +57,11 @@ constexpr int VF_THREADS = 256;            // warps 0, 2: TMA; 1: MMA; 3: idle; 
 
 template <int NCOL>
 struct VfLayout {
-  // K is consumed by S one tile ahead of the softmax, V by P V after it: V gets the deeper ring
+  // K is consumed by S one tile ahead of the softmax, V by P V after it: V
+  // gets the deeper ring (the bytes in flight set the bandwidth), P a single
+  // buffer (the softmax writes P(g) once P V(g - 1) has read P(g - 1))
   static constexpr int KST = 2;                   // K stages
-  static constexpr int VST = NCOL == 32 ? 3 : 2;  // V stages
+  static constexpr int VST = NCOL == 32 ? 4 : 3;  // V stages
   static constexpr int PP = NCOL * 128;           // one P panel: NCOL rows x 64 keys
   static constexpr int PBUF = 2 * PP;
   static constexpr int QP = NCOL * 128;           // one Q panel: NCOL rows x 64 head-dims
@@ -67,12 +69,12 @@ struct VfLayout {
   // P first: the P . V MMA (M = 128) reads 128 rows from each P panel, the
   // rows past NCOL land on what follows (unused results, in-bounds reads)
   static constexpr int P_OFF = 0;
-  static constexpr int Q_OFF = P_OFF + 2 * PBUF;
+  static constexpr int Q_OFF = P_OFF + PBUF;
   static constexpr int K_OFF = Q_OFF + 2 * QBUF;
   static constexpr int V_OFF = K_OFF + KST * VF_KV_BYTES;
   // red[2][4][NCOL] (column maxima of the 4 warps, double-buffered), lred[4][NCOL]
   // (column sums), mv[4][NCOL] (-m per warp), av[4][NCOL] (rescale factors per
-  // warp), em[2][NCOL], el[2][NCOL] (m and l of the two items whose epilogue may be pending)
+  // warp), em[2][NCOL], el[2][NCOL] (m and l of the items whose epilogue may be pending)
   static constexpr int RED_OFF = V_OFF + VST * VF_KV_BYTES;
   static constexpr int RED_FLOATS = 2 * 4 * NCOL + 3 * 4 * NCOL + 4 * NCOL;
   static constexpr int PFX_OFF = RED_OFF + RED_FLOATS * 4;   // long long pfx[VERIFY_SMEM_SEQS + 1]
@@ -85,7 +87,7 @@ struct VfLayout {
 struct VfShared {
   uint64_t q_full[2], q_empty[2], o_empty[2];
   uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
-  uint64_t k_full[2], k_empty[2], v_full[3], v_empty[3];
+  uint64_t k_full[2], k_empty[2], v_full[4], v_empty[4];
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -448,7 +450,7 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         if (rdy) {
           tc_fence_after();
           if (lane == 0) {
-            const uint32_t sp = sbase + L::P_OFF + b * L::PBUF;
+            const uint32_t sp = sbase + L::P_OFF;
             const uint32_t sv = sbase + L::V_OFF + vs * VF_KV_BYTES;
 #pragma unroll
             for (int kk = 0; kk < VF_N / 16; ++kk)  // keys 16 kk .. + 15: P columns of panel kk / 4, V rows 16 kk ..
@@ -496,9 +498,8 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
     bool ok = true;
 
     // An item's epilogue runs once its last P V has completed: after the
-    // softmax of the tile two past it has waited for that P V (so the item's
-    // end never stalls the next item's tiles), or earlier with a wait of its
-    // own when the next item ends first, or at the end of the range.
+    // softmax of the next tile has waited for that P V (so the item's end
+    // never stalls the next item's tiles), or at the end of the range.
     VfItem pend;
     uint32_t pend_g = 0, pend_i = 0;
     bool pending = false;
@@ -568,28 +569,59 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         softmax_bar();
         if (sh.merge) {
           __threadfence();
-          for (int c = 0; c < ncolv; ++c) {
+          // thread t: column t % NCOL, head-dims [d0, d0 + DPER) of it; every
+          // piece's values load as independent vectors
+          constexpr int DPER = VF_D * NCOL / 128;
+          const int c = t % NCOL, d0 = (t / NCOL) * DPER;
+          const long long r0 = vf_range_start(b0, T, nct);
+          auto piece = [&](int bb) -> const float* {
+            const int sl = (bb == b0 && pend.base != r0) ? 1 : 0;
+            return p.slots + (static_cast<long long>(bb) * 2 + sl) * verify_slot_floats(NCOL);
+          };
+          if (c < ncolv) {
             float mx = -INFINITY;
             for (int bb = b0; bb <= b1; ++bb) {
               if (vf_range_start(bb + 1, T, nct) == vf_range_start(bb, T, nct)) continue;  // empty range
-              const int sl = (bb == b0 && pend.base != vf_range_start(b0, T, nct)) ? 1 : 0;
-              const float* q = p.slots + (static_cast<long long>(bb) * 2 + sl) * verify_slot_floats(NCOL);
-              mx = fmaxf(mx, __ldcg(q + NCOL * VF_D + c));
-            }
-            float acc = 0.f, lt = 0.f;
-            for (int bb = b0; bb <= b1; ++bb) {
-              if (vf_range_start(bb + 1, T, nct) == vf_range_start(bb, T, nct)) continue;
-              const int sl = (bb == b0 && pend.base != vf_range_start(b0, T, nct)) ? 1 : 0;
-              const float* q = p.slots + (static_cast<long long>(bb) * 2 + sl) * verify_slot_floats(NCOL);
-              const float m = __ldcg(q + NCOL * VF_D + c);
-              const float wgt = m == -INFINITY ? 0.f : fast_exp2(m - mx);
-              lt += __ldcg(q + NCOL * VF_D + NCOL + c) * wgt;
-              acc += __ldcg(q + c * VF_D + t) * wgt;
+              mx = fmaxf(mx, __ldcg(piece(bb) + NCOL * VF_D + c));
             }
             __nv_bfloat16* orow =
                 static_cast<__nv_bfloat16*>(p.out) +
-                (static_cast<long long>(pend.q0 + c / G) * p.num_q_heads + pend.kvh * G + c % G) * VF_D;
-            orow[t] = __float2bfloat16_rn(lt > 0.f ? acc / lt : 0.f);
+                (static_cast<long long>(pend.q0 + c / G) * p.num_q_heads + pend.kvh * G + c % G) * VF_D + d0;
+#pragma unroll 1
+            for (int dc = 0; dc < DPER; dc += 32) {
+              float acc[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+              float lt = 0.f;
+              for (int bb = b0; bb <= b1; ++bb) {
+                if (vf_range_start(bb + 1, T, nct) == vf_range_start(bb, T, nct)) continue;
+                const float* q = piece(bb);
+                const float m = __ldcg(q + NCOL * VF_D + c);
+                const float wgt = m == -INFINITY ? 0.f : fast_exp2(m - mx);
+                lt += __ldcg(q + NCOL * VF_D + NCOL + c) * wgt;
+                const float4* o4 = reinterpret_cast<const float4*>(q + c * VF_D + d0 + dc);
+                float4 v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = __ldcg(o4 + e);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  acc[4 * e] += v[e].x * wgt;
+                  acc[4 * e + 1] += v[e].y * wgt;
+                  acc[4 * e + 2] += v[e].z * wgt;
+                  acc[4 * e + 3] += v[e].w * wgt;
+                }
+              }
+              const float inv = lt > 0.f ? 1.f / lt : 0.f;
+#pragma unroll
+              for (int e = 0; e < 32; e += 8) {
+                uint4 u;
+                u.x = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+                u.y = pack_bf16x2(acc[e + 2] * inv, acc[e + 3] * inv);
+                u.z = pack_bf16x2(acc[e + 4] * inv, acc[e + 5] * inv);
+                u.w = pack_bf16x2(acc[e + 6] * inv, acc[e + 7] * inv);
+                *reinterpret_cast<uint4*>(orow + dc + e) = u;
+              }
+            }
           }
           if (t == 0) p.counters[b1] = 0;  // back to zero for the next call
         }
@@ -692,25 +724,30 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
             lp[c + 3] *= a.w;
           }
         }
-        float pr[NCOL];
-#pragma unroll
-        for (int c = 0; c < NCOL; c += 4) {
-          const float4 nm = *reinterpret_cast<const float4*>(mvs + quad * NCOL + c);
-          pr[c] = fast_exp2(x[c] + nm.x);
-          pr[c + 1] = fast_exp2(x[c + 1] + nm.y);
-          pr[c + 2] = fast_exp2(x[c + 2] + nm.z);
-          pr[c + 3] = fast_exp2(x[c + 3] + nm.w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) lp[c + e] += pr[c + e];
-        }
-        // P_b last fed P V(g - 2): wait for it before overwriting
-        if (g >= 2) ok = vf_wait(sh, &sh.pv_done[b], ((g >> 1) - 1) & 1, p.status) && ok;
+        // P = exp2(S - m) by 32 columns; P last fed P V(g - 1): wait for it
+        // (after the first 32 exponentials) before overwriting
         {
-          uint8_t* pb = smem + L::P_OFF + b * L::PBUF + (t >> 6) * L::PP;
+          uint8_t* pb = smem + L::P_OFF + (t >> 6) * L::PP;
           const int kc = (t & 63) >> 3, ke = (t & 7) * 2;
 #pragma unroll
-          for (int c = 0; c < NCOL; ++c)
-            *reinterpret_cast<__nv_bfloat16*>(pb + c * 128 + ((kc ^ (c & 7)) << 4) + ke) = __float2bfloat16_rn(pr[c]);
+          for (int k = 0; k < NC32; ++k) {
+            float pr[32];
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+              const float4 nm = *reinterpret_cast<const float4*>(mvs + quad * NCOL + 32 * k + c);
+              pr[c] = fast_exp2(x[32 * k + c] + nm.x);
+              pr[c + 1] = fast_exp2(x[32 * k + c + 1] + nm.y);
+              pr[c + 2] = fast_exp2(x[32 * k + c + 2] + nm.z);
+              pr[c + 3] = fast_exp2(x[32 * k + c + 3] + nm.w);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) lp[32 * k + c + e] += pr[c + e];
+            }
+            if (k == 0 && g >= 1) ok = vf_wait(sh, &sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1, p.status) && ok;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              *reinterpret_cast<__nv_bfloat16*>(pb + (32 * k + c) * 128 + ((kc ^ (c & 7)) << 4) + ke) =
+                  __float2bfloat16_rn(pr[c]);
+          }
         }
         // keys past the context may hold anything (even NaN): zero their V rows
         const int valid = it.ctx - j * VF_N;
@@ -750,9 +787,9 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         tc_fence_before();
         mbar_arrive(&sh.p_full[b]);
         g_last = g;
-        // the P-buffer wait above covered P V(g - 2): the epilogue of an item
-        // that ended there can run now without waiting
-        if (pending && g == pend_g + 2) finish(false);
+        // the P wait above covered P V(g - 1): the epilogue of an item that
+        // ended there can run now without waiting
+        if (pending && g == pend_g + 1) finish(false);
       }
 
       // ---- end of the item: column sums now, the rest of the epilogue deferred
@@ -764,7 +801,6 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         lred[quad * NCOL + 32 * k + lane] = vf_reduce_scatter32<false>(v, lane);
       }
       softmax_bar();
-      if (pending) finish(true);  // the previous item ended one tile ago: its last P V needs a wait
       if (t < NCOL) {
         em[(i & 1) * NCOL + t] = (NC32 == 1 || quad == 0) ? mr[0] : mr[NC32 - 1];  // column t = lane + 32 quad
         el[(i & 1) * NCOL + t] = (lred[t] + lred[NCOL + t]) + (lred[2 * NCOL + t] + lred[3 * NCOL + t]);
