@@ -63,6 +63,7 @@ def measured_peaks():
 KERNEL_SOURCES = {  # the files whose text decides each kernel's code
     "pa_rows_kernel": ("pa_rows.cu", "pa_device.cuh"),
     "pa_chunk_kernel": ("pa_chunk.cu", "pa_device.cuh", "pa_umma.cuh"),
+    "pa_verify_kernel": ("pa_verify.cu", "pa_device.cuh", "pa_umma.cuh"),
 }
 
 
@@ -206,14 +207,25 @@ def rank_seed(workload: int, rank: int) -> int:
     return 445 + workload + 1000 * rank
 
 
-def step_launches(w, chunk_head_dims=(128,), chunk_groups=(1, 2, 4, 8, 16)) -> int:
-    """Kernel launches of one step: the append, the rows kernel, and the
-    tcgen05 chunk kernel when the batch has a multi-row sequence it takes."""
-    qs = np.asarray(w.query_start)
-    multi = bool(np.any(np.diff(qs) > 1))
-    chunk = (not w.is_decode and multi and w.head_dim in chunk_head_dims
-             and (w.num_q_heads // w.num_kv_heads) in chunk_groups)
-    return 2 + int(chunk)
+def step_launches(w, chunk_head_dims=(128,), chunk_groups=(1, 2, 4, 8, 16), verify_max_seqs=512) -> int:
+    """Kernel launches of one unfused step: the append and the rows kernel;
+    for a varlen batch at head_dim 128 with a supported group also the tcgen05
+    chunk kernel and the two multi-row kernels (32 and 64 columns), which
+    pa_prefill_chunk launches whatever the batch holds (each returns at once
+    when it has no work)."""
+    n = 2
+    if not w.is_decode and w.head_dim in chunk_head_dims and (w.num_q_heads // w.num_kv_heads) in chunk_groups:
+        n += 1 + (2 if w.num_seqs <= verify_max_seqs else 0)
+    return n
+
+
+def verify_batch(w, max_cols=64, max_seqs=512) -> bool:
+    """Every sequence of the batch has 2 .. max_cols/G query rows: the
+    multi-row (verification) kernel does all the attention work."""
+    g = w.num_q_heads // w.num_kv_heads
+    qlen = np.diff(np.asarray(w.query_start))
+    return (not w.is_decode and w.head_dim == 128 and w.num_seqs <= max_seqs and bool(np.all(qlen >= 2))
+            and bool(np.all(qlen * g <= max_cols)))
 
 
 def compose_value(total_kv_bytes: float, ms_step_max: float) -> float:
@@ -430,7 +442,9 @@ def run_ours(args, peaks):
     # the timed launch (or replay) also appends when fused or replayed as a graph
     launch_bytes = attn_bytes + (app_bytes if (g.fused or graph is not None) else 0)
     achieved = launch_bytes / (attn_avg_ms * 1e-3) / 1e9
-    traffic = profiled_traffic("pa_rows_kernel", w.name, "-fp8" if g.fp8 else "")
+    verify = verify_batch(w)
+    traffic = (profiled_traffic("pa_verify_kernel", w.name) if verify else
+               profiled_traffic("pa_rows_kernel", w.name, "-fp8" if g.fp8 else ""))
     line = {
         "metric": "paged-attn decode KV GB/s + seq-steps/s (70B layer, bs128); % of HBM peak",
         "value": round(compose_value(total_kv, ms_step), 2),
@@ -457,6 +471,9 @@ def run_ours(args, peaks):
         "frac_of_8tbs_nominal": round(compose_value(total_kv, ms_step) / 8000.0 / world, 4),
         "roofline": {
             "kernel": ("pa_rows_kernel, FP8 E4M3 cache (append + attention, one launch)" if g.fp8 else
+                       "pa_verify_kernel (timed as the whole pa_prefill_chunk call: its launches of the "
+                       "chunk and rows kernels find no work)" if verify else
+                       "pa_prefill_chunk call (chunk kernel + rows kernel)" if not w.is_decode else
                        "pa_cascade_kernel + pa_rows_kernel (shared prefixes once, then the private keys)"
                        if g.cascade else
                        "pa_rows_kernel (append + attention, one launch)" if g.fused else "pa_rows_kernel (attention)"),

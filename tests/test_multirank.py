@@ -96,5 +96,9 @@ def test_launch_count_per_step():
     mixed = workloads.custom([200, 30], [48, 1], 16, 2, 128, 16, seed=1)
     mixed_d64 = workloads.custom([200, 30], [48, 1], 16, 2, 64, 16, seed=1)
     assert bench.step_launches(decode) == 2
-    assert bench.step_launches(mixed) == 3
+    # append, chunk kernel, the two multi-row kernels, rows kernel (pa_prefill_chunk launches
+    # every kernel that may have work at head_dim 128, whatever the row counts are)
+    assert bench.step_launches(mixed) == 5
     assert bench.step_launches(mixed_d64) == 2
+    verify = workloads.custom([200, 30, 90], [4, 2, 8], 16, 2, 128, 16, seed=1)
+    assert bench.verify_batch(verify) and not bench.verify_batch(mixed) and not bench.verify_batch(decode)
