@@ -237,10 +237,15 @@ PA_API int pa_decode_cascade(void* out, const void* q, const void* k_new, const 
  * of a query block that ends at the last key is the one of "Inference
  * optimization", "Build it -- Step 2" (row i sees keys j <= i + Lk - Lq).
  *
- * q / out have total_q_tokens = query_start[num_seqs] rows.  Rows of
- * sequences with qlen > 1 run on the tcgen05 tensor-core path; rows with
- * qlen = 1 run on the decode path, concurrently.  A row with no key (p < 0)
- * produces zeros.
+ * q / out have total_q_tokens = query_start[num_seqs] rows.  At head_dim 128
+ * (query heads per KV head G in {1, 2, 4, 8, 16}) the call runs, one after
+ * another on `stream`: a tcgen05 kernel for sequences with 2 .. 64/G rows
+ * (speculative verification: the "Speculative decoding" section of
+ * "Inference optimization"; batches of at most 512 sequences), the tcgen05
+ * chunk kernel for longer chunks, and the decode path for qlen = 1.  Other
+ * head dims run every row on the decode path.  A row with no key (p < 0)
+ * produces zeros.  Workspace: pa_workspace_bytes(total_q_tokens, ...), under
+ * its contract (zero-filled once; the call leaves its counters at zero).
  */
 PA_API int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const void* k_cache,
                      const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
