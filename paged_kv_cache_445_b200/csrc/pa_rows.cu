@@ -318,34 +318,53 @@ __device__ __forceinline__ void seek(const RowsParams& p, const long long* pfx, 
 }
 
 // Fold the shared-prefix partials of (sequence seq, KV head kvh) into the state
-// of its segment: per query head, O <- O e^(m - m') + O_k e^(m_k - m'),
-// l likewise, m' = max(m, m_k), over the prefix slices k.
+// of its segment: per query head, with m' = max(m, max over the slices k of m_k),
+// O <- O e^(m - m') + sum_k O_k e^(m_k - m'), l likewise.  `slices` is a bit
+// mask over the records 0 .. CASCADE_SPLITS; all its records load at once
+// (maxima and sums first, then the O rows), not one slice after another.
 template <int D, int NT>
-__device__ __forceinline__ void fold_prefix(const RowsParams& p, int k_begin, int k_end, float (&o)[D / 16][NT][4],
+__device__ __forceinline__ void fold_prefix(const RowsParams& p, unsigned slices, float (&o)[D / 16][NT][4],
                                             float (&m)[NT][2], float (&l)[NT][2], int seq, int kvh, int lane) {
+  constexpr int NREC = CASCADE_SPLITS + 1;
+  constexpr int REC = cascade_record_floats(D);
   const int g = lane >> 2, c = lane & 3;
-  for (int k = k_begin; k < k_end; ++k) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int head = nt * 8 + 2 * c + e;
-        if (head >= p.group) continue;
-        const float* src = p.casc_partials +
-                           ((static_cast<long long>(seq) * p.num_q_heads + kvh * p.group + head) * (CASCADE_SPLITS + 1) +
-                            k) * cascade_record_floats(D);
-        const float mk = __ldcg(src + D), lk = __ldcg(src + D + 1);
-        const float mn = fmaxf(m[nt][e], mk);
-        const float f = fast_exp2(m[nt][e] - mn), w = fast_exp2(mk - mn);
-        m[nt][e] = mn;
-        l[nt][e] = l[nt][e] * f + w * lk;
+    for (int e = 0; e < 2; ++e) {
+      const int head = nt * 8 + 2 * c + e;
+      if (head >= p.group) continue;
+      const float* base = p.casc_partials +
+                          (static_cast<long long>(seq) * p.num_q_heads + kvh * p.group + head) * NREC * REC;
+      float mk[NREC], w[NREC];
+      float mn = m[nt][e];
 #pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {  // accumulator rows: head dim 16 mt + g and 16 mt + g + 8
-          o[mt][nt][e] = o[mt][nt][e] * f + w * __ldcg(src + 16 * mt + g);
-          o[mt][nt][2 + e] = o[mt][nt][2 + e] * f + w * __ldcg(src + 16 * mt + g + 8);
-        }
+      for (int k = 0; k < NREC; ++k) {
+        mk[k] = (slices >> k) & 1 ? __ldcg(base + k * REC + D) : -INFINITY;
+        mn = fmaxf(mn, mk[k]);
       }
-  }
+      const float f = fast_exp2(m[nt][e] - mn);
+      float lt = l[nt][e] * f;
+#pragma unroll
+      for (int k = 0; k < NREC; ++k) {
+        w[k] = (slices >> k) & 1 ? fast_exp2(mk[k] - mn) : 0.f;
+        if ((slices >> k) & 1) lt += w[k] * __ldcg(base + k * REC + D + 1);
+      }
+      m[nt][e] = mn;
+      l[nt][e] = lt;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {  // accumulator rows: head dim 16 mt + g and 16 mt + g + 8
+        float a = o[mt][nt][e] * f, b = o[mt][nt][2 + e] * f;
+#pragma unroll
+        for (int k = 0; k < NREC; ++k)
+          if ((slices >> k) & 1) {
+            a += w[k] * __ldcg(base + k * REC + 16 * mt + g);
+            b += w[k] * __ldcg(base + k * REC + 16 * mt + g + 8);
+          }
+        o[mt][nt][e] = a;
+        o[mt][nt][2 + e] = b;
+      }
+    }
 }
 
 // Store the unnormalised state of a whole private segment in the shared-prefix
@@ -427,9 +446,9 @@ __device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, 
   if (p.num_groups > 0) {
     const int span = seq_info(p, row).k0;  // decode: row = sequence; 0 if its keys were not split
     if (span > 0) {
-      // n == 0: the private part was one piece, kept in the last slot; then the prefix slices
-      if (n == 0) fold_prefix<D, NT>(p, CASCADE_SPLITS, CASCADE_SPLITS + 1, acc, mm, ll, row, kvh, lane);
-      fold_prefix<D, NT>(p, 0, cascade_splits(span), acc, mm, ll, row, kvh, lane);
+      // the prefix slices, and with n == 0 the private part too (one piece, kept in the last slot)
+      const unsigned slices = ((1u << cascade_splits(span)) - 1u) | (n == 0 ? 1u << CASCADE_SPLITS : 0u);
+      fold_prefix<D, NT>(p, slices, acc, mm, ll, row, kvh, lane);
     }
   }
   store_output<D, NT, F8>(p, acc, ll, row, kvh, lane);
