@@ -108,3 +108,14 @@ def test_sequences_without_rows_between_multi_row_ones():
     kc, vc = oracle_after_append(w)
     compare(got, _ref(w, kc, vc), "rowless sequences")
     assert int(ds.status.item()) == 0
+
+
+def test_groups_the_tensor_core_paths_do_not_take_run_on_the_decode_kernel():
+    # G = 6 at head_dim 128: multi-row sequences run row by row on the decode kernel
+    w = workloads.custom([300, 41, 1000], [4, 2, 7], 24, 4, 128, 16, seed=17, poison=True)
+    ds = DeviceStep(w)
+    got = ds.step()
+    kc, vc = oracle_after_append(w)
+    compare(got, _ref(w, kc, vc), "G 6")
+    assert int(ds.status.item()) == 0
+
