@@ -601,10 +601,11 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
     BtWindow win;
     win.s = -1;
 
+    const int bs_shift = p.block_size == 32 ? 5 : 4;
     auto issue = [&](int stage) {
       const bool first = lc.u == a, last = lc.u == e - 1;
       const int key0 = lc.k0 + lc.t * TILE_KEYS;
-      const int lb = key0 / p.block_size, y = key0 - lb * p.block_size;
+      const int lb = key0 >> bs_shift, y = key0 & (p.block_size - 1);  // block_size is 16 or 32
       const int blk = bt_lookup(p, win, lc.s, lb, lane);
       if (lc.t == 0 || first) {
         // warm L1 with query rows a segment ahead: the next segment's (row + 1
@@ -659,9 +660,15 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
     bool began = false;
     int piece_t0 = 0;
 
+    int next_stage = 0;
+    uint32_t next_phase = 0;
     for (long long j = 0; j < issued; ++j) {
-      const int stage = static_cast<int>(j % R);
-      const uint32_t phase = static_cast<uint32_t>((j / R) & 1);
+      const int stage = next_stage;  // j % R and (j / R) & 1, kept incrementally
+      const uint32_t phase = next_phase;
+      if (++next_stage == R) {
+        next_stage = 0;
+        next_phase ^= 1;
+      }
       if (!mbar_wait(&bar[stage], phase)) {
         set_status(p.status, PA_STATUS_BIT(PA_ERR_TIMEOUT));
         stopped_at = j;
