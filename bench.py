@@ -67,12 +67,23 @@ KERNEL_SOURCES = {  # the files whose text decides each kernel's code
 }
 
 
+def code_tokens(text: str) -> str:
+    """C/CUDA source without comments and with whitespace runs collapsed: an
+    edit of comments or layout leaves it (and the compiled kernel) unchanged.
+    The sources hold no string literal with a comment marker in it."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(kernel: str) -> str:
+    """Hash of the code (comments and whitespace aside) of the files that
+    decide a kernel's binary."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_445_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update((name + "\n" + code_tokens(f.read())).encode())
     return h.hexdigest()[:16]
 
 

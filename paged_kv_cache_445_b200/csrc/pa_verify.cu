@@ -1,4 +1,4 @@
-// pa_verify.cu -- attention of short multi-row queries (2 .. 8 rows per
+// pa_verify.cu -- attention of short multi-row queries (2 .. 64/G rows per
 // sequence, as when a target model checks draft tokens) over the paged KV
 // cache, on the 5th-generation tensor cores with the keys in M.
 //
@@ -26,10 +26,15 @@
 //    item cut by range ends leaves (m, l, O) pieces in per-CTA slots; the CTA
 //    that finishes the last piece of an item (a counter per cut item) merges
 //    the pieces in CTA order and writes the rows.
-//  * Roles (8 warps): warp 0 issues TMA, warp 1 owns tensor memory and issues
-//    tcgen05.mma from one thread, warps 4-7 run the softmax and the epilogue
-//    (thread = TMEM lane).  S and P are double-buffered per tile, Q and O per
-//    item, so an item's first tiles overlap the previous item's epilogue.
+//  * Roles (8 warps): warp 0 loads Q and the K tiles, warp 2 the V tiles (each
+//    refills its own ring as soon as a stage is free; V, read after the
+//    softmax, gets the deeper ring); warp 1 owns tensor memory and issues
+//    tcgen05.mma from one thread as soon as the inputs of an S or a P V are
+//    ready; warps 4-7 run the softmax and the epilogue (thread = TMEM lane).
+//    S is double-buffered per tile, P single (written once P V(g - 1) has read
+//    it), Q and O per item.  An item's epilogue runs one tile into the next
+//    item, when its last P V is known to be complete, so item ends do not
+//    stall the pipeline.
 //  * O is rescaled only when a column's running maximum rises by more than
 //    2^8 (between rescales the stale maximum is an exact reference point).
 //  * Every wait is bounded: on a timeout the CTA records PA_ERR_TIMEOUT,
