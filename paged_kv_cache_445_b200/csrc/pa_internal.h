@@ -40,6 +40,7 @@ struct RowsParams {
   int num_rows;                // query rows (Tq)
   int* status;      // optional device status word
   int total_warps;
+  int tile_shift;   // log2 of the keys per work unit (16, or 32 for the E4M3 kernel with one head tile)
   // Fused cache append (decode only; nullptr: none).  Row s of k_new / v_new
   // ([B, Hkv, D] bf16) is sequence s's newest token: the kernel writes it to
   // position context_lens[s] - 1 through the block table and attends to it

@@ -38,7 +38,7 @@
 
 namespace pa {
 
-constexpr int TILE_KEYS = 16;
+constexpr int TILE_KEYS = 16;  // keys per work unit, and per TMA box; a variant may take two boxes per unit
 constexpr int ROWS_WARPS = 4;
 constexpr int ROWS_THREADS = ROWS_WARPS * 32;
 constexpr int ROWS_SLOTS_PER_WARP = 2;  // a warp's range cuts at most its first and its last segment
@@ -49,13 +49,17 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
-__device__ __forceinline__ int ceil16(int n) { return (n + TILE_KEYS - 1) / TILE_KEYS; }
+// Work units (tiles of 2^tile_shift keys) of a segment with n keys.
+__device__ __forceinline__ int ceil_tiles(const RowsParams& p, int n) {
+  return (n + (1 << p.tile_shift) - 1) >> p.tile_shift;
+}
 
-// sum_{k=1}^{n} ceil(k / 16): tiles of the rows whose key counts are 1..n.
-__device__ __forceinline__ long long tiles_upto(int n) {
+// sum_{k=1}^{n} ceil(k / TK), TK = 2^tile_shift: tiles of the rows whose key counts are 1..n.
+__device__ __forceinline__ long long tiles_upto(const RowsParams& p, int n) {
   if (n <= 0) return 0;
-  const long long q = n >> 4, r = n & 15;
-  return 8 * q * (q + 1) + r * (q + 1);
+  const int sh = p.tile_shift;
+  const long long tk = 1ll << sh, q = n >> sh, r = n & (tk - 1);
+  return tk * q * (q + 1) / 2 + r * (q + 1);
 }
 
 __device__ __forceinline__ long long warp_sum64(long long v) {
@@ -127,7 +131,7 @@ __device__ __forceinline__ SeqInfo seq_info(const RowsParams& p, int s) {
 __device__ __forceinline__ long long seq_units(const RowsParams& p, const SeqInfo& si) {
   if (p.skip_multi && si.qlen > 1) return 0;
   const int p0 = si.ctx - si.qlen;
-  return static_cast<long long>(p.num_kv_heads) * (tiles_upto(si.ctx) - tiles_upto(p0 < 0 ? 0 : p0));
+  return static_cast<long long>(p.num_kv_heads) * (tiles_upto(p, si.ctx) - tiles_upto(p, p0 < 0 ? 0 : p0));
 }
 
 struct Cursor {
@@ -150,7 +154,7 @@ __device__ __forceinline__ bool enter_seq(const RowsParams& p, Cursor& c, int s)
   c.h = 0;
   c.t = 0;
   c.nkeys = c.p0 + c.i + 1;
-  c.n = ceil16(c.nkeys);
+  c.n = ceil_tiles(p, c.nkeys);
   return true;
 }
 
@@ -162,7 +166,7 @@ __device__ __forceinline__ void advance(const RowsParams& p, Cursor& c) {
   c.h = 0;
   if (++c.i < c.qlen) {
     ++c.nkeys;
-    c.n = ceil16(c.nkeys);
+    c.n = ceil_tiles(p, c.nkeys);
     return;
   }
   for (int s = c.s + 1; s < p.num_seqs; ++s)
@@ -194,10 +198,11 @@ __device__ __forceinline__ int bt_lookup(const RowsParams& p, BtWindow& w, int s
 
 __device__ __forceinline__ long long range_start(long long w, long long T, long long W) { return T * w / W; }
 
-template <int D, int NT, bool F8 = false>
+template <int D, int NT, bool F8 = false, int TK = TILE_KEYS>
 struct RowsShape {
   static constexpr int KT = D / 16;                    // k-steps of QK^T, m-tiles of PV
-  static constexpr int HALF_BYTES = TILE_KEYS * D * (F8 ? 1 : 2);  // K (or V) bytes of a tile
+  static constexpr int BOX_BYTES = TILE_KEYS * D * (F8 ? 1 : 2);  // one TMA box: 16 rows of one (block, head)
+  static constexpr int HALF_BYTES = TK * D * (F8 ? 1 : 2);        // K (or V) bytes of a tile
   static constexpr int STAGE_BYTES = 2 * HALF_BYTES;
   static constexpr int SLOT_O = KT * NT * 32 * 4;      // O^T fragment floats of a partial
   static constexpr int SLOT_M = SLOT_O;                // running maxima (8 NT floats)
@@ -299,19 +304,19 @@ __device__ __forceinline__ void seek(const RowsParams& p, const long long* pfx, 
   cc.p0 = si.ctx - si.qlen;
   const int i0 = cc.p0 < 0 ? -cc.p0 : 0;
   const long long o = a - seq_base;
-  const long long base_tiles = tiles_upto(cc.p0 + i0);
+  const long long base_tiles = tiles_upto(p, cc.p0 + i0);
   int lo = i0, hi = si.qlen - 1;
   while (lo < hi) {  // last row whose first unit is <= o
     const int mid = (lo + hi + 1) >> 1;
-    if (static_cast<long long>(p.num_kv_heads) * (tiles_upto(cc.p0 + mid) - base_tiles) <= o)
+    if (static_cast<long long>(p.num_kv_heads) * (tiles_upto(p, cc.p0 + mid) - base_tiles) <= o)
       lo = mid;
     else
       hi = mid - 1;
   }
   cc.i = lo;
   cc.nkeys = cc.p0 + lo + 1;
-  cc.n = ceil16(cc.nkeys);
-  const long long rem = o - static_cast<long long>(p.num_kv_heads) * (tiles_upto(cc.p0 + lo) - base_tiles);
+  cc.n = ceil_tiles(p, cc.nkeys);
+  const long long rem = o - static_cast<long long>(p.num_kv_heads) * (tiles_upto(p, cc.p0 + lo) - base_tiles);
   cc.h = static_cast<int>(rem / cc.n);
   cc.t = static_cast<int>(rem % cc.n);
   cc.u = a;
@@ -511,18 +516,24 @@ struct TileMeta {
 };
 
 // CTAs per SM a variant is compiled for: the E4M3 kernel with one head tile
-// is bound by instruction latency (the code conversions), so it runs three
-// CTAs per SM (12 warps) in at most 168 registers; the others run two.
-template <int D, int NT, bool F8>
+// and 16-key tiles is bound by instruction latency (the code conversions), so
+// it runs three CTAs per SM (12 warps) in at most 168 registers; the others
+// run two.
+template <int D, int NT, bool F8, int TK>
 constexpr int rows_ctas_per_sm() {
-  return (F8 && D == 128 && NT == 1) ? 3 : 2;
+  return (F8 && D == 128 && NT == 1 && TK == 16) ? 3 : 2;
 }
 
-template <int D, int NT, int R, bool F8>
-__global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() == 3 ? 3 : 1)
+// TK: keys per work unit and ring stage, 16 or 32.  With 32 (the E4M3 kernel
+// at head_dim 128 with one head tile) a stage holds two 16-row TMA boxes per
+// K and V and the warp takes two 16-key m-tiles per softmax step, so the
+// per-tile bookkeeping covers twice the bytes.
+template <int D, int NT, int R, bool F8, int TK>
+__global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8, TK>() == 3 ? 3 : 1)
     rows_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 const RowsParams p) {
-  using S = RowsShape<D, NT, F8>;
+  static_assert(TK == TILE_KEYS || (TK == 2 * TILE_KEYS && F8 && D == 128 && NT == 1), "32-key tiles: E4M3, D 128, G <= 8");
+  using S = RowsShape<D, NT, F8, TK>;
   constexpr int KT = S::KT;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[ROWS_WARPS][R];
@@ -604,9 +615,20 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
     const int bs_shift = p.block_size == 32 ? 5 : 4;
     auto issue = [&](int stage) {
       const bool first = lc.u == a, last = lc.u == e - 1;
-      const int key0 = lc.k0 + lc.t * TILE_KEYS;
+      const int key0 = lc.k0 + lc.t * TK;
       const int lb = key0 >> bs_shift, y = key0 & (p.block_size - 1);  // block_size is 16 or 32
       const int blk = bt_lookup(p, win, lc.s, lb, lane);
+      // 32-key tiles: the second 16 keys come in a box of their own, when the segment has them
+      bool two = false;
+      int blk2 = -1, y2 = 0;
+      if constexpr (TK == 2 * TILE_KEYS) {
+        two = lc.t * TK + TILE_KEYS < lc.nkeys;
+        if (two) {
+          const int key1 = key0 + TILE_KEYS;
+          y2 = key1 & (p.block_size - 1);
+          blk2 = bt_lookup(p, win, lc.s, key1 >> bs_shift, lane);
+        }
+      }
       if (lc.t == 0 || first) {
         // warm L1 with query rows a segment ahead: the next segment's (row + 1
         // after the last KV head: rows of consecutive sequences are consecutive),
@@ -632,10 +654,15 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
         m.nkeys = lc.nkeys;
         m.flags = (first ? 1 : 0) | (last ? 2 : 0);
         if (blk < 0 || blk >= p.num_blocks) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+        if (two && (blk2 < 0 || blk2 >= p.num_blocks)) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
         uint8_t* st = ring + stage * S::STAGE_BYTES;
-        mbar_arrive_expect_tx(&bar[stage], S::STAGE_BYTES);
+        mbar_arrive_expect_tx(&bar[stage], two ? 4 * S::BOX_BYTES : 2 * S::BOX_BYTES);
         tma_load_5d(st, &tmk, &bar[stage], 0, y, 0, lc.h, blk, pol);
         tma_load_5d(st + S::HALF_BYTES, &tmv, &bar[stage], 0, y, 0, lc.h, blk, pol);
+        if (two) {  // rows 16 .. 31 of the tile (the skipped box's stale rows are masked like any past the context)
+          tma_load_5d(st + S::BOX_BYTES, &tmk, &bar[stage], 0, y2, 0, lc.h, blk2, pol);
+          tma_load_5d(st + S::HALF_BYTES + S::BOX_BYTES, &tmv, &bar[stage], 0, y2, 0, lc.h, blk2, pol);
+        }
       }
       ++issued;
       if (!last)
@@ -727,7 +754,7 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
 
       uint8_t* kt = ring + stage * S::STAGE_BYTES;
       uint8_t* vt = kt + S::HALF_BYTES;
-      const int nvalid = min(TILE_KEYS, tm.nkeys - tm.t * TILE_KEYS);
+      const int nvalid = min(TK, tm.nkeys - tm.t * TK);
       if (p.k_new && tm.t == tm.n - 1) {
         // the newest key is row nvalid - 1 of this tile: overwrite what the
         // copy brought (the append of this very launch may not have landed)
@@ -743,194 +770,310 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
         __syncwarp();
       }
 
-      // Pull the tile into registers (K as the A operand of S^T = K Q^T, V^T via
-      // ldmatrix.trans as the A operand of O^T += V^T P^T) and hand the stage
-      // back to TMA at once, so the ring never waits on the math.  With
-      // head_dim 256 both bf16 fragments would not fit in registers: V is read
-      // after the softmax and the stage is released then (E4M3 codes, one byte
-      // each, fit).
-      constexpr bool kEarly = D <= 128 || F8;
-      uint32_t kf[KT][4], vf[KT][4];
-      const int mi = lane >> 3;
-      const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
-      auto load_v = [&]() {
-        if constexpr (F8) {
-          // E4M3 V: one ldmatrix.trans of byte pairs covers m-tiles X, X + 1
-          // (16-byte chunks X, X + 1 = head-dim 16X .. 16X + 31) for keys 0-7
-          // and 8-15.  A lane receives keys 2c, 2c+1 at head-dim 2g, 2g+1 of
-          // the chunk.  The bytes stay packed in vf[X / 2]; the product loop
-          // pairs them by head-dim into the f16 A rows g (head-dim 16X + 2g)
-          // and g + 8 (head-dim 16X + 2g + 1).
-          const int rv = (lane & 7) + ((lane >> 3) & 1) * 8;
+      if constexpr (TK == 2 * TILE_KEYS) {
+        // 32-key tile (E4M3, head_dim 128, one head tile): m-tiles h = 0, 1 are
+        // the tile's rows 16h .. 16h + 15, one TMA box each.  Both m-tiles'
+        // codes come into registers (as in the 16-key path, K by ldmatrix and
+        // V by ldmatrix.trans of byte pairs), the stage goes back to TMA, and one
+        // softmax step covers the 32 keys.
+        uint32_t kf2[2][KT / 2][4], vf2[2][KT / 2][4];
+        const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
+        const int rr = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int x = 0; x < KT; x += 2) {
             const int ch = x + (lane >> 4);
-            ldsm_x4_trans(vbase + (ch >> 3) * 2048 + sw128(rv, ch & 7), vf[x / 2][0], vf[x / 2][1], vf[x / 2][2],
-                          vf[x / 2][3]);
+            ldsm_x4(kbase + h * S::BOX_BYTES + sw128(rr, ch), kf2[h][x / 2][0], kf2[h][x / 2][1], kf2[h][x / 2][2],
+                    kf2[h][x / 2][3]);
+            ldsm_x4_trans(vbase + h * S::BOX_BYTES + sw128(rr, ch), vf2[h][x / 2][0], vf2[h][x / 2][1],
+                          vf2[h][x / 2][2], vf2[h][x / 2][3]);
           }
-        } else {
-          const int rv = (lane & 7) + (mi >> 1) * 8;
 #pragma unroll
-          for (int mt = 0; mt < KT; ++mt) {
-            const int cg = 2 * mt + (mi & 1);
-            ldsm_x4_trans(vbase + (cg >> 3) * 2048 + sw128(rv, cg & 7), vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3]);
-          }
-        }
-        if (nvalid < TILE_KEYS) {
-          // keys past the context may hold anything (even NaN): their V rows must
-          // be exact zeros, since P = 0 times NaN is NaN.  This lane holds keys
-          // 2c, 2c+1 (fragments 0, 1) and 8+2c, 9+2c (fragments 2, 3).
-          const uint32_t lo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
-          const uint32_t hi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
-          if constexpr (F8) {  // packed codes: registers 0, 2 hold keys 2c, 2c+1 and 1, 3 keys 8+2c, 9+2c
+        for (int h = 0; h < 2; ++h) {  // V rows of keys past the context: exact zeros (P = 0 times NaN is NaN)
+          const int nv = nvalid - TILE_KEYS * h;
+          if (nv < TILE_KEYS) {
+            const uint32_t lo = (2 * c < nv ? 0x0000ffffu : 0u) | (2 * c + 1 < nv ? 0xffff0000u : 0u);
+            const uint32_t hi = (2 * c + 8 < nv ? 0x0000ffffu : 0u) | (2 * c + 9 < nv ? 0xffff0000u : 0u);
 #pragma unroll
             for (int x = 0; x < KT / 2; ++x) {
-              vf[x][0] &= lo;
-              vf[x][1] &= hi;
-              vf[x][2] &= lo;
-              vf[x][3] &= hi;
-            }
-          } else {
-#pragma unroll
-            for (int mt = 0; mt < KT; ++mt) {
-              vf[mt][0] &= lo;
-              vf[mt][1] &= lo;
-              vf[mt][2] &= hi;
-              vf[mt][3] &= hi;
+              vf2[h][x][0] &= lo;
+              vf2[h][x][1] &= hi;
+              vf2[h][x][2] &= lo;
+              vf2[h][x][3] &= hi;
             }
           }
         }
-      };
-      auto release = [&]() {
         __syncwarp();
         if (loading) {
           if (lane == 0) fence_proxy_async_smem();
           issue(stage);
         }
-      };
-      if constexpr (F8) {
-        // E4M3 K: one ldmatrix of byte pairs covers k-steps X, X + 1 (16-byte
-        // chunks X, X + 1) for keys 0-7 and 8-15.  A lane receives head-dim
-        // 4c .. 4c+3 of the chunk; its low pair is the f16 A column pair 2c, 2c+1
-        // of the k-step and its high pair the pair 2c+8, 2c+9 (Q uses the same
-        // order).  The codes stay packed in kf[X / 2] until the product loop.
-        const int rk = (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int x = 0; x < KT; x += 2) {
-          const int ch = x + (lane >> 4);
-          ldsm_x4(kbase + (ch >> 3) * 2048 + sw128(rk, ch & 7), kf[x / 2][0], kf[x / 2][1], kf[x / 2][2],
-                  kf[x / 2][3]);
-        }
-      } else {
-        const int rk = (lane & 7) + (mi & 1) * 8;
-#pragma unroll
-        for (int kk = 0; kk < KT; ++kk)
-          ldsm_x4(kbase + (kk >> 2) * 2048 + sw128(rk, 2 * (kk & 3) + (mi >> 1)), kf[kk][0], kf[kk][1], kf[kk][2],
-                  kf[kk][3]);
-      }
-      if constexpr (kEarly) {
-        load_v();
-        release();
-      }
 
-      // S^T[key, head] = K . Q^T
-      float sacc[NT][4];
+        // S^T[key, head] = K . Q^T for each m-tile
+        float sv[2][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-      if constexpr (F8) {  // E4M3 -> f16 just before each pair of k-steps
+        for (int h = 0; h < 2; ++h) {
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int x = 0; x < KT / 2; ++x) {
-          const uint32_t* r = kf[x];
-          const uint32_t a0 = e4m3x2_lo_to_f16x2(r[0]), a1 = e4m3x2_lo_to_f16x2(r[1]);
-          const uint32_t a2 = e4m3x2_hi_to_f16x2(r[0]), a3 = e4m3x2_hi_to_f16x2(r[1]);
-          const uint32_t b0 = e4m3x2_lo_to_f16x2(r[2]), b1 = e4m3x2_lo_to_f16x2(r[3]);
-          const uint32_t b2 = e4m3x2_hi_to_f16x2(r[2]), b3 = e4m3x2_hi_to_f16x2(r[3]);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_f16_16816(sacc[nt], a0, a1, a2, a3, qb[nt][2 * x][0], qb[nt][2 * x][1]);
-            mma_f16_16816(sacc[nt], b0, b1, b2, b3, qb[nt][2 * x + 1][0], qb[nt][2 * x + 1][1]);
+          for (int x = 0; x < KT / 2; ++x) {
+            const uint32_t* r = kf2[h][x];
+            const uint32_t a0 = e4m3x2_lo_to_f16x2(r[0]), a1 = e4m3x2_lo_to_f16x2(r[1]);
+            const uint32_t a2 = e4m3x2_hi_to_f16x2(r[0]), a3 = e4m3x2_hi_to_f16x2(r[1]);
+            const uint32_t b0 = e4m3x2_lo_to_f16x2(r[2]), b1 = e4m3x2_lo_to_f16x2(r[3]);
+            const uint32_t b2 = e4m3x2_hi_to_f16x2(r[2]), b3 = e4m3x2_hi_to_f16x2(r[3]);
+            mma_f16_16816(acc, a0, a1, a2, a3, qb[0][2 * x][0], qb[0][2 * x][1]);
+            mma_f16_16816(acc, b0, b1, b2, b3, qb[0][2 * x + 1][0], qb[0][2 * x + 1][1]);
           }
+          // this lane: keys 16h + g and 16h + g + 8 of heads 2c, 2c + 1
+          sv[h][0] = acc[0] * p.scale_log2;
+          sv[h][1] = acc[1] * p.scale_log2;
+          sv[h][2] = acc[2] * p.scale_log2;
+          sv[h][3] = acc[3] * p.scale_log2;
+          if (TILE_KEYS * h + g >= nvalid) sv[h][0] = sv[h][1] = -INFINITY;
+          if (TILE_KEYS * h + g + 8 >= nvalid) sv[h][2] = sv[h][3] = -INFINITY;
         }
-      } else {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int kk = 0; kk < KT; ++kk)
-            mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
-      }
 
-      // online softmax on the fragment: this lane holds keys g, g+8 of heads 2c, 2c+1
-      uint32_t pb[NT][2];
-      float al[NT][2];
-      bool moved = false;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        float s0 = sacc[nt][0] * p.scale_log2, s1 = sacc[nt][1] * p.scale_log2;
-        float s2 = sacc[nt][2] * p.scale_log2, s3 = sacc[nt][3] * p.scale_log2;
-        if (g >= nvalid) s0 = s1 = -INFINITY;
-        if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
-        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+        // online softmax over the 32 keys
+        float mx0 = fmaxf(fmaxf(sv[0][0], sv[0][2]), fmaxf(sv[1][0], sv[1][2]));
+        float mx1 = fmaxf(fmaxf(sv[0][1], sv[0][3]), fmaxf(sv[1][1], sv[1][3]));
 #pragma unroll
         for (int off = 4; off < 32; off <<= 1) {
           mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
           mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
         }
-        const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
-        moved |= (mn0 != m[nt][0]) | (mn1 != m[nt][1]);
-        al[nt][0] = fast_exp2(m[nt][0] - mn0);
-        al[nt][1] = fast_exp2(m[nt][1] - mn1);
-        m[nt][0] = mn0;
-        m[nt][1] = mn1;
-        const float p0 = fast_exp2(s0 - mn0), p2 = fast_exp2(s2 - mn0);
-        const float p1 = fast_exp2(s1 - mn1), p3 = fast_exp2(s3 - mn1);
-        l[nt][0] = l[nt][0] * al[nt][0] + p0 + p2;
-        l[nt][1] = l[nt][1] * al[nt][1] + p1 + p3;
-        if constexpr (F8) {  // P in f16 for the f16 MMA
-          pb[nt][0] = movmatrix_trans(pack_f16x2(p0, p1));
-          pb[nt][1] = movmatrix_trans(pack_f16x2(p2, p3));
-        } else {
-          pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
-          pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
-        }
-      }
-      if (__any_sync(FULL_MASK, moved)) {  // rescale O only when some running maximum grew
+        const float mn0 = fmaxf(m[0][0], mx0), mn1 = fmaxf(m[0][1], mx1);
+        const bool moved = (mn0 != m[0][0]) | (mn1 != m[0][1]);
+        const float al0 = fast_exp2(m[0][0] - mn0), al1 = fast_exp2(m[0][1] - mn1);
+        m[0][0] = mn0;
+        m[0][1] = mn1;
+        uint32_t pb2[2][2];
+        float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int h = 0; h < 2; ++h) {
+          const float p0 = fast_exp2(sv[h][0] - mn0), p2 = fast_exp2(sv[h][2] - mn0);
+          const float p1 = fast_exp2(sv[h][1] - mn1), p3 = fast_exp2(sv[h][3] - mn1);
+          ls0 += p0 + p2;
+          ls1 += p1 + p3;
+          pb2[h][0] = movmatrix_trans(pack_f16x2(p0, p1));  // P in f16 for the f16 MMA
+          pb2[h][1] = movmatrix_trans(pack_f16x2(p2, p3));
+        }
+        l[0][0] = l[0][0] * al0 + ls0;
+        l[0][1] = l[0][1] * al1 + ls1;
+        if (__any_sync(FULL_MASK, moved)) {  // rescale O only when some running maximum grew
 #pragma unroll
           for (int mt = 0; mt < KT; ++mt) {
-            o[mt][nt][0] *= al[nt][0];
-            o[mt][nt][1] *= al[nt][1];
-            o[mt][nt][2] *= al[nt][0];
-            o[mt][nt][3] *= al[nt][1];
-          }
-      }
-
-      // O^T[d, head] += V^T . P^T
-      if constexpr (!kEarly) {
-        load_v();
-        release();
-      }
-      if constexpr (F8) {  // pair the codes by head-dim, E4M3 -> f16, two m-tiles per packed fragment
-#pragma unroll
-        for (int x = 0; x < KT / 2; ++x) {
-          const uint32_t r0 = pair_bytes(vf[x][0]), r1 = pair_bytes(vf[x][1]);
-          const uint32_t r2 = pair_bytes(vf[x][2]), r3 = pair_bytes(vf[x][3]);
-          const uint32_t a0 = e4m3x2_lo_to_f16x2(r0), a1 = e4m3x2_hi_to_f16x2(r0);
-          const uint32_t a2 = e4m3x2_lo_to_f16x2(r1), a3 = e4m3x2_hi_to_f16x2(r1);
-          const uint32_t b0 = e4m3x2_lo_to_f16x2(r2), b1 = e4m3x2_hi_to_f16x2(r2);
-          const uint32_t b2 = e4m3x2_lo_to_f16x2(r3), b3 = e4m3x2_hi_to_f16x2(r3);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            mma_f16_16816(o[2 * x][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
-            mma_f16_16816(o[2 * x + 1][nt], b0, b1, b2, b3, pb[nt][0], pb[nt][1]);
+            o[mt][0][0] *= al0;
+            o[mt][0][1] *= al1;
+            o[mt][0][2] *= al0;
+            o[mt][0][3] *= al1;
           }
         }
+
+        // O^T[d, head] += V^T . P^T, one k-step of 16 keys per m-tile
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int x = 0; x < KT / 2; ++x) {
+            const uint32_t r0 = pair_bytes(vf2[h][x][0]), r1 = pair_bytes(vf2[h][x][1]);
+            const uint32_t r2 = pair_bytes(vf2[h][x][2]), r3 = pair_bytes(vf2[h][x][3]);
+            const uint32_t a0 = e4m3x2_lo_to_f16x2(r0), a1 = e4m3x2_hi_to_f16x2(r0);
+            const uint32_t a2 = e4m3x2_lo_to_f16x2(r1), a3 = e4m3x2_hi_to_f16x2(r1);
+            const uint32_t b0 = e4m3x2_lo_to_f16x2(r2), b1 = e4m3x2_hi_to_f16x2(r2);
+            const uint32_t b2 = e4m3x2_lo_to_f16x2(r3), b3 = e4m3x2_hi_to_f16x2(r3);
+            mma_f16_16816(o[2 * x][0], a0, a1, a2, a3, pb2[h][0], pb2[h][1]);
+            mma_f16_16816(o[2 * x + 1][0], b0, b1, b2, b3, pb2[h][0], pb2[h][1]);
+          }
       } else {
-#pragma unroll
-        for (int mt = 0; mt < KT; ++mt)
-#pragma unroll
+        // Pull the tile into registers (K as the A operand of S^T = K Q^T, V^T via
+        // ldmatrix.trans as the A operand of O^T += V^T P^T) and hand the stage
+        // back to TMA at once, so the ring never waits on the math.  With
+        // head_dim 256 both bf16 fragments would not fit in registers: V is read
+        // after the softmax and the stage is released then (E4M3 codes, one byte
+        // each, fit).
+        constexpr bool kEarly = D <= 128 || F8;
+        uint32_t kf[KT][4], vf[KT][4];
+        const int mi = lane >> 3;
+        const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
+        auto load_v = [&]() {
+          if constexpr (F8) {
+            // E4M3 V: one ldmatrix.trans of byte pairs covers m-tiles X, X + 1
+            // (16-byte chunks X, X + 1 = head-dim 16X .. 16X + 31) for keys 0-7
+            // and 8-15.  A lane receives keys 2c, 2c+1 at head-dim 2g, 2g+1 of
+            // the chunk.  The bytes stay packed in vf[X / 2]; the product loop
+            // pairs them by head-dim into the f16 A rows g (head-dim 16X + 2g)
+            // and g + 8 (head-dim 16X + 2g + 1).
+            const int rv = (lane & 7) + ((lane >> 3) & 1) * 8;
+  #pragma unroll
+            for (int x = 0; x < KT; x += 2) {
+              const int ch = x + (lane >> 4);
+              ldsm_x4_trans(vbase + (ch >> 3) * 2048 + sw128(rv, ch & 7), vf[x / 2][0], vf[x / 2][1], vf[x / 2][2],
+                            vf[x / 2][3]);
+            }
+          } else {
+            const int rv = (lane & 7) + (mi >> 1) * 8;
+  #pragma unroll
+            for (int mt = 0; mt < KT; ++mt) {
+              const int cg = 2 * mt + (mi & 1);
+              ldsm_x4_trans(vbase + (cg >> 3) * 2048 + sw128(rv, cg & 7), vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3]);
+            }
+          }
+          if (nvalid < TILE_KEYS) {
+            // keys past the context may hold anything (even NaN): their V rows must
+            // be exact zeros, since P = 0 times NaN is NaN.  This lane holds keys
+            // 2c, 2c+1 (fragments 0, 1) and 8+2c, 9+2c (fragments 2, 3).
+            const uint32_t lo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+            const uint32_t hi = (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+            if constexpr (F8) {  // packed codes: registers 0, 2 hold keys 2c, 2c+1 and 1, 3 keys 8+2c, 9+2c
+  #pragma unroll
+              for (int x = 0; x < KT / 2; ++x) {
+                vf[x][0] &= lo;
+                vf[x][1] &= hi;
+                vf[x][2] &= lo;
+                vf[x][3] &= hi;
+              }
+            } else {
+  #pragma unroll
+              for (int mt = 0; mt < KT; ++mt) {
+                vf[mt][0] &= lo;
+                vf[mt][1] &= lo;
+                vf[mt][2] &= hi;
+                vf[mt][3] &= hi;
+              }
+            }
+          }
+        };
+        auto release = [&]() {
+          __syncwarp();
+          if (loading) {
+            if (lane == 0) fence_proxy_async_smem();
+            issue(stage);
+          }
+        };
+        if constexpr (F8) {
+          // E4M3 K: one ldmatrix of byte pairs covers k-steps X, X + 1 (16-byte
+          // chunks X, X + 1) for keys 0-7 and 8-15.  A lane receives head-dim
+          // 4c .. 4c+3 of the chunk; its low pair is the f16 A column pair 2c, 2c+1
+          // of the k-step and its high pair the pair 2c+8, 2c+9 (Q uses the same
+          // order).  The codes stay packed in kf[X / 2] until the product loop.
+          const int rk = (lane & 7) + ((lane >> 3) & 1) * 8;
+  #pragma unroll
+          for (int x = 0; x < KT; x += 2) {
+            const int ch = x + (lane >> 4);
+            ldsm_x4(kbase + (ch >> 3) * 2048 + sw128(rk, ch & 7), kf[x / 2][0], kf[x / 2][1], kf[x / 2][2],
+                    kf[x / 2][3]);
+          }
+        } else {
+          const int rk = (lane & 7) + (mi & 1) * 8;
+  #pragma unroll
+          for (int kk = 0; kk < KT; ++kk)
+            ldsm_x4(kbase + (kk >> 2) * 2048 + sw128(rk, 2 * (kk & 3) + (mi >> 1)), kf[kk][0], kf[kk][1], kf[kk][2],
+                    kf[kk][3]);
+        }
+        if constexpr (kEarly) {
+          load_v();
+          release();
+        }
+
+        // S^T[key, head] = K . Q^T
+        float sacc[NT][4];
+  #pragma unroll
+        for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+        if constexpr (F8) {  // E4M3 -> f16 just before each pair of k-steps
+  #pragma unroll
+          for (int x = 0; x < KT / 2; ++x) {
+            const uint32_t* r = kf[x];
+            const uint32_t a0 = e4m3x2_lo_to_f16x2(r[0]), a1 = e4m3x2_lo_to_f16x2(r[1]);
+            const uint32_t a2 = e4m3x2_hi_to_f16x2(r[0]), a3 = e4m3x2_hi_to_f16x2(r[1]);
+            const uint32_t b0 = e4m3x2_lo_to_f16x2(r[2]), b1 = e4m3x2_lo_to_f16x2(r[3]);
+            const uint32_t b2 = e4m3x2_hi_to_f16x2(r[2]), b3 = e4m3x2_hi_to_f16x2(r[3]);
+  #pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_f16_16816(sacc[nt], a0, a1, a2, a3, qb[nt][2 * x][0], qb[nt][2 * x][1]);
+              mma_f16_16816(sacc[nt], b0, b1, b2, b3, qb[nt][2 * x + 1][0], qb[nt][2 * x + 1][1]);
+            }
+          }
+        } else {
+  #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
-            mma_bf16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+  #pragma unroll
+            for (int kk = 0; kk < KT; ++kk)
+              mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
+        }
+
+        // online softmax on the fragment: this lane holds keys g, g+8 of heads 2c, 2c+1
+        uint32_t pb[NT][2];
+        float al[NT][2];
+        bool moved = false;
+  #pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float s0 = sacc[nt][0] * p.scale_log2, s1 = sacc[nt][1] * p.scale_log2;
+          float s2 = sacc[nt][2] * p.scale_log2, s3 = sacc[nt][3] * p.scale_log2;
+          if (g >= nvalid) s0 = s1 = -INFINITY;
+          if (g + 8 >= nvalid) s2 = s3 = -INFINITY;
+          float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+  #pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(FULL_MASK, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(FULL_MASK, mx1, off));
+          }
+          const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+          moved |= (mn0 != m[nt][0]) | (mn1 != m[nt][1]);
+          al[nt][0] = fast_exp2(m[nt][0] - mn0);
+          al[nt][1] = fast_exp2(m[nt][1] - mn1);
+          m[nt][0] = mn0;
+          m[nt][1] = mn1;
+          const float p0 = fast_exp2(s0 - mn0), p2 = fast_exp2(s2 - mn0);
+          const float p1 = fast_exp2(s1 - mn1), p3 = fast_exp2(s3 - mn1);
+          l[nt][0] = l[nt][0] * al[nt][0] + p0 + p2;
+          l[nt][1] = l[nt][1] * al[nt][1] + p1 + p3;
+          if constexpr (F8) {  // P in f16 for the f16 MMA
+            pb[nt][0] = movmatrix_trans(pack_f16x2(p0, p1));
+            pb[nt][1] = movmatrix_trans(pack_f16x2(p2, p3));
+          } else {
+            pb[nt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+            pb[nt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
+          }
+        }
+        if (__any_sync(FULL_MASK, moved)) {  // rescale O only when some running maximum grew
+  #pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+  #pragma unroll
+            for (int mt = 0; mt < KT; ++mt) {
+              o[mt][nt][0] *= al[nt][0];
+              o[mt][nt][1] *= al[nt][1];
+              o[mt][nt][2] *= al[nt][0];
+              o[mt][nt][3] *= al[nt][1];
+            }
+        }
+
+        // O^T[d, head] += V^T . P^T
+        if constexpr (!kEarly) {
+          load_v();
+          release();
+        }
+        if constexpr (F8) {  // pair the codes by head-dim, E4M3 -> f16, two m-tiles per packed fragment
+  #pragma unroll
+          for (int x = 0; x < KT / 2; ++x) {
+            const uint32_t r0 = pair_bytes(vf[x][0]), r1 = pair_bytes(vf[x][1]);
+            const uint32_t r2 = pair_bytes(vf[x][2]), r3 = pair_bytes(vf[x][3]);
+            const uint32_t a0 = e4m3x2_lo_to_f16x2(r0), a1 = e4m3x2_hi_to_f16x2(r0);
+            const uint32_t a2 = e4m3x2_lo_to_f16x2(r1), a3 = e4m3x2_hi_to_f16x2(r1);
+            const uint32_t b0 = e4m3x2_lo_to_f16x2(r2), b1 = e4m3x2_hi_to_f16x2(r2);
+            const uint32_t b2 = e4m3x2_lo_to_f16x2(r3), b3 = e4m3x2_hi_to_f16x2(r3);
+  #pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_f16_16816(o[2 * x][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+              mma_f16_16816(o[2 * x + 1][nt], b0, b1, b2, b3, pb[nt][0], pb[nt][1]);
+            }
+          }
+        } else {
+  #pragma unroll
+          for (int mt = 0; mt < KT; ++mt)
+  #pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              mma_bf16_16816(o[mt][nt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], pb[nt][0], pb[nt][1]);
+        }
       }
 
       // ---- end of a piece: write the output, or a partial linked to its segment
@@ -1034,12 +1177,12 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8>() ==
 
 // ------------------------------------------------------------------ host side
 
-template <int D, int NT, int R, bool F8 = false>
+template <int D, int NT, int R, bool F8 = false, int TK = TILE_KEYS>
 static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream,
                          int num_sms) {
-  using S = RowsShape<D, NT, F8>;
+  using S = RowsShape<D, NT, F8, TK>;
   const int smem = ROWS_WARPS * R * S::STAGE_BYTES + 1024 + (ROWS_SMEM_SEQS + 1) * 8;
-  auto kern = rows_kernel<D, NT, R, F8>;
+  auto kern = rows_kernel<D, NT, R, F8, TK>;
   static int configured_dev = -1;
   static int blocks_per_sm = 1;
   int dev = 0;
@@ -1050,11 +1193,12 @@ static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUt
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, ROWS_THREADS, smem) != cudaSuccess || nb < 1)
       return PA_ERR_CUDA;
-    constexpr int cap = rows_ctas_per_sm<D, NT, F8>();
+    constexpr int cap = rows_ctas_per_sm<D, NT, F8, TK>();
     blocks_per_sm = nb > cap ? cap : nb;
     configured_dev = dev;
   }
   RowsParams p = p0;
+  p.tile_shift = TK == 32 ? 5 : 4;
   const int grid = num_sms * blocks_per_sm;
   p.total_warps = grid * ROWS_WARPS;
   // Programmatic dependent launch: the prologue (a scan of the batch
@@ -1145,7 +1289,7 @@ int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& 
     switch (head_dim) {
       case 128:
         return two ? launch_rows_t<128, 2, 6, true>(p, tmk, tmv, stream, num_sms)
-                   : launch_rows_t<128, 1, 4, true>(p, tmk, tmv, stream, num_sms);
+                   : launch_rows_t<128, 1, 3, true, 32>(p, tmk, tmv, stream, num_sms);
       case 256:
         return launch_rows_t<256, 1, 3, true>(p, tmk, tmv, stream, num_sms);
       default:

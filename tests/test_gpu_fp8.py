@@ -70,6 +70,7 @@ FP8_SMALL = [  # prefix list, Hq, Hkv, d, bs
     ([30, 500, 2000], 16, 1, 128, 32),       # 16 heads per KV head: two 8-wide head tiles
     ([5, 300, 1500], 12, 2, 256, 16),
     ([32000, 24999], 16, 2, 128, 16),        # long contexts: segments split over many warps
+    ([7, 31, 32, 33, 47, 300, 1000], 8, 2, 128, 32),  # 32-token blocks: both 16-row halves of a tile in one block
 ]
 
 
