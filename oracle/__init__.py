@@ -50,11 +50,12 @@ PINS = {
     ],
     "cache_append": ["test_append_is_a_byte_copy", "test_append_then_attend_reads_new_row"],
     "slot_mapping": ["test_slot_mapping_closed_form", "test_allocator_slots_match_oracle"],
-    "e4m3_to_f64": ["test_e4m3_values_from_the_definition"],
-    "f32_to_e4m3": ["test_e4m3_round_trip_and_monotone", "test_e4m3_ties_to_even_and_saturation"],
-    "cache_append_fp8": ["test_fp8_append_writes_codes_of_the_scaled_rows"],
+    "e4m3_to_f64": ["test_e4m3_values_from_the_definition", "test_fp8_mutations_are_caught"],
+    "f32_to_e4m3": ["test_e4m3_round_trip_and_monotone", "test_e4m3_ties_to_even_and_saturation",
+                    "test_fp8_mutations_are_caught"],
+    "cache_append_fp8": ["test_fp8_append_writes_codes_of_the_scaled_rows", "test_fp8_mutations_are_caught"],
     "paged_attention_fp8": ["test_fp8_attention_equals_bf16_attention_on_exact_values",
-                            "test_fp8_scales_factor_out"],
+                            "test_fp8_scales_factor_out", "test_fp8_mutations_are_caught"],
 }
 
 

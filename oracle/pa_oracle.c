@@ -51,6 +51,10 @@
  *   3: the scale is ignored                          4: cache rows read head-major
  *   5: no normalisation by the weight sum            6: no max subtraction
  *   7: the append writes every head's row to head 0  8: offset = pos / block_size
+ *   FP8 (E4M3) cache:
+ *   9: exponent bias 8 when decoding                 10: encoding rounds toward zero
+ *  11: encoding does not saturate at 448            12: attention leaves out the V scale
+ *  13: the append multiplies by the scale, not by its inverse
  */
 #ifndef ORACLE_MUTATION
 #define ORACLE_MUTATION 0
@@ -309,7 +313,11 @@ double oracle_e4m3_to_f64(uint8_t c)
     int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
     if (e == 15 && m == 7)
         return NAN;
+#if ORACLE_MUTATION == 9
+    double v = (e == 0) ? ldexp(m / 8.0, -7) : ldexp(1.0 + m / 8.0, e - 8);
+#else
     double v = (e == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+#endif
     return sgn ? -v : v;
 }
 
@@ -328,9 +336,15 @@ uint8_t oracle_f32_to_e4m3(float xf)
     frexp(a, &e2);           /* a = f * 2^e2, f in [0.5, 1): floor(log2 a) = e2 - 1 */
     int ex = e2 - 1;
     double quantum = ex < -6 ? ldexp(1.0, -9) : ldexp(1.0, ex - 3);
+#if ORACLE_MUTATION == 10
+    double r = floor(a / quantum) * quantum;
+#else
     double r = nearbyint(a / quantum) * quantum; /* a / quantum is exact; ties to even */
+#endif
+#if ORACLE_MUTATION != 11
     if (r > 448.0)
         r = 448.0; /* saturate to the largest finite value */
+#endif
     if (r == 0.0)
         return sgn;
     frexp(r, &e2);
@@ -361,8 +375,13 @@ int oracle_cache_append_fp8(const uint16_t *k_new, const uint16_t *v_new, uint8_
             long long dst = ((blk * num_kv_heads + h) * block_size + off) * head_dim;
             long long src = ((long long)t * num_kv_heads + h) * head_dim;
             for (int d = 0; d < head_dim; ++d) {
+#if ORACLE_MUTATION == 13
+                float kx = (float)bf16_bits_to_double(k_new[src + d]) * (1.0f / k_inv_scale);
+                float vx = (float)bf16_bits_to_double(v_new[src + d]) * (1.0f / v_inv_scale);
+#else
                 float kx = (float)bf16_bits_to_double(k_new[src + d]) * k_inv_scale;
                 float vx = (float)bf16_bits_to_double(v_new[src + d]) * v_inv_scale;
+#endif
                 k_cache[dst + d] = oracle_f32_to_e4m3(kx);
                 v_cache[dst + d] = oracle_f32_to_e4m3(vx);
             }
@@ -405,7 +424,11 @@ static int attend_one_fp8(double *out, const uint16_t *q_row, const uint8_t *k_c
         long long blk = row / block_size, off = row % block_size;
         const uint8_t *vrow = v_cache + ((blk * num_kv_heads + kvh) * block_size + off) * head_dim;
         for (int d = 0; d < head_dim; ++d)
+#if ORACLE_MUTATION == 12
+            acc[d] += w * oracle_e4m3_to_f64(vrow[d]);
+#else
             acc[d] += w * (oracle_e4m3_to_f64(vrow[d]) * v_scale);
+#endif
         denom += w;
     }
     for (int d = 0; d < head_dim; ++d)
