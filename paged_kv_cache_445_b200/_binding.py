@@ -264,8 +264,9 @@ def pa_decode_fp8(out, q, k_cache, v_cache, block_tables, context_lens, scale, k
 
 def pa_prefill_chunk(out, q, query_start, k_cache, v_cache, block_tables, context_lens, scale, workspace,
                      dev_status=None, stream=None) -> None:
-    """Varlen batch of prefill chunks and decodes: q/out [Tq, Hq, d],
-    query_start [B + 1]; see include/pa.h."""
+    """Varlen batch of prefill chunks, multi-token verification rows and
+    decodes: q/out [Tq, Hq, d], query_start [B + 1]; see include/pa.h (which
+    kernel takes which sequences)."""
     op, qp, kc, vc, bt, cl, ws = _attention_args(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
     qs = _dev(query_start, "query_start", torch.int32, 1)
     if query_start.shape[0] != context_lens.shape[0] + 1:
