@@ -119,3 +119,20 @@ def test_groups_the_tensor_core_paths_do_not_take_run_on_the_decode_kernel():
     compare(got, _ref(w, kc, vc), "G 6")
     assert int(ds.status.item()) == 0
 
+
+
+def test_batches_past_the_multi_row_kernels_sequence_limit_run_on_the_chunk_kernel():
+    # 600 sequences of 4 rows: more than the multi-row kernel's 512, so the chunk kernel takes them
+    rng = np.random.default_rng(23)
+    prefix = rng.integers(20, 200, 600).tolist()
+    w = workloads.custom(prefix, [4] * 600, 16, 2, 128, 16, seed=23, poison=True)
+    ds = DeviceStep(w)
+    got = ds.step()
+    kc, vc = oracle_after_append(w)
+    rows = sorted({0, 1, 599, *rng.integers(0, 600, 20).tolist()})
+    only = np.array([(t, h) for s in rows for t in range(int(w.query_start[s]), int(w.query_start[s + 1]))
+                     for h in range(w.num_q_heads)])
+    ref = _ref(w, kc, vc, only=only)
+    idx = tuple(only.T)
+    compare(got[idx], ref[idx], "600 sequences")
+    assert int(ds.status.item()) == 0
