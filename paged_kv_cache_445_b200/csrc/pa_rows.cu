@@ -9,7 +9,8 @@
 // p = context_len - 1.
 //
 // How (B200):
-//  * Work unit = one 16-key tile of one (query row, KV head) "segment".  All
+//  * Work unit = one 16-key tile (32 keys in the E4M3 kernel at head_dim 128
+//    with one head tile) of one (query row, KV head) "segment".  All
 //    G = Hq / Hkv query heads of the KV head ride along, so each K/V byte is
 //    read from HBM once per step.  Each CTA scans context_lens into shared
 //    memory (tile prefix sums per sequence), every warp takes an equal

@@ -120,7 +120,6 @@ def test_groups_the_tensor_core_paths_do_not_take_run_on_the_decode_kernel():
     assert int(ds.status.item()) == 0
 
 
-
 def test_batches_past_the_multi_row_kernels_sequence_limit_run_on_the_chunk_kernel():
     # 600 sequences of 4 rows: more than the multi-row kernel's 512, so the chunk kernel takes them
     rng = np.random.default_rng(23)
