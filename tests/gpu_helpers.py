@@ -12,6 +12,15 @@ MAX_ABS = 1e-2
 REL_L2 = 5e-3
 
 
+def load_library() -> str:
+    """Compile the in-tree libpa.so if it is missing or older than its sources
+    (nvcc, about 30 s), then load it; raises if it cannot be built."""
+    from paged_kv_cache_445_b200.csrc import build as pabuild
+    pabuild.build()
+    import paged_kv_cache_445_b200 as pa
+    return pa.library_path  # touching a binding name loads the library
+
+
 def bf16_to_dev(bits: np.ndarray, device="cuda") -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
 

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from paged_kv_cache_445_b200 import workloads
-from tests.gpu_helpers import DeviceStep, compare, oracle_after_append
+from tests.gpu_helpers import DeviceStep, compare, load_library, oracle_after_append
 
 pytestmark = pytest.mark.gpu
 
@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(scope="module", autouse=True)
 def _gpu():
     assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
-    import paged_kv_cache_445_b200 as pa  # noqa: F401
+    load_library()
 
 
 def _ref(w, kc, vc, only=None):

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from paged_kv_cache_445_b200 import workloads
-from tests.gpu_helpers import DeviceStep, compare, i32
+from tests.gpu_helpers import DeviceStep, compare, i32, load_library
 
 pytestmark = pytest.mark.gpu
 
@@ -24,6 +24,7 @@ def _static(ds: DeviceStep, out: torch.Tensor):
 
 def test_static_scratch_matches_pa_decode_on_two_calls_in_a_row():
     assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    load_library()
     # long contexts next to short ones: many (row, head) segments are split
     # between warps, so the scratch (barrier counters, segment records,
     # partial results) is really used
