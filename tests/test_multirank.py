@@ -102,3 +102,17 @@ def test_launch_count_per_step():
     assert bench.step_launches(mixed_d64) == 2
     verify = workloads.custom([200, 30, 90], [4, 2, 8], 16, 2, 128, 16, seed=1)
     assert bench.verify_batch(verify) and not bench.verify_batch(mixed) and not bench.verify_batch(decode)
+
+
+def test_l2_is_flushed_exactly_for_workloads_whose_kv_fits_in_it():
+    from paged_kv_cache_445_b200 import roofline
+    flushed = []
+    for cfg in (1, 2, 3, 4, 5, 6):
+        w = workloads.standard(cfg)
+        unique = roofline.unique_kv_bytes(w.block_tables, w.context_lens, w.block_size, w.num_kv_heads, w.head_dim)
+        if bench.l2_flush_needed(unique):
+            flushed.append(cfg)
+            assert bench.l2_note(True, 0, unique).startswith("flushed")
+    # the tiny case and the shared-prefix batch (86 MB of distinct KV) fit in the 126 MB L2
+    assert flushed == [1, 4]
+    assert bench.FLUSH_BYTES > bench.L2_BYTES
