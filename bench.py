@@ -612,17 +612,30 @@ def oracle_baseline(w, seconds: float, max_rows: int = 16, fp8: bool = False):
         scales, sample_bytes = (k_scale, v_scale), sample_bytes // 2
     else:
         kc, vc = w.k_cache, w.v_cache  # appended in place: the same rows every step
-    n, t0 = 0, time.perf_counter()
-    while True:
-        oracle_step(oracle, w, only, kc, vc, scales)
-        n += 1
-        if time.perf_counter() - t0 >= seconds:
-            break
-    dt = (time.perf_counter() - t0) / n
-    return {"value": round(sample_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"{len(seqs)} sequences x {w.num_q_heads} heads of the same workload (append of all "
-                      f"{len(w.slot_mapping)} rows + attention of the sampled rows), {n} steps in {n * dt:.1f} s"}
+    def timed(budget_s):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            oracle_step(oracle, w, only, kc, vc, scales)
+            n += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        return n, (time.perf_counter() - t0) / n
+
+    cores = oracle.num_threads()
+    n, dt = timed(seconds)
+    what = (f"{len(seqs)} sequences x {w.num_q_heads} heads of the same workload (append of all "
+            f"{len(w.slot_mapping)} rows + attention of the sampled rows)")
+    line = {"value": round(sample_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{what}, {n} steps in {n * dt:.1f} s"}
+    if cores > 1:  # the same sample on one core
+        oracle.set_num_threads(1)
+        try:
+            n1, dt1 = timed(seconds / 4)
+        finally:
+            oracle.set_num_threads(cores)
+        line["single_core"] = {"value": round(sample_bytes / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                               "sample": f"{what}, {n1} steps in {n1 * dt1:.1f} s"}
+    return line
 
 
 def run_reference(args):

@@ -103,6 +103,8 @@ def _bind(lib):
     lib.oracle_paged_attention_fp8.restype = ci
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ci
+    lib.oracle_set_num_threads.argtypes = [ci]
+    lib.oracle_set_num_threads.restype = None
     return lib
 
 
@@ -124,6 +126,12 @@ def _c(a, dtype):
 def num_threads() -> int:
     """Threads the OpenMP runtime gives the oracle (OMP_NUM_THREADS or all cores)."""
     return int(load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the oracle's later calls from this thread (timing only: the
+    result does not depend on it)."""
+    load().oracle_set_num_threads(int(n))
 
 
 def slot_mapping(block_tables, context_lens, query_start, block_size, num_blocks, lib=None):

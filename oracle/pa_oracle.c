@@ -499,6 +499,16 @@ int oracle_paged_attention_fp8(double *out, const uint16_t *q, const uint8_t *k_
     return status;
 }
 
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 int oracle_num_threads(void)
 {
     int n = 1;

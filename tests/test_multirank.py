@@ -116,3 +116,13 @@ def test_l2_is_flushed_exactly_for_workloads_whose_kv_fits_in_it():
     # the tiny case and the shared-prefix batch (86 MB of distinct KV) fit in the 126 MB L2
     assert flushed == [1, 4]
     assert bench.FLUSH_BYTES > bench.L2_BYTES
+
+
+def test_cpu_baseline_reports_all_cores_and_one_core():
+    import oracle
+    cores = oracle.num_threads()
+    line = bench.oracle_baseline(workloads.standard(1), 0.2)
+    assert line["kind"] == "oracle" and line["cores"] == cores and line["value"] > 0
+    if cores > 1:
+        assert line["single_core"]["cores"] == 1 and line["single_core"]["value"] > 0
+    assert oracle.num_threads() == cores  # the thread count is restored
