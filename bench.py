@@ -548,7 +548,9 @@ def run_ours(args, peaks):
                        "pa_cascade_kernel + pa_rows_kernel (shared prefixes once, then the private keys)"
                        if g.cascade else
                        "pa_rows_kernel (append + attention, one launch)" if g.fused else "pa_rows_kernel (attention)"),
-            "bound": "hbm",
+            "bound": _rl.bound(flops, launch_bytes, bf16_burst * 1e12, hbm * 1e9),
+            "intensity_flop_per_byte": round(flops / launch_bytes, 2),
+            "ridge_flop_per_byte": round(_rl.ridge_point(bf16_burst * 1e12, hbm * 1e9), 1),
             "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
             if peak_src == "measured" else "fallback 6.65 TB/s",

@@ -64,3 +64,24 @@ def prefill_flops(context_lens, query_start, num_q_heads: int, head_dim: int) ->
         keys = int(n) - qlen + 1 + np.arange(qlen, dtype=np.int64)
         total += int(keys.sum())
     return 4 * head_dim * num_q_heads * total
+
+
+def ridge_point(peak_flops_per_s: float, peak_bytes_per_s: float) -> float:
+    """FLOP per byte at which a kernel stops being bound by memory bandwidth
+    and becomes bound by arithmetic: peak FLOP/s over peak bytes/s.  The
+    section on the ops:byte framework of "Inference optimization" (AI
+    Engineering from Scratch, Phase 10 / 12) puts A100's crossover near 156
+    this way, and its table of scenarios reads the bound off that point."""
+    return peak_flops_per_s / peak_bytes_per_s
+
+
+def stream_time_s(nbytes: float, bytes_per_s: float) -> float:
+    """Least time to read nbytes once at bytes_per_s: the floor that page's
+    section "Prefill vs decode" gives one decode step, every weight streamed
+    from HBM per token."""
+    return nbytes / bytes_per_s
+
+
+def bound(flops: float, nbytes: float, peak_flops_per_s: float, peak_bytes_per_s: float) -> str:
+    """"hbm" below the ridge point, "tensor" at or above it."""
+    return "hbm" if flops < ridge_point(peak_flops_per_s, peak_bytes_per_s) * nbytes else "tensor"

@@ -205,3 +205,14 @@ def test_bf16_rounding_ties_to_even():
     back = workloads.bf16_bits_to_f32(bits)
     assert back.tolist() == [1.0, 1.0, 1.0 + 2 ** -6, -2.5]
     assert math.isclose(float(workloads.bf16_bits_to_f32(workloads.f32_to_bf16_bits(np.float32([3.14159])))[0]), 3.140625)
+
+
+def test_roofline_points_match_the_printed_numbers():
+    fx = json.load(open(os.path.join(GOLDEN, "roofline_points.json")))
+    r = fx["ridge"]
+    assert roofline.ridge_point(r["peak_flops_per_s"], r["peak_bytes_per_s"]) == pytest.approx(r["printed"])
+    f = fx["floor"]
+    assert roofline.stream_time_s(f["bytes"], f["bytes_per_s"]) * 1e3 == pytest.approx(f["printed_ms"])
+    for row in fx["table"]:  # the page's bound column, from the ridge point ("batch 256" sits on the edge: left out)
+        got = roofline.bound(row["ops_per_byte"] * 1e9, 1e9, r["peak_flops_per_s"], r["peak_bytes_per_s"])
+        assert got == row["expect"], row["scenario"]
