@@ -428,7 +428,7 @@ def run_ours(args, peaks):
     if flush:
         # the same steps with L2 flushed before each; only the steps are timed
         warm_ms_step = max_over_ranks(ms_total / args.steps, world)
-        scratch = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        scratch = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=g.out.device)
         whole = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                  for _ in range(args.steps)]
         barrier(world)
@@ -484,7 +484,7 @@ def run_ours(args, peaks):
     barrier(world)
     e2e_ms = max_over_ranks(e_start.elapsed_time(e_end) / args.steps, world)
     if flush:  # as above: L2 flushed before each step, the steps alone timed
-        scratch = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+        scratch = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=g.out.device)
         whole = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                  for _ in range(args.steps)]
         barrier(world)
