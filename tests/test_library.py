@@ -92,3 +92,45 @@ def test_static_scratch_size_matches_the_header():
     m = re.search(r"#define\s+PA_STATIC_SCRATCH_BYTES\s+\((\d+)u\s*\*\s*(\d+)u\s*\*\s*(\d+)u\)", open(HEADER).read())
     assert m, "PA_STATIC_SCRATCH_BYTES not found"
     assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == _binding.STATIC_SCRATCH_BYTES
+
+
+def test_every_entry_point_rejects_bad_arguments_before_touching_a_device():
+    # each case returns from the host checks, before any CUDA call (this machine may have no GPU)
+    from paged_kv_cache_445_b200 import _binding as b
+    L, f, odd = b._lib, 4096, 4098  # f: a 16-byte aligned stand-in pointer; odd: a misaligned one
+
+    def decode(out=f, q=f, ws=f, seqs=4, d=128):
+        return L.pa_decode(out, q, f, f, f, 4, f, seqs, 8, 2, d, 16, 10, 0.1, ws, 1 << 20, None, None)
+    assert decode(seqs=0) == b.PA_OK                       # empty batch: nothing to do
+    assert decode(out=odd) == b.PA_ERR_SHAPE               # misaligned output
+    assert decode(ws=None) == b.PA_ERR_NULL                # no workspace
+
+    def fused(k_new, v_new):
+        return L.pa_decode_append(f, f, k_new, v_new, f, f, f, 4, f, 4, 8, 2, 128, 16, 10, 0.1, f, 1 << 20, None,
+                                  None)
+    assert fused(None, f) == b.PA_ERR_NULL and fused(f, None) == b.PA_ERR_NULL
+    assert fused(odd, f) == b.PA_ERR_SHAPE
+
+    def fp8(k_scale=0.5, v_scale=0.25, d=128, k_new=None, v_new=None):
+        return L.pa_decode_fp8(f, f, k_new, v_new, f, f, f, 4, f, 4, 8, 2, d, 16, 10, 0.1, k_scale, v_scale, f,
+                               1 << 20, None, None)
+    for ks, vs in ((0.0, 0.25), (0.5, -1.0), (float("inf"), 0.25), (0.5, float("nan"))):
+        assert fp8(ks, vs) == b.PA_ERR_SHAPE, (ks, vs)
+    assert fp8(d=64) == b.PA_ERR_UNSUPPORTED
+    assert fp8(k_new=f) == b.PA_ERR_NULL
+
+    def app8(n=3, d=128, ks=0.5):
+        return L.pa_cache_append_fp8(f, f, f, f, f, n, 10, 2, d, 16, ks, 0.25, None, None)
+    assert app8(ks=0.0) == b.PA_ERR_SHAPE and app8(d=100) == b.PA_ERR_UNSUPPORTED and app8(n=0) == b.PA_OK
+
+    def chunk(qs=f, seqs=4, total=9):
+        return L.pa_prefill_chunk(f, f, qs, f, f, f, 4, f, seqs, total, 8, 2, 128, 16, 10, 0.1, f, 1 << 20, None,
+                                  None)
+    assert chunk(qs=None) == b.PA_ERR_NULL and chunk(total=-1) == b.PA_ERR_SHAPE and chunk(seqs=0) == b.PA_OK
+
+    assert L.pa_decode_cascade(f, f, f, None, f, f, f, 4, f, 4, 8, 2, 128, 16, 10, 0.1, f, f, 1, f, 1 << 20, None,
+                               None) == b.PA_ERR_NULL
+    assert L.pa_cascade_workspace_bytes(4, 6, 4, 128, 8, 16) == 0  # Hq not a multiple of Hkv
+    assert L.pa_decode_static_scratch(f, f, f, f, f, 4, f, 4, 8, 2, 96, 16, 10, 0.1, None,
+                                      None) == b.PA_ERR_UNSUPPORTED
+    assert L.pa_decode_static_scratch(None, f, f, f, f, 4, f, 4, 8, 2, 128, 16, 10, 0.1, None, None) == b.PA_ERR_NULL
