@@ -134,3 +134,32 @@ def test_every_entry_point_rejects_bad_arguments_before_touching_a_device():
     assert L.pa_decode_static_scratch(f, f, f, f, f, 4, f, 4, 8, 2, 96, 16, 10, 0.1, None,
                                       None) == b.PA_ERR_UNSUPPORTED
     assert L.pa_decode_static_scratch(None, f, f, f, f, 4, f, 4, 8, 2, 128, 16, 10, 0.1, None, None) == b.PA_ERR_NULL
+
+
+def test_oracle_and_product_share_no_code():
+    # the oracle imports nothing of the product package, the product nothing of the oracle, and the
+    # oracle's C file includes no header of the CUDA library
+    import ast
+    import glob
+    root = pabuild.ROOT
+
+    def imports(path):
+        names = set()
+        for node in ast.walk(ast.parse(open(path).read())):
+            if isinstance(node, ast.Import):
+                names |= {a.name.split(".")[0] for a in node.names}
+            elif isinstance(node, ast.ImportFrom) and node.module and node.level == 0:
+                names.add(node.module.split(".")[0])
+            elif isinstance(node, ast.ImportFrom) and node.level > 0:
+                names.add(".")
+        return names
+    for path in glob.glob(os.path.join(root, "oracle", "*.py")):
+        assert "paged_kv_cache_445_b200" not in imports(path), path
+    for path in glob.glob(os.path.join(root, "paged_kv_cache_445_b200", "**", "*.py"), recursive=True):
+        assert "oracle" not in imports(path), path
+    c_src = open(os.path.join(root, "oracle", "pa_oracle.c")).read()
+    included = re.findall(r'#include\s+[<"]([^>"]+)[>"]', c_src)
+    assert included and all(not h.startswith("pa") for h in included), included
+    for path in glob.glob(os.path.join(root, "paged_kv_cache_445_b200", "csrc", "*")):
+        if path.endswith((".cu", ".cuh", ".h")):
+            assert "pa_oracle" not in open(path).read(), path
