@@ -163,3 +163,22 @@ def test_oracle_and_product_share_no_code():
     for path in glob.glob(os.path.join(root, "paged_kv_cache_445_b200", "csrc", "*")):
         if path.endswith((".cu", ".cuh", ".h")):
             assert "pa_oracle" not in open(path).read(), path
+
+
+def test_a_missing_library_fails_loudly(tmp_path):
+    # the package without libpa.so: touching any entry point raises, there is no fallback
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(pabuild.ROOT, "paged_kv_cache_445_b200")
+    dst = tmp_path / "paged_kv_cache_445_b200"
+    dst.mkdir()
+    for name in os.listdir(pkg):
+        if name.endswith(".py"):
+            shutil.copy(os.path.join(pkg, name), dst / name)
+    code = ("import paged_kv_cache_445_b200 as pa\n"
+            "try:\n    pa.pa_decode\nexcept ImportError as e:\n    print('raised:', e)\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True, timeout=300,
+                       env={**os.environ, "PYTHONPATH": str(tmp_path)})
+    assert r.returncode == 0, r.stderr
+    assert "raised:" in r.stdout and "no CPU fallback" in r.stdout
