@@ -14,6 +14,8 @@ import os
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import oracle
 from oracle import brute
@@ -315,3 +317,25 @@ def test_mutations_are_caught(mutation):
         except (AssertionError, ValueError):
             failed.append(pin.__name__)
     assert failed, f"mutation {mutation} passed every pin"
+
+
+@settings(max_examples=40, deadline=None)
+@given(st.data())
+def test_paged_equals_contiguous_brute_on_random_shapes(data):
+    # the brute-force pin over shapes drawn at random: lengths 1..70, rows 1..len, groups 1..4,
+    # head dims 8..32, blocks of 4..32 tokens, any physical placement, NaN in every unused slot
+    hkv = data.draw(st.integers(1, 3))
+    hq = hkv * data.draw(st.integers(1, 4))
+    d = data.draw(st.sampled_from([8, 16, 32]))
+    bs = data.draw(st.sampled_from([4, 8, 16, 32]))
+    lens = data.draw(st.lists(st.integers(1, 70), min_size=1, max_size=4))
+    qlens = [data.draw(st.integers(1, n)) for n in lens]
+    seed = data.draw(st.integers(0, 2**31 - 1))
+    rng = np.random.default_rng(seed)
+    k_seqs, v_seqs, q, nb = _contiguous_case(rng, lens, qlens, hq, hkv, d, bs, extra_blocks=2)
+    kc, vc, bt = scatter_to_pool(k_seqs, v_seqs, bs, nb, rng.permutation(nb))
+    qs = np.concatenate([[0], np.cumsum(qlens)])
+    scale = 1.0 / math.sqrt(d)
+    got = _attend(oracle.load(), q, kc, vc, bt, np.array(lens), qs, scale)
+    want = _brute_all(q, k_seqs, v_seqs, qlens, hq, scale)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-10)
