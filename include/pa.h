@@ -276,7 +276,13 @@ PA_API int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start
  *
  * Set-up: the first call on a device, with that device current, looks up the
  * array's device address (which may load the library's device code there).
- * Make that first call before any stream capture on that device.
+ * Make that first call before any stream capture on that device.  The address
+ * is kept per device with the identity of the CUDA context it belongs to;
+ * after a device reset (a new primary context) the next call looks it up
+ * again, so it too should come before any capture.
+ *
+ * An empty batch (num_seqs = 0) goes through exactly pa_decode's checks and
+ * launches nothing.
  */
 #define PA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
 PA_API int pa_decode_static_scratch(void* out, const void* q, const void* k_cache, const void* v_cache,

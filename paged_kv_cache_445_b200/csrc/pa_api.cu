@@ -25,8 +25,6 @@ EncodeTiledFn encode_fn() {
 
 namespace {
 
-constexpr int MAX_DEVICES = 64;
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 
@@ -34,16 +32,15 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 }  // namespace
 
 int device_info(DeviceInfo* info) {
-  static int sms[MAX_DEVICES] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return PA_ERR_CUDA;
-  if (sms[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return PA_ERR_CUDA;
-    sms[dev] = n;
-  }
-  info->num_sms = sms[dev];
-  return PA_OK;
+  static PerDevice sms;
+  return per_device(
+      sms,
+      [](int dev) {
+        int n = 0;
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n
+                                                                                                       : PA_ERR_CUDA;
+      },
+      &info->num_sms);
 }
 
 // [num_blocks, Hkv, block_size, D] bf16 viewed as a 5-D tensor

@@ -12,6 +12,7 @@
 // consecutive 16-byte pieces of k_new (coalesced) and write whole 128..512-byte
 // rows of the cache.
 #include "pa_device.cuh"
+#include "pa_internal.h"
 
 namespace pa {
 
@@ -103,13 +104,17 @@ int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_c
   if (total == 0) return PA_OK;
   // Ask for the same L1/shared split as the attention kernels that follow,
   // so that the SMs need no reconfiguration between the two launches.
-  static int carveout_dev = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && carveout_dev != dev) {
-    cudaFuncSetAttribute(append_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                         cudaSharedmemCarveoutMaxShared);
-    carveout_dev = dev;
-  }
+  static PerDevice carveout;
+  int done = 0;
+  (void)per_device(
+      carveout,
+      [](int) {
+        (void)cudaFuncSetAttribute(append_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                   cudaSharedmemCarveoutMaxShared);
+        (void)cudaGetLastError();  // a preference only: a refusal is not an error
+        return 1;
+      },
+      &done);
   const int threads = 256;
   long long blocks = (total + threads - 1) / threads;
   const long long cap = static_cast<long long>(num_sms) * 8;

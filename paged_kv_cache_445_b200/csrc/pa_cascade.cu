@@ -475,14 +475,16 @@ static int launch_cascade_t(const CascadeParams& p, const void* q, const void* k
   }
   auto kern = cascade_kernel<D>;
   const int smem = S::SMEM_TOTAL + 1024;
-  static int configured_dev = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  if (configured_dev != dev) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return PA_ERR_CUDA;
-    configured_dev = dev;
-  }
+  static PerDevice configured;
+  int done = 0;
+  const int rc_setup = per_device(
+      configured,
+      [&](int) {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1
+                                                                                                           : PA_ERR_CUDA;
+      },
+      &done);
+  if (rc_setup != PA_OK) return rc_setup;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(num_sms));  // persistent: the item count is known on the device only
   cfg.blockDim = dim3(CS_THREADS);

@@ -581,14 +581,16 @@ static int launch_chunk_t(const ChunkParams& p, const CUtensorMap& tq, const CUt
                           cudaStream_t stream, int num_sms) {
   auto kern = chunk_kernel<G>;
   const int smem = SMEM_TOTAL + 1024;
-  static int configured_dev = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  if (configured_dev != dev) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return PA_ERR_CUDA;
-    configured_dev = dev;
-  }
+  static PerDevice configured;
+  int done = 0;
+  const int rc_setup = per_device(
+      configured,
+      [&](int) {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1
+                                                                                                           : PA_ERR_CUDA;
+      },
+      &done);
+  if (rc_setup != PA_OK) return rc_setup;
   const int grid = num_sms;  // persistent: CTAs walk the items (their count is known on the device only)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));

@@ -6,9 +6,36 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "pa.h"
 
 namespace pa {
+
+// Per-device launch set-up of one kernel (its shared-memory opt-in, its CTAs
+// per SM), done once per device and safe under concurrent callers: the value
+// is an atomic, and two threads that set the same device up at once both make
+// the same idempotent CUDA calls and store the same value.
+constexpr int PA_MAX_DEVICES = 64;
+struct PerDevice {
+  std::atomic<int> value[PA_MAX_DEVICES];  // 0: not set up on that device yet
+};
+
+// The current device's value of `cache`, computed by setup() (a positive
+// value, else a pa_status) the first time.  Returns a pa_status.
+template <class Setup>
+int per_device(PerDevice& cache, Setup setup, int* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= PA_MAX_DEVICES) return PA_ERR_CUDA;
+  int v = cache.value[dev].load(std::memory_order_acquire);
+  if (v <= 0) {
+    v = setup(dev);
+    if (v <= 0) return v < 0 ? v : PA_ERR_CUDA;
+    cache.value[dev].store(v, std::memory_order_release);
+  }
+  *out = v;
+  return PA_OK;
+}
 
 // Batch size up to which the rows kernel keeps per-sequence prefix sums of
 // tile counts in shared memory (larger batches scan context_lens instead).

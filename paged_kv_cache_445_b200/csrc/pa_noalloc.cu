@@ -17,9 +17,12 @@
 //    the part that must start at zero (barrier counters and segment records)
 //    on the caller's stream, so a call that follows a failed one is still
 //    correct.
-//  * The first call on a device looks the array's address up (that may load
-//    this file's device code on the device).  Make that first call before any
-//    stream capture on that device.
+//  * The first call on a device (in each CUDA context of it) looks the array's
+//    address up; that may load this file's device code on the device.  Make
+//    that first call before any stream capture on that device.  The address is
+//    cached per device together with the identity of the context it was taken
+//    in: after a device reset the primary context is a new one, its copy of
+//    the array may sit at another address, and the next call looks it up again.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -35,24 +38,66 @@ namespace pa {
 namespace {
 
 constexpr int MAX_DEVICES = 64;
-std::mutex g_setup_mu;
-void* g_scratch_ptr[MAX_DEVICES] = {};
 
-// Address of this device's copy of g_decode_scratch; looked up once per device.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+struct ScratchAddress {
+  unsigned long long ctx_id;  // the context the address belongs to
+  void* ptr;                  // nullptr: not looked up yet
+};
+
+std::mutex g_setup_mu;
+ScratchAddress g_scratch[MAX_DEVICES] = {};
+
+// Unique ID of the calling thread's current CUDA context (IDs are never reused
+// within a process, unlike context handles).  Returns false if there is none.
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Address of the current device's copy of g_decode_scratch, looked up once per
+// (device, context) with that device current.
 int scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return PA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      (void)cudaGetLastError();
-      return PA_ERR_CUDA;
-    }
-    g_scratch_ptr[dev] = p;
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id);
+  if (have_id && g_scratch[dev].ptr && g_scratch[dev].ctx_id == id) {
+    *out = g_scratch[dev].ptr;
+    return PA_OK;
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    (void)cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
+  // the lookup makes the device's primary context current if no context was
+  unsigned long long id_now = 0;
+  if (current_context_id(&id_now)) {
+    g_scratch[dev].ctx_id = id_now;
+    g_scratch[dev].ptr = p;
+  }
+  *out = p;
   return PA_OK;
 }
 
@@ -67,16 +112,17 @@ extern "C" int pa_decode_static_scratch(void* out, const void* q, const void* k_
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
   if (num_seqs < 0) return PA_ERR_SHAPE;
   const size_t need =
-      pa_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size);
+      num_seqs > 0 ? pa_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size)
+                   : 0;
   if (need == 0) {
-    // invalid sizes: let the shared checks name the error (they return before any launch)
+    // an empty batch or invalid sizes: pa_decode's own checks decide, and
+    // they return before any launch and before the workspace is looked at
     static unsigned char dummy[256];
     return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                              num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                              scale, dummy, 0, dev_status, stream);
   }
   if (need > PA_STATIC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
-  if (num_seqs == 0) return PA_OK;
   void* ws = nullptr;
   int rc = pa::scratch_for_current_device(&ws);
   if (rc != PA_OK) return rc;

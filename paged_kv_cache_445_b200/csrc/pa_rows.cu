@@ -1184,20 +1184,21 @@ static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUt
   using S = RowsShape<D, NT, F8, TK>;
   const int smem = ROWS_WARPS * R * S::STAGE_BYTES + 1024 + (ROWS_SMEM_SEQS + 1) * 8;
   auto kern = rows_kernel<D, NT, R, F8, TK>;
-  static int configured_dev = -1;
-  static int blocks_per_sm = 1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  if (configured_dev != dev) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return PA_ERR_CUDA;
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, ROWS_THREADS, smem) != cudaSuccess || nb < 1)
-      return PA_ERR_CUDA;
-    constexpr int cap = rows_ctas_per_sm<D, NT, F8, TK>();
-    blocks_per_sm = nb > cap ? cap : nb;
-    configured_dev = dev;
-  }
+  static PerDevice configured;  // CTAs per SM on each device
+  int blocks_per_sm = 0;
+  const int rc_setup = per_device(
+      configured,
+      [&](int) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+          return static_cast<int>(PA_ERR_CUDA);
+        int nb = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, ROWS_THREADS, smem) != cudaSuccess || nb < 1)
+          return static_cast<int>(PA_ERR_CUDA);
+        constexpr int cap = rows_ctas_per_sm<D, NT, F8, TK>();
+        return nb > cap ? cap : nb;
+      },
+      &blocks_per_sm);
+  if (rc_setup != PA_OK) return rc_setup;
   RowsParams p = p0;
   p.tile_shift = TK == 32 ? 5 : 4;
   const int grid = num_sms * blocks_per_sm;

@@ -858,14 +858,16 @@ static int launch_verify_t(const VerifyParams& p0, const CUtensorMap& tq, const 
                            const CUtensorMap& tv, cudaStream_t stream, int num_sms) {
   auto kern = verify_kernel<NCOL>;
   const int smem = VfLayout<NCOL>::BYTES + 1024;
-  static int configured_dev = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-  if (configured_dev != dev) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return PA_ERR_CUDA;
-    configured_dev = dev;
-  }
+  static PerDevice configured;
+  int done = 0;
+  const int rc_setup = per_device(
+      configured,
+      [&](int) {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1
+                                                                                                           : PA_ERR_CUDA;
+      },
+      &done);
+  if (rc_setup != PA_OK) return rc_setup;
   VerifyParams p = p0;
   p.ncol_lo = NCOL == 32 ? 0 : 32;
   p.ncol_hi = NCOL;

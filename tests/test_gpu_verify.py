@@ -128,10 +128,5 @@ def test_batches_past_the_multi_row_kernels_sequence_limit_run_on_the_chunk_kern
     ds = DeviceStep(w)
     got = ds.step()
     kc, vc = oracle_after_append(w)
-    rows = sorted({0, 1, 599, *rng.integers(0, 600, 20).tolist()})
-    only = np.array([(t, h) for s in rows for t in range(int(w.query_start[s]), int(w.query_start[s + 1]))
-                     for h in range(w.num_q_heads)])
-    ref = _ref(w, kc, vc, only=only)
-    idx = tuple(only.T)
-    compare(got[idx], ref[idx], "600 sequences")
+    compare(got, _ref(w, kc, vc), "600 sequences, every row")
     assert int(ds.status.item()) == 0

@@ -134,6 +134,12 @@ def test_every_entry_point_rejects_bad_arguments_before_touching_a_device():
     assert L.pa_decode_static_scratch(f, f, f, f, f, 4, f, 4, 8, 2, 96, 16, 10, 0.1, None,
                                       None) == b.PA_ERR_UNSUPPORTED
     assert L.pa_decode_static_scratch(None, f, f, f, f, 4, f, 4, 8, 2, 128, 16, 10, 0.1, None, None) == b.PA_ERR_NULL
+    # an empty batch gets pa_decode's answer, errors included
+    for nb, hq, d in ((10, 8, 128), (0, 8, 128), (10, 6, 128), (10, 8, 96)):
+        want = L.pa_decode(f, f, f, f, f, 4, f, 0, hq, 2, d, 16, nb, 0.1, f, 1 << 20, None, None)
+        got = L.pa_decode_static_scratch(f, f, f, f, f, 4, f, 0, hq, 2, d, 16, nb, 0.1, None, None)
+        assert got == want, (nb, hq, d, got, want)
+    assert L.pa_decode_static_scratch(f, f, f, f, f, 4, f, 0, 8, 2, 128, 16, 0, 0.1, None, None) == b.PA_ERR_SHAPE
 
 
 def test_oracle_and_product_share_no_code():
