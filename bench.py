@@ -232,6 +232,18 @@ def step_launches(w, chunk_head_dims=(128,), chunk_groups=(1, 2, 4, 8, 16), veri
     return n
 
 
+def plan_launches(words) -> int:
+    """Kernel launches of a planned pa_prefill_chunk_planned call: one per
+    kernel that has work (the plan's flags: 32- and 64-column verification,
+    chunk, rows)."""
+    return bin(words[1] & 15).count("1")
+
+
+def plan_split(words):
+    """SMs of the decode rows beside the chunk kernel (0: one after the other)."""
+    return int(words[2])
+
+
 def verify_batch(w, max_cols=64, max_seqs=512) -> bool:
     """Every sequence of the batch has 2 .. max_cols/G query rows: the
     multi-row (verification) kernel does all the attention work."""
@@ -276,7 +288,7 @@ class GpuStep:
     fused launch (pa_decode_append) unless fused=False; a mixed batch runs
     pa_cache_append then pa_prefill_chunk."""
 
-    def __init__(self, w, device, fused=True, cascade=True, fp8=False):
+    def __init__(self, w, device, fused=True, cascade=True, fp8=False, plan=True):
         import torch
 
         import paged_kv_cache_445_b200 as pa
@@ -311,9 +323,18 @@ class GpuStep:
         else:
             self.workspace = pa.make_workspace(w.num_query_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim,
                                                w.block_tables.shape[1], w.block_size, device)
+        # a varlen batch: the host plan (made before timing from the host copies
+        # of query_start and context_lens, as a scheduler would) picks the
+        # kernels with work and how decode rows and chunk rows share the SMs
+        self.plan = None
+        if not self.decode and plan:
+            self.plan = pa.pa_plan_batch(w.query_start, w.context_lens, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                         w.block_size, w.block_tables.shape[1])
         # kernel launches per step
         if self.cascade:
             self.launches = 2 if self.fused else 3
+        elif self.plan is not None:
+            self.launches = 1 + plan_launches(list(self.plan.words))
         else:
             self.launches = 1 if self.fused else step_launches(w)
         # host-to-device inputs of one step (what e2e copies)
@@ -349,6 +370,10 @@ class GpuStep:
         elif self.decode:
             self.pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables, self.context_lens,
                               self.w.scale, self.workspace, self.status)
+        elif self.plan is not None:
+            self.pa.pa_prefill_chunk_planned(self.out, self.q, self.query_start, self.k_cache, self.v_cache,
+                                             self.block_tables, self.context_lens, self.w.scale, self.workspace,
+                                             self.plan, self.status)
         else:
             self.pa.pa_prefill_chunk(self.out, self.q, self.query_start, self.k_cache, self.v_cache,
                                      self.block_tables, self.context_lens, self.w.scale, self.workspace, self.status)
@@ -359,17 +384,18 @@ def workloads_fp8_caches(w):
     return workloads.fp8_caches(w, seed=445)
 
 
-def run_ours(args, peaks):
+def measure(args, peaks, workload, rank, world, local, *, cascade, fp8, plan=True, cpu_seconds=None):
+    """Time one workload's step (device events, then end to end through the
+    C ABI with host buffers) and return its JSON line as a dict."""
     import torch
 
     from paged_kv_cache_445_b200 import workloads
-    rank, world, local = dist_setup(args.gpus)
     device = torch.device("cuda", local)
     t0 = time.time()
-    w = workloads.standard(args.workload, seed=rank_seed(args.workload, rank))
+    w = workloads.standard(workload, seed=rank_seed(workload, rank))
     log(f"[rank {rank}] workload {w.name}: {w.num_seqs} seqs, {w.num_query_tokens} query rows, "
         f"{int(w.context_lens.sum())} keys, pool {w.num_blocks} blocks ({time.time() - t0:.1f}s to generate)")
-    g = GpuStep(w, device, fused=not args.separate_append, cascade=args.cascade, fp8=args.kv_dtype == "fp8")
+    g = GpuStep(w, device, fused=not args.separate_append, cascade=cascade, fp8=fp8, plan=plan)
     kv_bytes, attn_bytes, app_bytes, flops = step_bytes(w)
     if g.fp8:  # one byte per cached element instead of two; the appended rows are written as bytes too
         attn_bytes -= kv_bytes // 2
@@ -504,7 +530,7 @@ def run_ours(args, peaks):
     # ---- CPU baseline: the oracle on this host's cores, rank 0 at N = 1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_baseline(w, args.cpu_seconds, fp8=g.fp8)
+        cpu = oracle_baseline(w, args.cpu_seconds if cpu_seconds is None else cpu_seconds, fp8=g.fp8)
 
     clocks = sampler.summary()
     hbm, bf16_burst, bf16_sust, peak_src = peaks
@@ -536,6 +562,8 @@ def run_ours(args, peaks):
             "l2": l2_note(flush, kv_bytes, unique_kv),
             "parallelism": f"dp{world} (independent batch per GPU)",
             "cuda_graph": graph is not None,
+            "host_plan": None if g.plan is None else {"launches": plan_launches(list(g.plan.words)),
+                                                       "decode_sms": plan_split(list(g.plan.words))},
         },
         "seq_steps_per_s": round(total_seqs / (ms_step * 1e-3), 1),
         "frac_of_hbm_peak": round(compose_value(total_kv, ms_step) / hbm / world, 4),
@@ -544,7 +572,11 @@ def run_ours(args, peaks):
             "kernel": ("pa_rows_kernel, FP8 E4M3 cache (append + attention, one launch)" if g.fp8 else
                        "pa_verify_kernel (timed as the whole pa_prefill_chunk call: its launches of the "
                        "chunk and rows kernels find no work)" if verify else
-                       "pa_prefill_chunk call (chunk kernel + rows kernel)" if not w.is_decode else
+                       ("pa_prefill_chunk_planned call: decode rows (rows kernel, %d SMs) beside the tcgen05 "
+                        "chunk kernel (the other SMs)" % plan_split(list(g.plan.words))
+                        if g.plan is not None and plan_split(list(g.plan.words)) > 0 else
+                        "pa_prefill_chunk call (chunk kernel + rows kernel, one after the other)")
+                       if not w.is_decode else
                        "pa_cascade_kernel + pa_rows_kernel (shared prefixes once, then the private keys)"
                        if g.cascade else
                        "pa_rows_kernel (append + attention, one launch)" if g.fused else "pa_rows_kernel (attention)"),
@@ -570,11 +602,45 @@ def run_ours(args, peaks):
     if not w.is_decode:
         line["roofline_tensor"] = {"flops_per_step": flops, "achieved_tflops": round(flops / (attn_avg_ms * 1e-3) / 1e12, 1),
                                    "peak": bf16_sust, "unit": "TFLOP/s"}
+        # both kernels at once: the step cannot beat the slower of the two rooflines
+        bound_ms = max(kv_bytes / (hbm * 1e9), flops / (bf16_burst * 1e12)) * 1e3
+        line["overlap_bound"] = {"ms": round(bound_ms, 5), "frac": round(bound_ms / attn_avg_ms, 4),
+                                 "what": "max(decode KV bytes / measured HBM, chunk FLOPs / measured bf16 burst) "
+                                         "over the timed call"}
+    del g
+    torch.cuda.empty_cache()
+    return line
+
+
+SUB_RECORDS = [  # (key, workload, cascade, fp8): the other workloads of the default run, at N = 1
+    ("grpo-shared-prefix", 4, False, False),
+    ("grpo-shared-prefix-cascade", 4, True, False),
+    ("mixed-chunk-decode", 5, False, False),
+    ("llama3.3-70b-layer-decode-b128-fp8", 3, False, True),
+]
+
+
+def run_ours(args, peaks):
+    rank, world, local = dist_setup(args.gpus)
+    line = measure(args, peaks, args.workload, rank, world, local, cascade=args.cascade,
+                   fp8=args.kv_dtype == "fp8", plan=not args.no_plan)
+    if world == 1 and not args.no_sub_records and args.workload == 3 and args.kv_dtype == "bf16" \
+            and not args.cascade and not args.graph:
+        # the other workloads, each with its own roofline, clocks and short CPU baseline
+        subs = {}
+        for key, wl, casc, f8 in SUB_RECORDS:
+            sub = measure(args, peaks, wl, rank, world, local, cascade=casc, fp8=f8, cpu_seconds=args.sub_cpu_seconds)
+            for k in ("metric", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "vs_baseline", "data"):
+                sub.pop(k, None)
+            subs[key] = sub
+        line["workloads"] = subs
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
 
 
 # --------------------------------------------------------------------- oracle
@@ -703,6 +769,13 @@ def main(argv=None):
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix batches: pa_decode_cascade (each shared prefix read once per group) "
                          "instead of plain decode")
+    ap.add_argument("--no-plan", action="store_true",
+                    help="varlen batches: pa_prefill_chunk without the host plan (every kernel launched, one after "
+                         "the other on the whole GPU)")
+    ap.add_argument("--no-sub-records", action="store_true",
+                    help="the default run: leave out the other workloads' records (GRPO plain and cascade, mixed, FP8)")
+    ap.add_argument("--sub-cpu-seconds", type=float, default=4.0,
+                    help="oracle seconds of each sub-record's CPU baseline")
     ap.add_argument("--separate-append", action="store_true",
                     help="decode batches: pa_cache_append + pa_decode instead of the fused pa_decode_append")
     args = ap.parse_args(argv)

@@ -95,6 +95,11 @@ PA_API int pa_cache_append(const void* k_new, const void* v_new, void* k_cache, 
  * tables are `max_blocks_per_seq` wide, on the CURRENT device (the figure
  * depends on its SM count).  Returns 0 for invalid sizes.
  *
+ * It covers every call the batch may take: at head_dim 128 with a group the
+ * tcgen05 kernels support it includes the prefill chunk kernel's piece area
+ * (two slots of 256 rows x 132 floats per SM, about 40 MB on a 148-SM GPU),
+ * which decode calls do not use.
+ *
  * Workspace contract: the caller allocates it and ZERO-FILLS it once before
  * its first use; it may then reuse it for any later call on the same stream.
  * The library keeps its counters in it and every call that returns PA_OK and
@@ -254,6 +259,46 @@ PA_API int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start
                      void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
 
 /*
+ * pa_plan_batch / pa_prefill_chunk_planned -- pa_prefill_chunk with a plan
+ * made on the host from host copies of query_start and context_lens (the
+ * scheduler that builds a batch has them before it copies them to the
+ * device).  The plan records which of the call's kernels have work, so that
+ * only those are launched, and, for a batch that mixes decode rows with
+ * prefill chunks ("vLLM serving internals", "Chunked prefill protects the
+ * TTFT tail" and "What the scheduler looks like": the scheduler's one batch
+ * per step), how the GPU's SMs are shared: the decode rows, bound by HBM,
+ * stream on some SMs while the tcgen05 chunk kernel, bound by the tensor
+ * cores, computes on the others, both at once.  Results equal
+ * pa_prefill_chunk's up to rounding (the same definition; a chunk item cut
+ * between SMs is merged from its pieces).
+ *
+ * pa_plan_batch: query_start [num_seqs + 1] and context_lens [num_seqs] are
+ * HOST arrays (int32) with the values the device arrays will hold; the other
+ * sizes are those of the pa_prefill_chunk call.  Make the plan with the
+ * device current that will run the call (it records its SM count).  Returns
+ * PA_ERR_NULL / PA_ERR_SHAPE / PA_ERR_UNSUPPORTED for bad arguments.
+ *
+ * pa_prefill_chunk_planned: the arguments of pa_prefill_chunk plus the plan.
+ * A plan whose batch shape (num_seqs, total_q_tokens, group, head_dim) or SM
+ * count differs from the call's is rejected with PA_ERR_SHAPE.  A plan that
+ * does not match the device arrays' values leaves rows unwritten or
+ * misassigned: the caller keeps the two in step.  Workspace as for
+ * pa_prefill_chunk.
+ */
+#define PA_PLAN_WORDS 16
+typedef struct pa_plan {
+  int32_t words[PA_PLAN_WORDS];
+} pa_plan;
+PA_API int pa_plan_batch(const int32_t* query_start, const int32_t* context_lens, int num_seqs, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, pa_plan* plan);
+PA_API int pa_prefill_chunk_planned(void* out, const void* q, const int32_t* query_start, const void* k_cache,
+                                    const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                                    const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
+                                    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                                    void* workspace, size_t workspace_bytes, const pa_plan* plan, int* dev_status,
+                                    void* stream);
+
+/*
  * pa_decode_static_scratch -- pa_decode without a caller workspace.  Same
  * arguments, layouts, result and errors as pa_decode, minus `workspace` and
  * `workspace_bytes`.  The sources this library follows describe no such call:
@@ -263,10 +308,11 @@ PA_API int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start
  *
  * Scratch: a library-owned device array of PA_STATIC_SCRATCH_BYTES per device
  * (64 MiB), part of the library's device image, so this call allocates
- * nothing.  A batch whose pa_workspace_bytes(num_seqs, ...) exceeds that size
- * is rejected with PA_ERR_WORKSPACE before any launch (for example, 8 query
- * heads per KV head at head_dim 128 on a 148-SM B200 fits about 1,570
- * sequences with 512-block tables).
+ * nothing.  A batch whose decode workspace (the part of pa_workspace_bytes a
+ * decode call uses; pa_workspace_bytes also counts the prefill kernels'
+ * part) exceeds that size is rejected with PA_ERR_WORKSPACE before any
+ * launch (for example, 8 query heads per KV head at head_dim 128 on a 148-SM
+ * B200 fits about 1,570 sequences with 512-block tables).
  *
  * Sharing: every call on a device uses the same array.  Calls that overlap in
  * time on one device (other streams, other host threads) race on it and give
@@ -293,6 +339,18 @@ PA_API int pa_decode_static_scratch(void* out, const void* q, const void* k_cach
 
 /* Human-readable name of a pa_status value (static storage). */
 PA_API const char* pa_status_string(int status);
+
+/*
+ * The CUDA failure behind the last PA_ERR_CUDA returned on the calling host
+ * thread: pa_last_cuda_error() gives its cudaError_t (or, for the driver's
+ * tensor-map encoder, CUresult) value, 0 if no call on this thread failed;
+ * pa_last_cuda_error_string() names the failing call and the error
+ * (thread-local storage, "" if none).  A launch that reports an error left by
+ * an earlier kernel that faulted (a sticky error such as an illegal address)
+ * names that error.  Not part of the pages' problem statement: diagnostics.
+ */
+PA_API int pa_last_cuda_error(void);
+PA_API const char* pa_last_cuda_error_string(void);
 
 #ifdef __cplusplus
 }

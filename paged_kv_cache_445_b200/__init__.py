@@ -13,7 +13,8 @@ __all__ = [
     "pa_cache_append", "pa_decode", "pa_decode_append", "pa_cache_append_fp8", "pa_decode_fp8",
     "pa_decode_cascade", "pa_cascade_workspace_bytes",
     "make_cascade_workspace", "pa_prefill_chunk", "pa_workspace_bytes", "pa_decode_static_scratch",
-    "pa_status_string", "PAError", "library_path", "make_workspace", "status_bit",
+    "pa_status_string", "pa_last_cuda_error", "pa_last_cuda_error_string", "PAError", "library_path",
+    "make_workspace", "status_bit", "pa_plan_batch", "pa_prefill_chunk_planned", "Plan",
 ]
 
 

@@ -49,6 +49,23 @@ _lib.pa_decode_static_scratch.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p,
 _lib.pa_decode_static_scratch.restype = _ci
 _lib.pa_status_string.argtypes = [_ci]
 _lib.pa_status_string.restype = ctypes.c_char_p
+PLAN_WORDS = 16  # PA_PLAN_WORDS of include/pa.h
+
+
+class Plan(ctypes.Structure):
+    """pa_plan: the host plan of a varlen batch (opaque words)."""
+    _fields_ = [("words", ctypes.c_int32 * PLAN_WORDS)]
+
+
+_lib.pa_plan_batch.argtypes = [_vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, ctypes.POINTER(Plan)]
+_lib.pa_plan_batch.restype = _ci
+_lib.pa_prefill_chunk_planned.argtypes = [_vp, _vp, _i32p, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
+                                          _ci, ctypes.c_float, _vp, ctypes.c_size_t, ctypes.POINTER(Plan), _vp, _vp]
+_lib.pa_prefill_chunk_planned.restype = _ci
+_lib.pa_last_cuda_error.argtypes = []
+_lib.pa_last_cuda_error.restype = _ci
+_lib.pa_last_cuda_error_string.argtypes = []
+_lib.pa_last_cuda_error_string.restype = ctypes.c_char_p
 
 PA_OK = 0
 PA_ERR_NULL, PA_ERR_SHAPE, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE = -1, -2, -3, -4
@@ -72,9 +89,18 @@ def pa_status_string(code: int) -> str:
     return _lib.pa_status_string(int(code)).decode()
 
 
+def pa_last_cuda_error() -> int:
+    """cudaError_t (or CUresult) behind the last PA_ERR_CUDA on this thread; 0 if none."""
+    return int(_lib.pa_last_cuda_error())
+
+
+def pa_last_cuda_error_string() -> str:
+    return _lib.pa_last_cuda_error_string().decode()
+
+
 def _check(rc: int) -> None:
     if rc != PA_OK:
-        raise PAError(rc)
+        raise PAError(rc, pa_last_cuda_error_string() if rc == PA_ERR_CUDA else None)
 
 
 def _dev(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int | None = None) -> int:
@@ -277,6 +303,49 @@ def pa_prefill_chunk(out, q, query_start, k_cache, v_cache, block_tables, contex
                                  _status_ptr(dev_status), _stream_ptr(stream)))
 
 
+def _host_i32(a, name):
+    import numpy as np
+    if isinstance(a, torch.Tensor):
+        if a.is_cuda:
+            raise ValueError(f"{name} must be a host array (the plan is made on the host)")
+        a = a.numpy()
+    a = np.ascontiguousarray(a, dtype=np.int32)
+    if a.ndim != 1:
+        raise ValueError(f"{name} must be one-dimensional")
+    return a
+
+
+def pa_plan_batch(query_start, context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
+                  max_blocks_per_seq: int) -> Plan:
+    """Host plan of a varlen batch from HOST copies of query_start [B + 1] and
+    context_lens [B]: which kernels have work, and how decode rows and
+    prefill chunks share the SMs.  Make it with the device current that runs
+    the call."""
+    qs = _host_i32(query_start, "query_start")
+    cl = _host_i32(context_lens, "context_lens")
+    if qs.shape[0] != cl.shape[0] + 1:
+        raise ValueError("query_start must have num_seqs + 1 entries")
+    plan = Plan()
+    _check(_lib.pa_plan_batch(qs.ctypes.data, cl.ctypes.data, cl.shape[0], num_q_heads, num_kv_heads, head_dim,
+                              block_size, max_blocks_per_seq, ctypes.byref(plan)))
+    return plan
+
+
+def pa_prefill_chunk_planned(out, q, query_start, k_cache, v_cache, block_tables, context_lens, scale, workspace,
+                             plan: Plan, dev_status=None, stream=None) -> None:
+    """pa_prefill_chunk with a plan from pa_plan_batch (made for this batch)."""
+    op, qp, kc, vc, bt, cl, ws = _attention_args(out, q, k_cache, v_cache, block_tables, context_lens, workspace)
+    qs = _dev(query_start, "query_start", torch.int32, 1)
+    if query_start.shape[0] != context_lens.shape[0] + 1:
+        raise ValueError("query_start must have num_seqs + 1 entries")
+    if not isinstance(plan, Plan):
+        raise TypeError("plan must come from pa_plan_batch")
+    nb, hkv, bs, d = k_cache.shape
+    _check(_lib.pa_prefill_chunk_planned(op, qp, qs, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0],
+                                         q.shape[0], q.shape[1], hkv, d, bs, nb, float(scale), ws, workspace.numel(),
+                                         ctypes.byref(plan), _status_ptr(dev_status), _stream_ptr(stream)))
+
+
 def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale, dev_status=None,
                              stream=None) -> None:
     """pa_decode without a workspace argument, for callers that cannot allocate
@@ -301,13 +370,13 @@ def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_len
                                        q.shape[1], hkv, d, bs, nb, float(scale), _status_ptr(dev_status),
                                        _stream_ptr(stream))
     if rc == PA_ERR_WORKSPACE:
-        need = int(_lib.pa_workspace_bytes(context_lens.shape[0], q.shape[1], hkv, d, block_tables.shape[1], bs))
-        raise PAError(rc, f"this batch needs {need} bytes of scratch, more than the {STATIC_SCRATCH_BYTES}-byte "
-                          "static array: use pa_decode with a workspace")
+        raise PAError(rc, f"this batch needs more scratch than the {STATIC_SCRATCH_BYTES}-byte static array: "
+                          "use pa_decode with a workspace")
     _check(rc)
 
 
 def exported_symbols() -> list[str]:
     return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_decode_append", "pa_cache_append_fp8",
             "pa_decode_fp8", "pa_cascade_workspace_bytes", "pa_decode_cascade", "pa_prefill_chunk",
-            "pa_decode_static_scratch", "pa_status_string"]
+            "pa_decode_static_scratch", "pa_status_string", "pa_last_cuda_error", "pa_last_cuda_error_string",
+            "pa_plan_batch", "pa_prefill_chunk_planned"]

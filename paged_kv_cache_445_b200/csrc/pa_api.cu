@@ -4,11 +4,30 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdio>
 #include <mutex>
 
 #include "pa_internal.h"
 
 namespace pa {
+
+namespace {
+thread_local int t_cuda_error = 0;
+thread_local char t_cuda_error_text[192] = "";
+}  // namespace
+
+int cuda_fail(cudaError_t e, const char* call) {
+  t_cuda_error = static_cast<int>(e);
+  snprintf(t_cuda_error_text, sizeof t_cuda_error_text, "%s: %s (%s)", call, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return PA_ERR_CUDA;
+}
+
+int cu_fail(CUresult r, const char* call) {
+  t_cuda_error = static_cast<int>(r);
+  snprintf(t_cuda_error_text, sizeof t_cuda_error_text, "%s: CUresult %d", call, static_cast<int>(r));
+  return PA_ERR_CUDA;
+}
 
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -31,14 +50,48 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 
 }  // namespace
 
+namespace {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+}  // namespace
+
+// A host thread that has made no CUDA runtime call yet has no current
+// context, and the driver's tensor-map encoder then fails.  Make the current
+// device's primary context current in that case (cudaSetDevice does so); a
+// context the caller made current itself is left alone.
+int ensure_context(int dev) {
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (get && get(&ctx) == CUDA_SUCCESS && ctx != nullptr) return PA_OK;
+  const cudaError_t e = cudaSetDevice(dev);
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "cudaSetDevice");
+}
+
 int device_info(DeviceInfo* info) {
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const int rc = ensure_context(dev);
+  if (rc != PA_OK) return rc;
   static PerDevice sms;
   return per_device(
       sms,
       [](int dev) {
         int n = 0;
-        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n
-                                                                                                       : PA_ERR_CUDA;
+        const cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        return n > 0 ? n : static_cast<int>(PA_ERR_CUDA);
       },
       &info->num_sms);
 }
@@ -61,7 +114,7 @@ int encode_kv_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(cache), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+  return r == CUDA_SUCCESS ? PA_OK : cu_fail(r, "cuTensorMapEncodeTiled");
 }
 
 // FP8 cache [num_blocks, Hkv, block_size, D] bytes viewed as (128, block_size,
@@ -81,7 +134,7 @@ static int encode_kv_tmap_fp8(CUtensorMap* map, const void* cache, int num_block
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(cache), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+  return r == CUDA_SUCCESS ? PA_OK : cu_fail(r, "cuTensorMapEncodeTiled");
 }
 
 static int check_attention_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
@@ -100,13 +153,24 @@ static size_t workspace_needed(int num_query_tokens, int num_q_heads, int num_kv
   return rows_workspace_bytes(num_query_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, num_sms);
 }
 
+// Multi-row sequences of a batch of num_query_tokens rows: at most half of them.
+static int multirow_seq_bound(int num_query_tokens) { return num_query_tokens / 2 + 1; }
+
+// The chunk kernel's piece area, for varlen batches on the tcgen05 path.
+static size_t chunk_part(int num_query_tokens, int num_q_heads, int num_kv_heads, int head_dim, int num_sms) {
+  const int group = num_q_heads / num_kv_heads;
+  if (!chunk_supported(group, head_dim)) return 0;
+  return chunk_workspace_bytes(num_query_tokens, multirow_seq_bound(num_query_tokens), num_kv_heads, group, num_sms);
+}
+
 int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache,
                          const void* v_cache, const int32_t* block_tables, int max_blocks,
                          const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
                          int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
                          void* workspace, size_t workspace_bytes, int* dev_status, void* stream,
                          const void* k_new, const void* v_new, const int32_t* group_start,
-                         const int32_t* group_prefix, int num_groups, int kv_fp8, float k_scale, float v_scale) {
+                         const int32_t* group_prefix, int num_groups, int kv_fp8, float k_scale, float v_scale,
+                         const int32_t* plan) {
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace) return PA_ERR_NULL;
   if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
   if (k_new && query_start) return PA_ERR_UNSUPPORTED;  // the fused append serves one-row (decode) batches
@@ -133,7 +197,16 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
     if (!cascade_supported(num_q_heads / num_kv_heads, head_dim)) return PA_ERR_UNSUPPORTED;
   }
   const size_t casc_bytes = num_groups > 0 ? cascade_partials_bytes(num_seqs, num_q_heads, head_dim) : 0;
-  if (workspace_bytes < rows_bytes + casc_bytes) return PA_ERR_WORKSPACE;
+  const bool chunk_path = query_start && !kv_fp8 && chunk_supported(num_q_heads / num_kv_heads, head_dim);
+  const size_t chunk_bytes =
+      chunk_path ? chunk_part(total_q_tokens, num_q_heads, num_kv_heads, head_dim, di.num_sms) : 0;
+  if (workspace_bytes < rows_bytes + casc_bytes + chunk_bytes) return PA_ERR_WORKSPACE;
+  if (plan) {  // a plan made for this batch shape on a GPU of this size
+    if (plan[PLAN_MAGIC] != PLAN_MAGIC_VALUE || plan[PLAN_NUM_SEQS] != num_seqs ||
+        plan[PLAN_TOTAL_Q] != total_q_tokens || plan[PLAN_GROUP] != num_q_heads / num_kv_heads ||
+        plan[PLAN_HEAD_DIM] != head_dim || plan[PLAN_NUM_SMS] != di.num_sms)
+      return PA_ERR_SHAPE;
+  }
 
   CUtensorMap tmk, tmv;
   if (kv_fp8) {
@@ -197,12 +270,22 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
     c.status = dev_status;
     if ((rc = launch_cascade(c, q, k_cache, v_cache, total_q_tokens, head_dim, st, di.num_sms)) != PA_OK) return rc;
   }
-  if (query_start && !kv_fp8 && chunk_supported(p.group, head_dim)) {
+  if (chunk_path) {
     // sequences with 2 .. 64/G query rows run on the tcgen05 multi-row kernel,
     // longer ones on the tcgen05 chunk kernel, the single rows (decodes) on the
-    // rows kernel after both
+    // rows kernel.  Without a plan all three are launched (one that finds no
+    // work returns at once), one after another on the whole GPU.  With a plan
+    // only those with work are, and the decode rows may stream on part of the
+    // SMs while the chunk kernel computes on the rest.
     const bool verify = verify_supported(p.group, head_dim, num_seqs);
-    if (verify) {
+    int verify_which = verify ? 3 : 0, run_chunk = 1, run_rows = 1, decode_ctas = 0;
+    if (plan) {
+      verify_which = verify ? (plan[PLAN_FLAGS] & (PLAN_VERIFY32 | PLAN_VERIFY64)) : 0;
+      run_chunk = (plan[PLAN_FLAGS] & PLAN_CHUNK) != 0;
+      run_rows = (plan[PLAN_FLAGS] & PLAN_ROWS) != 0;
+      decode_ctas = plan[PLAN_DECODE_CTAS];
+    }
+    if (verify_which) {
       VerifyParams v{};
       v.out = out;
       v.block_tables = block_tables;
@@ -219,7 +302,8 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
       v.status = dev_status;
       v.slots = p.partials;
       v.counters = p.verify_counters;
-      if ((rc = launch_verify(v, q, k_cache, v_cache, total_q_tokens, st, di.num_sms)) != PA_OK) return rc;
+      if ((rc = launch_verify(v, q, k_cache, v_cache, total_q_tokens, st, di.num_sms, verify_which)) != PA_OK)
+        return rc;
     }
     ChunkParams c{};
     c.min_qlen = verify ? VERIFY_MAX_COLS / p.group + 1 : 2;
@@ -236,15 +320,133 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
     c.num_blocks = num_blocks;
     c.scale_log2 = p.scale_log2;
     c.status = dev_status;
-    if ((rc = launch_chunk(c, q, k_cache, v_cache, total_q_tokens, st, di.num_sms)) != PA_OK) return rc;
+    chunk_workspace_layout(static_cast<uint8_t*>(workspace) + rows_bytes, total_q_tokens,
+                           multirow_seq_bound(total_q_tokens), num_kv_heads, p.group, di.num_sms, &c);
     p.skip_multi = 1;
+    if (run_chunk && run_rows && decode_ctas > 0 && decode_ctas < di.num_sms) {
+      // the decode rows first, on decode_ctas SMs; they release the chunk
+      // kernel, which takes the other SMs and finishes after them
+      p.trigger_early = 1;
+      if ((rc = launch_rows(p, tmk, tmv, head_dim, st, di.num_sms, decode_ctas)) != PA_OK) return rc;
+      c.dep_at_end = 1;
+      return launch_chunk(c, q, k_cache, v_cache, total_q_tokens, st, di.num_sms, di.num_sms - decode_ctas);
+    }
+    if (run_chunk && (rc = launch_chunk(c, q, k_cache, v_cache, total_q_tokens, st, di.num_sms, di.num_sms)) != PA_OK)
+      return rc;
+    if (!run_rows) return PA_OK;
   }
   return launch_rows(p, tmk, tmv, head_dim, st, di.num_sms);
 }
 
+size_t decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                              int block_size) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads) return 0;
+  if (max_blocks_per_seq <= 0 || (block_size != 16 && block_size != 32)) return 0;
+  if (!rows_supported(num_q_heads / num_kv_heads, head_dim)) return 0;
+  DeviceInfo di;
+  if (device_info(&di) != PA_OK) return 0;
+  return (workspace_needed(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                           static_cast<long long>(max_blocks_per_seq) * block_size, di.num_sms) +
+          255) / 256 * 256;
+}
+
+namespace {
+// Per-SM rates of the kernels on a B200, used only to share the SMs between
+// the decode rows and the chunk rows of one batch (measured: an 8-warp decode
+// CTA streams about 150 GB/s of KV when few SMs load HBM, the decode rows of
+// a whole GPU about 6.2 TB/s, the tcgen05 chunk kernel about 6.5 TFLOP/s per
+// SM).  A split is used when its model time beats running the two kernels
+// one after the other on the whole GPU by 5 %.
+constexpr double DECODE_BYTES_PER_S_PER_SM = 150e9;
+constexpr double DECODE_BYTES_PER_S_ALL = 6.2e12;
+constexpr double CHUNK_FLOPS_PER_S_PER_SM = 6.5e12;
+
+int plan_split(double decode_bytes, double chunk_flops, int num_sms) {
+  const double serial = decode_bytes / DECODE_BYTES_PER_S_ALL + chunk_flops / (num_sms * CHUNK_FLOPS_PER_S_PER_SM);
+  double best = serial;
+  int best_n = 0;
+  for (int n = 1; n < num_sms; ++n) {
+    const double bw = n * DECODE_BYTES_PER_S_PER_SM < DECODE_BYTES_PER_S_ALL ? n * DECODE_BYTES_PER_S_PER_SM
+                                                                             : DECODE_BYTES_PER_S_ALL;
+    const double td = decode_bytes / bw, tc = chunk_flops / ((num_sms - n) * CHUNK_FLOPS_PER_S_PER_SM);
+    const double t = td > tc ? td : tc;
+    if (t < best) {
+      best = t;
+      best_n = n;
+    }
+  }
+  return best < 0.95 * serial ? best_n : 0;
+}
+}  // namespace
+
 }  // namespace pa
 
 extern "C" {
+
+int pa_plan_batch(const int32_t* query_start, const int32_t* context_lens, int num_seqs, int num_q_heads,
+                  int num_kv_heads, int head_dim, int block_size, int max_blocks_per_seq, pa_plan* plan) {
+  if (!query_start || !context_lens || !plan) return PA_ERR_NULL;
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_blocks_per_seq <= 0) return PA_ERR_SHAPE;
+  if (num_q_heads % num_kv_heads != 0) return PA_ERR_SHAPE;
+  if (block_size != 16 && block_size != 32) return PA_ERR_UNSUPPORTED;
+  const int group = num_q_heads / num_kv_heads;
+  if (!pa::rows_supported(group, head_dim)) return PA_ERR_UNSUPPORTED;
+  if (query_start[0] != 0) return PA_ERR_SHAPE;
+  pa::DeviceInfo di;
+  int rc = pa::device_info(&di);
+  if (rc != PA_OK) return rc;
+  const bool chunk = pa::chunk_supported(group, head_dim);
+  const bool verify = chunk && pa::verify_supported(group, head_dim, num_seqs);
+  const int min_qlen = verify ? pa::VERIFY_MAX_COLS / group + 1 : 2;
+  const long long cap = static_cast<long long>(max_blocks_per_seq) * block_size;
+  int32_t flags = 0;
+  double decode_bytes = 0.0, chunk_flops = 0.0;
+  for (int s = 0; s < num_seqs; ++s) {
+    const long long qlen = static_cast<long long>(query_start[s + 1]) - query_start[s];
+    if (qlen < 0) return PA_ERR_SHAPE;
+    long long ctx = context_lens[s] < 0 ? 0 : context_lens[s];
+    if (ctx > cap) ctx = cap;
+    if (qlen == 0) continue;
+    if (qlen > ctx) flags |= pa::PLAN_ROWS;  // rows with no key are written as zeros by the rows kernel
+    if (!chunk || qlen == 1) {
+      flags |= pa::PLAN_ROWS;
+      decode_bytes += static_cast<double>(ctx) * num_kv_heads * head_dim * 4.0 * static_cast<double>(qlen);
+    } else if (verify && qlen * group <= pa::VERIFY_MAX_COLS) {
+      flags |= qlen * group <= 32 ? pa::PLAN_VERIFY32 : pa::PLAN_VERIFY64;
+    } else if (qlen >= min_qlen) {
+      flags |= pa::PLAN_CHUNK;
+      // causal: row i sees ctx - qlen + i + 1 keys
+      const double first = static_cast<double>(ctx - qlen + 1);
+      const double keys = qlen * first + 0.5 * static_cast<double>(qlen) * static_cast<double>(qlen - 1);
+      chunk_flops += keys * num_q_heads * head_dim * 4.0;
+    }
+  }
+  int32_t* w = plan->words;
+  for (int i = 0; i < PA_PLAN_WORDS; ++i) w[i] = 0;
+  w[pa::PLAN_MAGIC] = pa::PLAN_MAGIC_VALUE;
+  w[pa::PLAN_FLAGS] = flags;
+  w[pa::PLAN_DECODE_CTAS] =
+      (flags & pa::PLAN_CHUNK) && (flags & pa::PLAN_ROWS) ? pa::plan_split(decode_bytes, chunk_flops, di.num_sms) : 0;
+  w[pa::PLAN_NUM_SMS] = di.num_sms;
+  w[pa::PLAN_NUM_SEQS] = num_seqs;
+  w[pa::PLAN_TOTAL_Q] = query_start[num_seqs];
+  w[pa::PLAN_GROUP] = group;
+  w[pa::PLAN_HEAD_DIM] = head_dim;
+  return PA_OK;
+}
+
+int pa_prefill_chunk_planned(void* out, const void* q, const int32_t* query_start, const void* k_cache,
+                             const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                             const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
+                             int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                             void* workspace, size_t workspace_bytes, const pa_plan* plan, int* dev_status,
+                             void* stream) {
+  if (!query_start || !plan) return PA_ERR_NULL;
+  return pa::run_attention(out, q, query_start, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                           num_seqs, total_q_tokens, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                           scale, workspace, workspace_bytes, dev_status, stream, nullptr, nullptr, nullptr, nullptr,
+                           0, 0, 1.f, 1.f, plan->words);
+}
 
 int pa_cache_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache, const int32_t* slot_mapping,
                     int num_tokens, int num_blocks, int num_kv_heads, int head_dim, int block_size, int* dev_status,
@@ -270,8 +472,10 @@ size_t pa_workspace_bytes(int num_query_tokens, int num_q_heads, int num_kv_head
   if (!pa::rows_supported(num_q_heads / num_kv_heads, head_dim)) return 0;
   pa::DeviceInfo di;
   if (pa::device_info(&di) != PA_OK) return 0;
-  return pa::workspace_needed(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
-                              static_cast<long long>(max_blocks_per_seq) * block_size, di.num_sms);
+  const size_t rows = (pa::workspace_needed(num_query_tokens, num_q_heads, num_kv_heads, head_dim,
+                                            static_cast<long long>(max_blocks_per_seq) * block_size, di.num_sms) +
+                       255) / 256 * 256;
+  return rows + pa::chunk_part(num_query_tokens, num_q_heads, num_kv_heads, head_dim, di.num_sms);
 }
 
 int pa_decode(void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -353,6 +557,10 @@ int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const
                            num_seqs, total_q_tokens, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                            scale, workspace, workspace_bytes, dev_status, stream);
 }
+
+int pa_last_cuda_error(void) { return pa::t_cuda_error; }
+
+const char* pa_last_cuda_error_string(void) { return pa::t_cuda_error_text; }
 
 const char* pa_status_string(int status) {
   switch (status) {

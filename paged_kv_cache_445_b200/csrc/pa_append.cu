@@ -93,7 +93,7 @@ int launch_append_fp8(const void* k_new, const void* v_new, void* k_cache, void*
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint2*>(k_cache),
       static_cast<uint2*>(v_cache), slot_mapping, num_tokens, num_kv_heads, vec_per_row, block_size,
       static_cast<long long>(num_blocks) * block_size, k_inv, v_inv, dev_status);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return check_launch(cudaSuccess, "append_kernel (fp8) launch");
 }
 
 int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_cache, const int32_t* slot_mapping,
@@ -123,7 +123,7 @@ int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_c
       static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), static_cast<uint4*>(k_cache),
       static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, vec_per_row, block_size,
       static_cast<long long>(num_blocks) * block_size, dev_status);
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return check_launch(cudaSuccess, "append_kernel launch");
 }
 
 }  // namespace pa

@@ -459,7 +459,7 @@ static int launch_cascade_t(const CascadeParams& p, const void* q, const void* k
     if (fn(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return PA_ERR_CUDA;
+      return cu_fail(CUDA_ERROR_INVALID_VALUE, "cuTensorMapEncodeTiled");
   }
   for (int which = 0; which < 2; ++which) {  // caches as (D, bs, Hkv, NB); box = 64 columns x 16 rows
     const cuuint64_t row = static_cast<cuuint64_t>(D) * 2;
@@ -471,7 +471,7 @@ static int launch_cascade_t(const CascadeParams& p, const void* q, const void* k
     if (fn(which ? &tv : &tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(which ? v_cache : k_cache),
            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return PA_ERR_CUDA;
+      return cu_fail(CUDA_ERROR_INVALID_VALUE, "cuTensorMapEncodeTiled");
   }
   auto kern = cascade_kernel<D>;
   const int smem = S::SMEM_TOTAL + 1024;
@@ -480,8 +480,8 @@ static int launch_cascade_t(const CascadeParams& p, const void* q, const void* k
   const int rc_setup = per_device(
       configured,
       [&](int) {
-        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1
-                                                                                                           : PA_ERR_CUDA;
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        return e == cudaSuccess ? 1 : cuda_fail(e, "cudaFuncSetAttribute");
       },
       &done);
   if (rc_setup != PA_OK) return rc_setup;
@@ -495,8 +495,7 @@ static int launch_cascade_t(const CascadeParams& p, const void* q, const void* k
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p) != cudaSuccess) return PA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return check_launch(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p), "cascade_kernel launch");
 }
 
 int launch_cascade(const CascadeParams& p, const void* q, const void* k_cache, const void* v_cache,

@@ -34,6 +34,17 @@
 //    maximum rises by more than 2^8 (between rescales the stale maximum is an
 //    exact reference point).  Key rows past the context are zeroed in V
 //    before P V.
+//  * Work split (stream-K): the batch's (item, 128-key tile) units, in item
+//    order, are cut into one equal contiguous range per CTA, so every CTA gets
+//    the same number of tiles whatever the item count.  An item cut by a range
+//    boundary leaves unnormalised (O, m, l) pieces, one per CTA that touched
+//    it, in that CTA's two piece slots; the CTA that lands the item's last
+//    piece (an atomic count per item, back to zero afterwards) merges them in
+//    CTA order and writes the rows.
+//  * Beside the decode kernel: launched after it on part of the GPU, the
+//    kernel takes the other SMs while the decode rows stream; it then waits
+//    for that grid at its end rather than its start (the decode kernel
+//    releases it only after the cache append before both has completed).
 //  * Every wait is bounded; on a timeout the CTA raises PA_ERR_TIMEOUT, stops
 //    all roles through a shared abort flag, drains its tensor-core work and
 //    frees its tensor memory.
@@ -63,6 +74,7 @@ constexpr int SMEM_TOTAL = SMEM_V + VST * KV_BYTES;           // 224 KB
 constexpr uint32_t TMEM_COLS = 512;                           // S_A, S_B, O_A, O_B: 128 columns each
 constexpr uint32_t TMEM_O = 256;                              // O of M-tile w at TMEM_O + 128 w
 constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when the max rises by > 2^8
+constexpr int SLOT_STRIDE = CH_D + 4;  // piece slot row: O[128], m, l, 2 floats of padding
 // Register split (setmaxnreg): the launch gives 168 per thread (65,536 / 384,
 // rounded down to 8); warpgroup 0 drops to 80, the softmax warpgroups rise to
 // 208: 128 x 80 + 256 x 208 = 63,488 <= 384 x 168 = 64,512, the launch's total
@@ -83,48 +95,24 @@ struct Shared {
   uint64_t k_full[KST], k_empty[KST], v_full[VST], v_empty[VST];
   uint32_t tmem_base;
   int abort;
-  long long total;
+  int merge;        // this CTA landed the last piece of the item being finished
+  int units;  // (item, key tile) units of the batch
 };
 
 }  // namespace
 
 // Items = (multi-row sequence, pair of token blocks, KV head), numbered
-// sequence by sequence; every CTA walks items blockIdx.x, + gridDim.x, ...
+// sequence by sequence, KV head fastest; an item's units are its key tiles.
 // The batch is scanned from global memory by each role (it is small and
 // L1-resident).
-__device__ __forceinline__ bool chunk_item(const ChunkParams& p, int pair_tok, long long idx, Item& it) {
-  long long base = 0;
-  for (int s = 0; s < p.num_seqs; ++s) {
-    const int q0 = __ldg(p.query_start + s), qlen = __ldg(p.query_start + s + 1) - q0;
-    if (qlen < p.min_qlen) continue;
-    int ctx = __ldg(p.context_lens + s);
-    const int cap = p.max_blocks * p.block_size;
-    if (ctx > cap) ctx = cap;
-    const int npair = (qlen + pair_tok - 1) / pair_tok;
-    const long long n = static_cast<long long>(npair) * p.num_kv_heads;
-    if (idx < base + n) {
-      const int r = static_cast<int>(idx - base);
-      it.s = s;
-      it.q0 = q0;
-      it.qlen = qlen;
-      it.ctx = ctx;
-      it.p0 = ctx - qlen;
-      it.tp = r / p.num_kv_heads;
-      it.kvh = r % p.num_kv_heads;
-      return true;
-    }
-    base += n;
-  }
-  return false;
-}
-
-__device__ __forceinline__ long long chunk_total(const ChunkParams& p, int pair_tok) {
-  long long n = 0;
-  for (int s = 0; s < p.num_seqs; ++s) {
-    const int qlen = __ldg(p.query_start + s + 1) - __ldg(p.query_start + s);
-    if (qlen >= p.min_qlen) n += static_cast<long long>((qlen + pair_tok - 1) / pair_tok) * p.num_kv_heads;
-  }
-  return n;
+__device__ __forceinline__ void fill_item(int s, int q0, int qlen, int ctx, int tp, Item& it) {
+  it.s = s;
+  it.q0 = q0;
+  it.qlen = qlen;
+  it.ctx = ctx;
+  it.p0 = ctx - qlen;
+  it.tp = tp;
+  it.kvh = 0;
 }
 
 // Key tiles an item needs: up to the last position of its pair's last row
@@ -133,6 +121,63 @@ __device__ __forceinline__ int item_tiles(const Item& it, int pair_tok) {
   int last = it.p0 + min((it.tp + 1) * pair_tok, it.qlen) - 1;
   if (last >= it.ctx) last = it.ctx - 1;
   return last < 0 ? 0 : last / CH_N + 1;
+}
+
+// Total units of the batch.
+__device__ __forceinline__ long long chunk_units(const ChunkParams& p, int pair_tok) {
+  long long n = 0;
+  const int cap = p.max_blocks * p.block_size;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int q0 = __ldg(p.query_start + s), qlen = __ldg(p.query_start + s + 1) - q0;
+    if (qlen < p.min_qlen) continue;
+    const int ctx = min(__ldg(p.context_lens + s), cap);
+    Item it;
+    for (int tp = 0; tp * pair_tok < qlen; ++tp) {
+      fill_item(s, q0, qlen, ctx, tp, it);
+      n += static_cast<long long>(item_tiles(it, pair_tok)) * p.num_kv_heads;
+    }
+  }
+  return n;
+}
+
+// The item that holds unit u: the item, its index (for its piece counter),
+// its first unit and its tile count.  False if u is past the last unit.
+__device__ __forceinline__ bool chunk_unit_item(const ChunkParams& p, int pair_tok, int u, Item& it, int& idx,
+                                                int& ubase, int& nt) {
+  int base = 0, item_base = 0;
+  const int cap = p.max_blocks * p.block_size;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int q0 = __ldg(p.query_start + s), qlen = __ldg(p.query_start + s + 1) - q0;
+    if (qlen < p.min_qlen) continue;
+    const int ctx = min(__ldg(p.context_lens + s), cap);
+    for (int tp = 0; tp * pair_tok < qlen; ++tp) {
+      fill_item(s, q0, qlen, ctx, tp, it);
+      const int n = item_tiles(it, pair_tok);
+      const int units = n * p.num_kv_heads;
+      if (u < base + units) {
+        const int kvh = (u - base) / n;
+        it.kvh = kvh;
+        idx = item_base + kvh;
+        ubase = base + kvh * n;
+        nt = n;
+        return true;
+      }
+      base += units;
+      item_base += p.num_kv_heads;
+    }
+  }
+  return false;
+}
+
+// First unit of CTA c's range, and the CTA whose range holds unit u.
+__device__ __forceinline__ int cta_range_start(int units, int c, int ncta) {
+  return static_cast<int>(static_cast<long long>(units) * c / ncta);
+}
+__device__ __forceinline__ int cta_of_unit(int units, int u, int ncta) {
+  int c = static_cast<int>(static_cast<long long>(u) * ncta / units);
+  while (c + 1 < ncta && cta_range_start(units, c + 1, ncta) <= u) ++c;
+  while (c > 0 && cta_range_start(units, c, ncta) > u) --c;
+  return c;
 }
 
 __device__ __forceinline__ bool ch_wait(Shared& sh, uint64_t* bar, uint32_t phase, int* status) {
@@ -181,7 +226,9 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       mbar_init(&sh.v_empty[b], 1);
     }
     sh.abort = 0;
-    sh.total = chunk_total(p, PAIR);
+    const long long u_all = chunk_units(p, PAIR);
+    if (u_all > 0x7fffffffLL) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));  // far beyond any real batch
+    sh.units = u_all > 0x7fffffffLL ? 0 : static_cast<int>(u_all);
     fence_mbar_init();
   }
   if (warp == 1) {  // tensor memory: S_A, S_B, O_A, O_B
@@ -194,9 +241,15 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
-  grid_dependency_wait();  // the cache may still be being appended by the kernel before this one
+  // the cache may still be being appended by the kernel before this one
+  // (beside the decode kernel: that kernel released this one after it had
+  // waited for the append itself, and this one waits for it at the end)
+  if (!p.dep_at_end) grid_dependency_wait();
 
-  const long long total = sh.total;
+  // this CTA's contiguous range [ua, ub) of the batch's (item, key tile) units
+  const int units = sh.units;
+  const int ncta = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+  const int ua = cta_range_start(units, cta, ncta), ub = cta_range_start(units, cta + 1, ncta);
   if (warp < 4) {
     // ================================================================ warpgroup 0
     regs_dec<REGS_PRODUCER>();
@@ -209,10 +262,14 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
     }
     const uint64_t pol = policy_evict_last();  // a chunk's K/V is re-read by every item of the chunk
     uint32_t items = 0, tcount = 0;  // tiles issued over all items (stage and phase bookkeeping)
-    for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x, ++items) {
+    for (int u = ua; u < ub && !sh.abort; ++items) {
       Item it;
-      if (!chunk_item(p, PAIR, idx, it)) break;
-      const int nt = item_tiles(it, PAIR);
+      int idx, ubase, nt;
+      if (!chunk_unit_item(p, PAIR, u, it, idx, ubase, nt)) break;
+      // this CTA's piece of the item: key tiles j0 .. j1 - 1
+      const int j0 = u - ubase;
+      const int j1 = ub - ubase < nt ? ub - ubase : nt;
+      u = ubase + j1;
       const int nblk_ctx = (it.ctx + p.block_size - 1) / p.block_size;
       const int32_t* table = p.block_tables + static_cast<long long>(it.s) * p.max_blocks;
       // lane b < 8 owns the b-th 16-key group of a tile: block id and row offset in the block
@@ -227,8 +284,8 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         }
       };
       int blk_cur, y_cur, blk_prev = -1, y_prev = 0, blk_next, y_next;
-      tile_ids(0, blk_cur, y_cur);
-      tile_ids(1, blk_next, y_next);
+      tile_ids(j0, blk_cur, y_cur);
+      tile_ids(j0 + 1, blk_next, y_next);
       // the previous item's last QK^T has read both Q tiles
       if (items > 0 && !ch_wait(sh, &sh.q_empty, (items - 1) & 1, p.status)) break;
       if (lane == 0) {
@@ -255,17 +312,19 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         return true;
       };
       bool ok = true;
-      for (int j = 0; ok && j < nt; ++j) {
-        ok = load_tile(&tmk, sh.k_full, sh.k_empty, KST, SMEM_K, tcount + j, blk_cur, y_cur);
-        if (ok && j > 0) ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + j - 1, blk_prev, y_prev);
+      for (int j = j0; ok && j < j1; ++j) {
+        ok = load_tile(&tmk, sh.k_full, sh.k_empty, KST, SMEM_K, tcount + (j - j0), blk_cur, y_cur);
+        if (ok && j > j0)
+          ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + (j - j0) - 1, blk_prev, y_prev);
         blk_prev = blk_cur;
         y_prev = y_cur;
         blk_cur = blk_next;
         y_cur = y_next;
         tile_ids(j + 2, blk_next, y_next);  // one tile of lead for the block-table reads
       }
-      if (ok && nt > 0) ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + nt - 1, blk_prev, y_prev);
-      tcount += nt;
+      if (ok && j1 > j0)
+        ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + (j1 - j0) - 1, blk_prev, y_prev);
+      tcount += j1 - j0;
       if (!ok) break;
     }
     if (sh.abort) {  // let this CTA's copies still in flight land before its shared memory goes away
@@ -287,10 +346,14 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
     uint32_t q_phase = 0, p_phase[2] = {0, 0}, o_phase = 0, kv_count = 0;
     uint32_t pv_commits[2] = {0, 0};  // completions committed to pv_done[w] so far
     bool first_item = true;
-    for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x) {
+    for (int u = ua; u < ub && !sh.abort;) {
       Item it;
-      if (!chunk_item(p, PAIR, idx, it)) break;
-      const int nt = item_tiles(it, PAIR);
+      int idx, ubase, nt;
+      if (!chunk_unit_item(p, PAIR, u, it, idx, ubase, nt)) break;
+      // this CTA's piece of the item: key tiles j0 .. j1 - 1
+      const int j0 = u - ubase;
+      const int j1 = ub - ubase < nt ? ub - ubase : nt;
+      u = ubase + j1;
       if (!ch_wait(sh, &sh.q_full, q_phase, p.status)) break;
       q_phase ^= 1;
       if (!first_item) {  // both epilogues of the previous item have read O
@@ -299,7 +362,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         o_phase ^= 1;
       }
       first_item = false;
-      if (nt == 0) {  // nothing to multiply: Q is free, and each epilogue gets its one P V completion
+      if (j1 <= j0) {  // nothing to multiply: Q is free, and each epilogue gets its one P V completion
         if (lane == 0) {
           umma_commit(&sh.q_empty);
           umma_commit(&sh.pv_done[0]);
@@ -314,9 +377,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       // P V_w(j - 1): wait until that MMA has completed before overwriting it
       // (for j = 0, the previous item's epilogue already waited for its last P V).
       auto qk = [&](int w, int j) -> bool {
-        const int stage = (kv_count + j) % KST;
-        if (w == 0 && !ch_wait(sh, &sh.k_full[stage], ((kv_count + j) / KST) & 1, p.status)) return false;
-        if (j > 0 && !ch_wait(sh, &sh.pv_done[w], (pv_commits[w] - 1) & 1, p.status)) return false;
+        const uint32_t t = kv_count + (j - j0);  // tiles this CTA has taken so far
+        const int stage = t % KST;
+        if (w == 0 && !ch_wait(sh, &sh.k_full[stage], (t / KST) & 1, p.status)) return false;
+        if (j > j0 && !ch_wait(sh, &sh.pv_done[w], (pv_commits[w] - 1) & 1, p.status)) return false;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sk = smem_u32(smem + SMEM_K + stage * KV_BYTES);
@@ -330,7 +394,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           umma_commit(&sh.s_full[w]);
           if (w == 1) {
             umma_commit(&sh.k_empty[stage]);
-            if (j == nt - 1) umma_commit(&sh.q_empty);
+            if (j == j1 - 1) umma_commit(&sh.q_empty);
           }
         }
         __syncwarp();
@@ -340,8 +404,9 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       auto pv = [&](int w, int j) -> bool {
         if (!ch_wait(sh, &sh.p_full[w], p_phase[w], p.status)) return false;
         p_phase[w] ^= 1;
-        const int stage = (kv_count + j) % VST;
-        if (w == 0 && !ch_wait(sh, &sh.v_full[stage], ((kv_count + j) / VST) & 1, p.status)) return false;
+        const uint32_t t = kv_count + (j - j0);
+        const int stage = t % VST;
+        if (w == 0 && !ch_wait(sh, &sh.v_full[stage], (t / VST) & 1, p.status)) return false;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t sv = smem_u32(smem + SMEM_V + stage * KV_BYTES);
@@ -349,7 +414,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < CH_N / 16; ++kk)  // keys 16kk.. = P columns 8kk..; V rows 16kk.., both panels
             umma_f16_ts(tmem + TMEM_O + w * CH_N, pt + 8 * kk, umma_desc(sv + kk * 16 * 128, PANEL, 1024),
-                        idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                        idesc_pv, (j > j0 || kk > 0) ? 1u : 0u);
           umma_commit(&sh.pv_done[w]);
           if (w == 1) umma_commit(&sh.v_empty[stage]);
         }
@@ -357,10 +422,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         ++pv_commits[w];
         return true;
       };
-      bool ok = qk(0, 0) && qk(1, 0);
-      for (int j = 1; ok && j < nt; ++j) ok = pv(0, j - 1) && qk(0, j) && pv(1, j - 1) && qk(1, j);
-      if (ok) ok = pv(0, nt - 1) && pv(1, nt - 1);
-      kv_count += nt;
+      bool ok = qk(0, j0) && qk(1, j0);
+      for (int j = j0 + 1; ok && j < j1; ++j) ok = pv(0, j - 1) && qk(0, j) && pv(1, j - 1) && qk(1, j);
+      if (ok) ok = pv(0, j1 - 1) && pv(1, j1 - 1);
+      kv_count += j1 - j0;
       if (!ok) break;
     }
     }
@@ -376,18 +441,33 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
     // kv_count: key tiles of earlier items (V stages); pv_count: completions
     // of pv_done[w] so far (one per tile, one for an item without tiles)
     uint32_t s_phase = 0, kv_count = 0, pv_count = 0;
-    for (long long idx = blockIdx.x; idx < total && !sh.abort; idx += gridDim.x) {
+    for (int u = ua; u < ub && !sh.abort;) {
       Item it;
-      if (!chunk_item(p, PAIR, idx, it)) break;
-      const int nt = item_tiles(it, PAIR);
+      int idx, ubase, nt;
+      if (!chunk_unit_item(p, PAIR, u, it, idx, ubase, nt)) break;
+      // this CTA's piece of the item: key tiles j0 .. j1 - 1
+      const int j0 = u - ubase;
+      const int j1 = ub - ubase < nt ? ub - ubase : nt;
+      u = ubase + j1;
       const int tok = it.tp * PAIR + w * TOK + tok_in_tile;  // row's token within the chunk
       const int last_key = it.p0 + tok;                       // causal limit (inclusive)
       const bool row_valid = tok < it.qlen && last_key >= 0;
       const int tile_last = it.p0 + it.tp * PAIR + w * TOK;   // first row of this M-tile: keys beyond it are
                                                               // masked for some row of the tile
+      // a cut item: the CTAs c_first .. c_last hold its pieces; c_first's is
+      // the last piece of its range (slot 1) unless its range starts with it
+      const bool whole = j0 == 0 && j1 == nt;
+      int c_first = 0, c_last = 0, first_slot = 0;
+      if (!whole) {
+        c_first = cta_of_unit(units, ubase, ncta);
+        c_last = cta_of_unit(units, ubase + nt - 1, ncta);
+        first_slot = cta_range_start(units, c_first, ncta) == ubase ? 0 : 1;
+      }
+      const int my_slot = (ubase + j0 == ua) ? 0 : 1;  // this CTA's first piece, or its last
+      int* const cnt = p.counters + static_cast<long long>(idx) * (2 * CH_M) + w * CH_M + row;
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int j = 0; j < nt && ok; ++j) {
+      for (int j = j0; j < j1 && ok; ++j) {
         if (!(ok = ch_wait(sh, &sh.s_full[w], s_phase, p.status))) break;
         s_phase ^= 1;
         tc_fence_after();
@@ -459,10 +539,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         // O holds tiles 0..j-1: wait for P V_w(j - 1), then scale O in tensor
         // memory.  tcgen05.ld/st are warp-collective, so the whole warp takes
         // this branch when any of its rows rescales (the others scale by 1).
-        if (j > 0 && __any_sync(FULL_MASK, resc)) {
+        if (j > j0 && __any_sync(FULL_MASK, resc)) {
           // pv_done[w] completes once per tile; P V_w(j) cannot have completed
           // (it waits for this thread's P), so the parity names the phase
-          if (!(ok = ch_wait(sh, &sh.pv_done[w], (pv_count + j - 1) & 1, p.status))) break;
+          if (!(ok = ch_wait(sh, &sh.pv_done[w], (pv_count + (j - j0) - 1) & 1, p.status))) break;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < CH_D / 32; ++c) {
@@ -479,8 +559,9 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         // (M-tile A's warpgroup does it; P V_B(j) is issued after P V_A(j))
         const int valid_keys = it.ctx - key0;
         if (w == 0 && valid_keys < CH_N) {
-          const int stage = (kv_count + j) % VST;
-          if (!(ok = ch_wait(sh, &sh.v_full[stage], ((kv_count + j) / VST) & 1, p.status))) break;
+          const uint32_t t = kv_count + (j - j0);
+          const int stage = t % VST;
+          if (!(ok = ch_wait(sh, &sh.v_full[stage], (t / VST) & 1, p.status))) break;
           uint8_t* vst = smem + SMEM_V + stage * KV_BYTES;
           const int nz = (CH_N - max(valid_keys, 0)) * 2 * 8;  // 16-byte chunks in both panels
           for (int k = threadIdx.x - 128; k < nz; k += 128) {
@@ -492,41 +573,111 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         tc_fence_before();
         mbar_arrive(&sh.p_full[w]);
       }
-      kv_count += nt;
-      pv_count += nt > 0 ? nt : 1;
+      kv_count += j1 - j0;
+      pv_count += j1 > j0 ? j1 - j0 : 1;
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> out (after the item's last pv_done completion)
       if (!ch_wait(sh, &sh.pv_done[w], (pv_count - 1) & 1, p.status)) break;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
                             (static_cast<long long>(it.q0 + tok) * p.num_q_heads + it.kvh * G + head_in_group) * CH_D;
+      if (whole) {  // the whole item: O / l -> bf16 -> out
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int c = 0; c < CH_D / 32; ++c) {
+          float v[32];
+          if (nt > 0) {
+            tmem_ld32(o_col + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+          if (row_valid) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              uint4 u4;
+              u4.x = pack_bf16x2(v[i] * inv, v[i + 1] * inv);
+              u4.y = pack_bf16x2(v[i + 2] * inv, v[i + 3] * inv);
+              u4.z = pack_bf16x2(v[i + 4] * inv, v[i + 5] * inv);
+              u4.w = pack_bf16x2(v[i + 6] * inv, v[i + 7] * inv);
+              *reinterpret_cast<uint4*>(orow + c * 32 + i) = u4;
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sh.o_empty[w]);
+        continue;
+      }
+      // ---- a piece of a cut item: the unnormalised (O, m, l) of this row go
+      // to this CTA's slot (0: the first piece of its range, 1: the last)
+      const int wrow = w * CH_M + row;  // row of the item (both M-tiles)
+      float* dst = p.partials + ((static_cast<long long>(cta) * 2 + my_slot) * 2 * CH_M + wrow) * SLOT_STRIDE;
 #pragma unroll
       for (int c = 0; c < CH_D / 32; ++c) {
         float v[32];
-        if (nt > 0) {
-          tmem_ld32(o_col + c * 32, v);
-          tmem_wait_ld();
-        } else {
+        tmem_ld32(o_col + c * 32, v);
+        tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0.f;
-        }
-        if (row_valid) {
+        for (int i = 0; i < 32; i += 4)
+          __stcg(reinterpret_cast<float4*>(dst + c * 32 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+      }
+      __stcg(reinterpret_cast<float2*>(dst + CH_D), make_float2(m_ref, l));
+      tc_fence_before();
+      mbar_arrive(&sh.o_empty[w]);  // O has been read
+      // One count per (item, row): the thread that lands a row's last piece
+      // merges that row, with no wait on any other thread.
+      __threadfence();
+      if (atomicAdd(cnt, 1) != c_last - c_first) continue;
+      *cnt = 0;  // every piece of this row has arrived: back to zero for the next call
+      __threadfence();
+      // merge in CTA order: m = max m_k, out = sum_k 2^(m_k - m) O_k / sum_k 2^(m_k - m) l_k
+      float mmax = -INFINITY, lsum = 0.f;
+      for (int c = c_first; c <= c_last; ++c) {
+        const int sl = c == c_first ? first_slot : 0;
+        const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
+        mmax = fmaxf(mmax, __ldcg(src + CH_D));
+      }
+      for (int c = c_first; c <= c_last; ++c) {
+        const int sl = c == c_first ? first_slot : 0;
+        const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(src + CH_D));
+        lsum += ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mmax) * ml.y;
+      }
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      if (!row_valid) continue;
+#pragma unroll 1
+      for (int cc = 0; cc < CH_D / 32; ++cc) {
+        float acc[32];
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 u;
-            u.x = pack_bf16x2(v[i] * inv, v[i + 1] * inv);
-            u.y = pack_bf16x2(v[i + 2] * inv, v[i + 3] * inv);
-            u.z = pack_bf16x2(v[i + 4] * inv, v[i + 5] * inv);
-            u.w = pack_bf16x2(v[i + 6] * inv, v[i + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + i) = u;
+        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+        for (int c = c_first; c <= c_last; ++c) {
+          const int sl = c == c_first ? first_slot : 0;
+          const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
+          const float mk = __ldcg(src + CH_D);
+          const float wk = mk == -INFINITY ? 0.f : fast_exp2(mk - mmax);
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src + cc * 32 + i));
+            acc[i] += wk * v4.x;
+            acc[i + 1] += wk * v4.y;
+            acc[i + 2] += wk * v4.z;
+            acc[i + 3] += wk * v4.w;
           }
         }
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 u4;
+          u4.x = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+          u4.y = pack_bf16x2(acc[i + 2] * inv, acc[i + 3] * inv);
+          u4.z = pack_bf16x2(acc[i + 4] * inv, acc[i + 5] * inv);
+          u4.w = pack_bf16x2(acc[i + 6] * inv, acc[i + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + cc * 32 + i) = u4;
+        }
       }
-      tc_fence_before();
-      mbar_arrive(&sh.o_empty[w]);
     }
   }
+
 
   // ---- teardown: drain this CTA's tensor-core work, then free tensor memory
   if (warp == 1) {
@@ -540,6 +691,9 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
   }
+  // beside the decode kernel: this grid completes only after that one has, so
+  // the stream's later work is ordered after both
+  if (p.dep_at_end) grid_dependency_wait();
 }
 
 // ------------------------------------------------------------------ host side
@@ -558,7 +712,7 @@ static int encode_q_tmap(CUtensorMap* map, const void* q, int total_q_tokens, in
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+  return r == CUDA_SUCCESS ? PA_OK : cu_fail(r, "cuTensorMapEncodeTiled");
 }
 
 // [num_blocks, Hkv, block_size, D] as a 4-D tensor; box = 64 columns x 16 rows of one (block, head).
@@ -573,12 +727,12 @@ int encode_kv16_tmap(CUtensorMap* map, const void* cache, int num_blocks, int nu
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(cache), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+  return r == CUDA_SUCCESS ? PA_OK : cu_fail(r, "cuTensorMapEncodeTiled");
 }
 
 template <int G>
 static int launch_chunk_t(const ChunkParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          cudaStream_t stream, int num_sms) {
+                          cudaStream_t stream, int num_sms, int ctas) {
   auto kern = chunk_kernel<G>;
   const int smem = SMEM_TOTAL + 1024;
   static PerDevice configured;
@@ -586,12 +740,12 @@ static int launch_chunk_t(const ChunkParams& p, const CUtensorMap& tq, const CUt
   const int rc_setup = per_device(
       configured,
       [&](int) {
-        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1
-                                                                                                           : PA_ERR_CUDA;
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        return e == cudaSuccess ? 1 : cuda_fail(e, "cudaFuncSetAttribute");
       },
       &done);
   if (rc_setup != PA_OK) return rc_setup;
-  const int grid = num_sms;  // persistent: CTAs walk the items (their count is known on the device only)
+  const int grid = ctas > 0 && ctas < num_sms ? ctas : num_sms;  // one CTA per SM, one unit range each
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(CH_THREADS);
@@ -602,12 +756,35 @@ static int launch_chunk_t(const ChunkParams& p, const CUtensorMap& tq, const CUt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p) != cudaSuccess) return PA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return check_launch(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p), "chunk_kernel launch");
+}
+
+// Items of a batch: pairs of M-tiles (256 / G tokens) of each multi-row
+// sequence, times the KV heads; at most (rows * G / 256 + sequences) * Hkv.
+static size_t chunk_max_items(int num_query_tokens, int num_seqs_bound, int num_kv_heads, int group) {
+  return (static_cast<size_t>(num_query_tokens) * group / (2 * CH_M) + static_cast<size_t>(num_seqs_bound)) *
+         static_cast<size_t>(num_kv_heads);
+}
+
+static size_t round256_c(size_t n) { return (n + 255) / 256 * 256; }
+
+size_t chunk_workspace_bytes(int num_query_tokens, int num_seqs_bound, int num_kv_heads, int group, int num_sms) {
+  const size_t counters = chunk_max_items(num_query_tokens, num_seqs_bound, num_kv_heads, group) * 2 * CH_M * sizeof(int);
+  const size_t slots = static_cast<size_t>(num_sms) * 2 * 2 * CH_M * SLOT_STRIDE * sizeof(float);
+  return round256_c(counters) + slots;
+}
+
+void chunk_workspace_layout(void* ws, int num_query_tokens, int num_seqs_bound, int num_kv_heads, int group,
+                            int num_sms, ChunkParams* p) {
+  (void)num_sms;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  p->counters = reinterpret_cast<int*>(b);
+  b += round256_c(chunk_max_items(num_query_tokens, num_seqs_bound, num_kv_heads, group) * 2 * CH_M * sizeof(int));
+  p->partials = reinterpret_cast<float*>(b);
 }
 
 int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const void* v_cache, int total_q_tokens,
-                 cudaStream_t stream, int num_sms) {
+                 cudaStream_t stream, int num_sms, int ctas) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return PA_ERR_CUDA;
   CUtensorMap tq, tk, tv;
@@ -616,11 +793,11 @@ int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const
   if ((rc = encode_kv16_tmap(&tk, k_cache, p.num_blocks, p.num_kv_heads, p.block_size, fn)) != PA_OK) return rc;
   if ((rc = encode_kv16_tmap(&tv, v_cache, p.num_blocks, p.num_kv_heads, p.block_size, fn)) != PA_OK) return rc;
   switch (p.group) {
-    case 1: return launch_chunk_t<1>(p, tq, tk, tv, stream, num_sms);
-    case 2: return launch_chunk_t<2>(p, tq, tk, tv, stream, num_sms);
-    case 4: return launch_chunk_t<4>(p, tq, tk, tv, stream, num_sms);
-    case 8: return launch_chunk_t<8>(p, tq, tk, tv, stream, num_sms);
-    case 16: return launch_chunk_t<16>(p, tq, tk, tv, stream, num_sms);
+    case 1: return launch_chunk_t<1>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 2: return launch_chunk_t<2>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 4: return launch_chunk_t<4>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 8: return launch_chunk_t<8>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 16: return launch_chunk_t<16>(p, tq, tk, tv, stream, num_sms, ctas);
     default: return PA_ERR_UNSUPPORTED;
   }
 }

@@ -12,6 +12,22 @@
 
 namespace pa {
 
+// A CUDA call failed: remember its error for pa_last_cuda_error() (per host
+// thread) and return PA_ERR_CUDA.
+int cuda_fail(cudaError_t e, const char* call);
+int cu_fail(CUresult r, const char* call);
+// The result of a kernel launch: the launch call's own error, else the
+// thread's last runtime error (a launch-configuration error, or a sticky error
+// left by an earlier kernel that faulted).
+inline int check_launch(cudaError_t launch_rc, const char* what) {
+  if (launch_rc != cudaSuccess) {
+    (void)cudaGetLastError();
+    return cuda_fail(launch_rc, what);
+  }
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, what);
+}
+
 // Per-device launch set-up of one kernel (its shared-memory opt-in, its CTAs
 // per SM), done once per device and safe under concurrent callers: the value
 // is an atomic, and two threads that set the same device up at once both make
@@ -26,7 +42,9 @@ struct PerDevice {
 template <class Setup>
 int per_device(PerDevice& cache, Setup setup, int* out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= PA_MAX_DEVICES) return PA_ERR_CUDA;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= PA_MAX_DEVICES) return PA_ERR_CUDA;
   int v = cache.value[dev].load(std::memory_order_acquire);
   if (v <= 0) {
     v = setup(dev);
@@ -68,6 +86,7 @@ struct RowsParams {
   int* status;      // optional device status word
   int total_warps;
   int tile_shift;   // log2 of the keys per work unit (16, or 32 for the E4M3 kernel with one head tile)
+  int trigger_early;  // 1: release the dependent grid (the chunk kernel beside this one) once the append is visible
   // Fused cache append (decode only; nullptr: none).  Row s of k_new / v_new
   // ([B, Hkv, D] bf16) is sequence s's newest token: the kernel writes it to
   // position context_lens[s] - 1 through the block table and attends to it
@@ -165,8 +184,9 @@ struct VerifyParams {
 };
 
 int verify_supported(int group, int head_dim, int num_seqs);
+// which: bit 0 launches the 32-column kernel, bit 1 the 64-column one.
 int launch_verify(const VerifyParams& p, const void* q, const void* k_cache, const void* v_cache,
-                  int total_q_tokens, cudaStream_t stream, int num_sms);
+                  int total_q_tokens, cudaStream_t stream, int num_sms, int which = 3);
 
 struct ChunkParams {
   void* out;                    // bf16 [Tq, Hq, 128]
@@ -183,7 +203,18 @@ struct ChunkParams {
   float scale_log2;
   int* status;
   int min_qlen;  // sequences with fewer query rows belong to the other kernels
+  // Stream-K pieces: two (O, m, l) slots per CTA, each [256 rows][132 floats],
+  // and one count per (item, row), zero between calls.
+  float* partials;
+  int* counters;
+  int dep_at_end;  // 1: launched beside the decode kernel; wait for the grid before at the end
 };
+
+// Workspace of the chunk kernel's pieces for a batch of at most
+// num_query_tokens rows, and its carving (after the rows kernel's part).
+size_t chunk_workspace_bytes(int num_query_tokens, int num_seqs_bound, int num_kv_heads, int group, int num_sms);
+void chunk_workspace_layout(void* ws, int num_query_tokens, int num_seqs_bound, int num_kv_heads, int group,
+                            int num_sms, ChunkParams* p);
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -197,7 +228,10 @@ struct DeviceInfo {
   int num_sms;
 };
 
+// The current device's SM count; makes the device's primary context current
+// first if the calling host thread has no current context.
 int device_info(DeviceInfo* info);
+int ensure_context(int dev);
 int encode_kv_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
                    int head_dim);
 
@@ -208,8 +242,10 @@ int launch_append(const void* k_new, const void* v_new, void* k_cache, void* v_c
 int launch_append_fp8(const void* k_new, const void* v_new, void* k_cache, void* v_cache,
                       const int32_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads, int head_dim,
                       int block_size, float k_inv, float v_inv, int* dev_status, cudaStream_t stream, int num_sms);
+// ctas > 0: launch that many 8-warp CTAs (one per SM) instead of filling the
+// GPU, leaving the other SMs to a kernel launched beside it (head_dim 128).
 int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
-                cudaStream_t stream, int num_sms);
+                cudaStream_t stream, int num_sms, int ctas = 0);
 // Workspace of the rows kernel for at most num_rows query rows on a device with
 // num_sms SMs, and the carving of a buffer of that size into RowsParams.
 // max_keys bounds the keys of any row (max_blocks_per_seq * block_size).
@@ -219,12 +255,27 @@ void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_h
                            long long max_keys, int num_sms, RowsParams* p);
 int rows_supported(int group, int head_dim);
 int chunk_supported(int group, int head_dim);
+// ctas: CTAs of the launch (one per SM), at most num_sms.
 int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const void* v_cache, int total_q_tokens,
-                 cudaStream_t stream, int num_sms);
+                 cudaStream_t stream, int num_sms, int ctas);
 int cascade_supported(int group, int head_dim);
 size_t cascade_partials_bytes(int num_seqs, int num_q_heads, int head_dim);
 int launch_cascade(const CascadeParams& p, const void* q, const void* k_cache, const void* v_cache,
                    int total_q_tokens, int head_dim, cudaStream_t stream, int num_sms);
+// Host plan of a varlen batch (the words of pa_plan).
+enum PlanWord {
+  PLAN_MAGIC = 0,    // PLAN_MAGIC_VALUE once filled in
+  PLAN_FLAGS,        // PLAN_VERIFY32 | PLAN_VERIFY64 | PLAN_CHUNK | PLAN_ROWS: kernels that have work
+  PLAN_DECODE_CTAS,  // > 0: decode rows on this many SMs beside the chunk kernel on the others
+  PLAN_NUM_SMS,      // SM count the split was made for
+  PLAN_NUM_SEQS,
+  PLAN_TOTAL_Q,
+  PLAN_GROUP,
+  PLAN_HEAD_DIM,
+};
+constexpr int32_t PLAN_MAGIC_VALUE = 0x50414e31;  // "PAN1"
+constexpr int32_t PLAN_VERIFY32 = 1, PLAN_VERIFY64 = 2, PLAN_CHUNK = 4, PLAN_ROWS = 8;
+
 // Argument checks, tensor maps and kernel dispatch shared by the attention
 // entry points (query_start == nullptr: one query row per sequence).
 int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,
@@ -233,6 +284,10 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                   int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
                   void* stream, const void* k_new = nullptr, const void* v_new = nullptr,
                   const int32_t* group_start = nullptr, const int32_t* group_prefix = nullptr, int num_groups = 0,
-                  int kv_fp8 = 0, float k_scale = 1.f, float v_scale = 1.f);
+                  int kv_fp8 = 0, float k_scale = 1.f, float v_scale = 1.f, const int32_t* plan = nullptr);
+// Bytes of workspace a decode call (one query row per sequence) needs: the
+// rows kernel's part of pa_workspace_bytes.
+size_t decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                              int block_size);
 
 }  // namespace pa

@@ -78,6 +78,8 @@ bool current_context_id(unsigned long long* id) {
 int scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return PA_ERR_CUDA;
+  const int rc = ensure_context(dev);
+  if (rc != PA_OK) return rc;
   std::lock_guard<std::mutex> lock(g_setup_mu);
   unsigned long long id = 0;
   const bool have_id = current_context_id(&id);
@@ -89,7 +91,7 @@ int scratch_for_current_device(void** out) {
   const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
   if (e != cudaSuccess || p == nullptr) {
     (void)cudaGetLastError();
-    return PA_ERR_CUDA;
+    return e != cudaSuccess ? cuda_fail(e, "cudaGetSymbolAddress") : static_cast<int>(PA_ERR_CUDA);
   }
   // the lookup makes the device's primary context current if no context was
   unsigned long long id_now = 0;
@@ -112,8 +114,9 @@ extern "C" int pa_decode_static_scratch(void* out, const void* q, const void* k_
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_ERR_NULL;
   if (num_seqs < 0) return PA_ERR_SHAPE;
   const size_t need =
-      num_seqs > 0 ? pa_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size)
-                   : 0;
+      num_seqs > 0
+          ? pa::decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, block_size)
+          : 0;
   if (need == 0) {
     // an empty batch or invalid sizes: pa_decode's own checks decide, and
     // they return before any launch and before the workspace is looked at
@@ -135,7 +138,8 @@ extern "C" int pa_decode_static_scratch(void* out, const void* q, const void* k_
                             static_cast<long long>(max_blocks_per_seq) * block_size, di.num_sms, &lay);
   const size_t zero_bytes =
       static_cast<size_t>(reinterpret_cast<unsigned char*>(lay.table) - static_cast<unsigned char*>(ws));
-  if (cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  const cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return pa::cuda_fail(e, "cudaMemsetAsync");
   return pa::run_attention(out, q, nullptr, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                            num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                            ws, PA_STATIC_SCRATCH_BYTES, dev_status, stream);

@@ -40,11 +40,16 @@
 namespace pa {
 
 constexpr int TILE_KEYS = 16;  // keys per work unit, and per TMA box; a variant may take two boxes per unit
-constexpr int ROWS_WARPS = 4;
-constexpr int ROWS_THREADS = ROWS_WARPS * 32;
+constexpr int ROWS_WARPS = 4;       // warps per CTA of the usual launch (2 or 3 CTAs per SM)
+constexpr int ROWS_WARPS_WIDE = 8;  // warps per CTA when a CTA holds a whole SM (a launch on part of the GPU)
 constexpr int ROWS_SLOTS_PER_WARP = 2;  // a warp's range cuts at most its first and its last segment
 constexpr int ROWS_SMEM_SEQS = ROWS_SMEM_SEQS_HOST;  // sequences whose tile prefix sums live in shared memory
 constexpr int ROWS_MAX_CTAS_PER_SM = 3;  // the workspace holds partial slots for this many CTAs per SM
+// Accumulation chains of S = K Q^T per tile (bf16 path): 1, or 2 (even and odd k-steps).
+#ifndef PA_ROWS_S_CHAINS
+#define PA_ROWS_S_CHAINS 1
+#endif
+constexpr int ROWS_S_CHAINS = PA_ROWS_S_CHAINS;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -406,7 +411,7 @@ __device__ __forceinline__ void store_own_partial(const RowsParams& p, const flo
 // table entry of its first unit, so the walk visits the pieces in order; one
 // pass with a running maximum.
 template <int D, int NT, bool F8>
-__device__ __noinline__ void merge_segment(const RowsParams& p, long long segA, int n, int row, int kvh, int lane) {
+__device__ __forceinline__ void merge_segment(const RowsParams& p, long long segA, int n, int row, int kvh, int lane) {
   using S = RowsShape<D, NT, F8>;
   constexpr int KT = S::KT;
   const int c = lane & 3;
@@ -529,23 +534,24 @@ constexpr int rows_ctas_per_sm() {
 // at head_dim 128 with one head tile) a stage holds two 16-row TMA boxes per
 // K and V and the warp takes two 16-key m-tiles per softmax step, so the
 // per-tile bookkeeping covers twice the bytes.
-template <int D, int NT, int R, bool F8, int TK>
-__global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8, TK>() == 3 ? 3 : 1)
+template <int D, int NT, int R, bool F8, int TK, int NW>
+__global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 3 ? 3 : 1)
     rows_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                 const RowsParams p) {
   static_assert(TK == TILE_KEYS || (TK == 2 * TILE_KEYS && F8 && D == 128 && NT == 1), "32-key tiles: E4M3, D 128, G <= 8");
   using S = RowsShape<D, NT, F8, TK>;
   constexpr int KT = S::KT;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[ROWS_WARPS][R];
-  __shared__ TileMeta metas[ROWS_WARPS][R];
+  constexpr int ROWS_THREADS = NW * 32;
+  __shared__ __align__(8) uint64_t bars[NW][R];
+  __shared__ TileMeta metas[NW][R];
 
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int gw = blockIdx.x * ROWS_WARPS + warp;
+  const int gw = blockIdx.x * NW + warp;
   const int g = lane >> 2, c = lane & 3;
   uint8_t* base = align1024(smem_raw);
   const bool use_pfx = p.num_seqs <= ROWS_SMEM_SEQS;
-  long long* pfx = use_pfx ? reinterpret_cast<long long*>(base + ROWS_WARPS * R * S::STAGE_BYTES) : nullptr;
+  long long* pfx = use_pfx ? reinterpret_cast<long long*>(base + NW * R * S::STAGE_BYTES) : nullptr;
 
   // ---- prologue: tiles of every sequence, their prefix sums, the total T.
   // Rows without a key are written as zeros here (each by one thread).
@@ -577,6 +583,9 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8, TK>(
   // reads the cache (which the append kernel before it may still be writing)
   // and writes out: wait for the grids this launch depends on.
   grid_dependency_wait();
+  // beside the chunk kernel: the append is visible now, so that kernel may
+  // take the SMs this launch leaves free
+  if (p.trigger_early) grid_launch_dependents();
   for (int s = blockIdx.x * ROWS_THREADS + threadIdx.x; s < p.num_seqs; s += gridDim.x * ROWS_THREADS) {
     const SeqInfo si = seq_info(p, s);  // rows without a key are written as zeros
     const int nzero = min(si.qlen, max(0, si.qlen - si.ctx));
@@ -994,6 +1003,24 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8, TK>(
               mma_f16_16816(sacc[nt], b0, b1, b2, b3, qb[nt][2 * x + 1][0], qb[nt][2 * x + 1][1]);
             }
           }
+        } else if constexpr (ROWS_S_CHAINS == 2) {
+          // two independent accumulation chains (even and odd k-steps), summed:
+          // half the dependent MMA latency on the per-tile critical path
+          float sacc2[NT][4];
+  #pragma unroll
+          for (int nt = 0; nt < NT; ++nt) sacc2[nt][0] = sacc2[nt][1] = sacc2[nt][2] = sacc2[nt][3] = 0.f;
+  #pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+  #pragma unroll
+            for (int kk = 0; kk < KT; kk += 2) {
+              mma_bf16_16816(sacc[nt], kf[kk][0], kf[kk][1], kf[kk][2], kf[kk][3], qb[nt][kk][0], qb[nt][kk][1]);
+              mma_bf16_16816(sacc2[nt], kf[kk + 1][0], kf[kk + 1][1], kf[kk + 1][2], kf[kk + 1][3], qb[nt][kk + 1][0],
+                             qb[nt][kk + 1][1]);
+            }
+  #pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+  #pragma unroll
+            for (int r = 0; r < 4; ++r) sacc[nt][r] += sacc2[nt][r];
         } else {
   #pragma unroll
           for (int nt = 0; nt < NT; ++nt)
@@ -1178,22 +1205,24 @@ __global__ void __launch_bounds__(ROWS_THREADS, rows_ctas_per_sm<D, NT, F8, TK>(
 
 // ------------------------------------------------------------------ host side
 
-template <int D, int NT, int R, bool F8 = false, int TK = TILE_KEYS>
+template <int D, int NT, int R, bool F8 = false, int TK = TILE_KEYS, int NW = ROWS_WARPS>
 static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUtensorMap& tmv, cudaStream_t stream,
-                         int num_sms) {
+                         int num_sms, int ctas) {
+  constexpr int ROWS_THREADS = NW * 32;
   using S = RowsShape<D, NT, F8, TK>;
-  const int smem = ROWS_WARPS * R * S::STAGE_BYTES + 1024 + (ROWS_SMEM_SEQS + 1) * 8;
-  auto kern = rows_kernel<D, NT, R, F8, TK>;
+  const int smem = NW * R * S::STAGE_BYTES + 1024 + (ROWS_SMEM_SEQS + 1) * 8;
+  auto kern = rows_kernel<D, NT, R, F8, TK, NW>;
   static PerDevice configured;  // CTAs per SM on each device
   int blocks_per_sm = 0;
   const int rc_setup = per_device(
       configured,
       [&](int) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-          return static_cast<int>(PA_ERR_CUDA);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         int nb = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, ROWS_THREADS, smem) != cudaSuccess || nb < 1)
-          return static_cast<int>(PA_ERR_CUDA);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, ROWS_THREADS, smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+        if (nb < 1) return static_cast<int>(PA_ERR_CUDA);
         constexpr int cap = rows_ctas_per_sm<D, NT, F8, TK>();
         return nb > cap ? cap : nb;
       },
@@ -1201,8 +1230,11 @@ static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUt
   if (rc_setup != PA_OK) return rc_setup;
   RowsParams p = p0;
   p.tile_shift = TK == 32 ? 5 : 4;
-  const int grid = num_sms * blocks_per_sm;
-  p.total_warps = grid * ROWS_WARPS;
+  // ctas > 0: a launch on part of the GPU (one CTA per SM, the rest of the
+  // SMs left to a kernel that runs beside it)
+  const int grid = ctas > 0 ? (ctas < num_sms * blocks_per_sm ? ctas : num_sms * blocks_per_sm)
+                            : num_sms * blocks_per_sm;
+  p.total_warps = grid * NW;
   // Programmatic dependent launch: the prologue (a scan of the batch
   // metadata) overlaps the kernel before it, typically the cache append;
   // the kernel waits for that grid before it reads the cache.
@@ -1220,8 +1252,7 @@ static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUt
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p) != cudaSuccess) return PA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return check_launch(cudaLaunchKernelEx(&cfg, kern, tmk, tmv, p), "rows_kernel launch");
 }
 
 int rows_supported(int group, int head_dim) {
@@ -1240,6 +1271,7 @@ size_t slot_bytes(int group, int head_dim) {
   return (o + 16 * nt + 1 + 63) / 64 * 64 * sizeof(float);
 }
 size_t max_warps(int num_sms) { return static_cast<size_t>(num_sms) * ROWS_MAX_CTAS_PER_SM * ROWS_WARPS; }
+static_assert(ROWS_WARPS_WIDE <= ROWS_MAX_CTAS_PER_SM * ROWS_WARPS, "partial slots per SM");
 }  // namespace
 
 namespace {
@@ -1285,28 +1317,33 @@ void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_h
 }
 
 int launch_rows(const RowsParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv, int head_dim,
-                cudaStream_t stream, int num_sms) {
+                cudaStream_t stream, int num_sms, int ctas) {
   const bool two = p.group > 8;
   if (p.kv_fp8) {  // E4M3 caches: a tile is half the bytes, so more stages (or more CTAs) per SM
     switch (head_dim) {
       case 128:
-        return two ? launch_rows_t<128, 2, 6, true>(p, tmk, tmv, stream, num_sms)
-                   : launch_rows_t<128, 1, 3, true, 32>(p, tmk, tmv, stream, num_sms);
+        return two ? launch_rows_t<128, 2, 6, true>(p, tmk, tmv, stream, num_sms, 0)
+                   : launch_rows_t<128, 1, 3, true, 32>(p, tmk, tmv, stream, num_sms, 0);
       case 256:
-        return launch_rows_t<256, 1, 3, true>(p, tmk, tmv, stream, num_sms);
+        return launch_rows_t<256, 1, 3, true>(p, tmk, tmv, stream, num_sms, 0);
       default:
         return PA_ERR_UNSUPPORTED;
     }
   }
+  if (ctas > 0) {  // part of the GPU, one 8-warp CTA per SM (head_dim 128: the tcgen05 chunk path's shapes)
+    if (head_dim != 128) return PA_ERR_UNSUPPORTED;
+    return two ? launch_rows_t<128, 2, 3, false, TILE_KEYS, ROWS_WARPS_WIDE>(p, tmk, tmv, stream, num_sms, ctas)
+               : launch_rows_t<128, 1, 3, false, TILE_KEYS, ROWS_WARPS_WIDE>(p, tmk, tmv, stream, num_sms, ctas);
+  }
   switch (head_dim) {
     case 64:
-      return two ? launch_rows_t<64, 2, 8>(p, tmk, tmv, stream, num_sms)
-                 : launch_rows_t<64, 1, 8>(p, tmk, tmv, stream, num_sms);
+      return two ? launch_rows_t<64, 2, 8>(p, tmk, tmv, stream, num_sms, 0)
+                 : launch_rows_t<64, 1, 8>(p, tmk, tmv, stream, num_sms, 0);
     case 128:
-      return two ? launch_rows_t<128, 2, 3>(p, tmk, tmv, stream, num_sms)
-                 : launch_rows_t<128, 1, 3>(p, tmk, tmv, stream, num_sms);
+      return two ? launch_rows_t<128, 2, 3>(p, tmk, tmv, stream, num_sms, 0)
+                 : launch_rows_t<128, 1, 3>(p, tmk, tmv, stream, num_sms, 0);
     case 256:
-      return launch_rows_t<256, 1, 3>(p, tmk, tmv, stream, num_sms);
+      return launch_rows_t<256, 1, 3>(p, tmk, tmv, stream, num_sms, 0);
     default:
       return PA_ERR_UNSUPPORTED;
   }

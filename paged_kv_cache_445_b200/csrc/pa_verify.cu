@@ -850,7 +850,7 @@ static int encode_vq_tmap(CUtensorMap* map, const void* q, int total_q_tokens, i
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+  return r == CUDA_SUCCESS ? PA_OK : cu_fail(r, "cuTensorMapEncodeTiled");
 }
 
 template <int NCOL>
@@ -863,8 +863,8 @@ static int launch_verify_t(const VerifyParams& p0, const CUtensorMap& tq, const 
   const int rc_setup = per_device(
       configured,
       [&](int) {
-        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess ? 1
-                                                                                                           : PA_ERR_CUDA;
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        return e == cudaSuccess ? 1 : cuda_fail(e, "cudaFuncSetAttribute");
       },
       &done);
   if (rc_setup != PA_OK) return rc_setup;
@@ -881,12 +881,11 @@ static int launch_verify_t(const VerifyParams& p0, const CUtensorMap& tq, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p) != cudaSuccess) return PA_ERR_CUDA;
-  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return check_launch(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p), "verify_kernel launch");
 }
 
 int launch_verify(const VerifyParams& p, const void* q, const void* k_cache, const void* v_cache,
-                  int total_q_tokens, cudaStream_t stream, int num_sms) {
+                  int total_q_tokens, cudaStream_t stream, int num_sms, int which) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return PA_ERR_CUDA;
   CUtensorMap tk, tv;
@@ -895,10 +894,15 @@ int launch_verify(const VerifyParams& p, const void* q, const void* k_cache, con
   if ((rc = encode_kv16_tmap(&tv, v_cache, p.num_blocks, p.num_kv_heads, p.block_size, fn)) != PA_OK) return rc;
   // columns <= 32 on the 32-wide kernel, 33 .. 64 on the 64-wide one
   CUtensorMap tq;
-  if ((rc = encode_vq_tmap(&tq, q, total_q_tokens, p.num_q_heads, p.group, 32, fn)) != PA_OK) return rc;
-  if ((rc = launch_verify_t<32>(p, tq, tk, tv, stream, num_sms)) != PA_OK) return rc;
-  if ((rc = encode_vq_tmap(&tq, q, total_q_tokens, p.num_q_heads, p.group, 64, fn)) != PA_OK) return rc;
-  return launch_verify_t<64>(p, tq, tk, tv, stream, num_sms);
+  if (which & 1) {
+    if ((rc = encode_vq_tmap(&tq, q, total_q_tokens, p.num_q_heads, p.group, 32, fn)) != PA_OK) return rc;
+    if ((rc = launch_verify_t<32>(p, tq, tk, tv, stream, num_sms)) != PA_OK) return rc;
+  }
+  if (which & 2) {
+    if ((rc = encode_vq_tmap(&tq, q, total_q_tokens, p.num_q_heads, p.group, 64, fn)) != PA_OK) return rc;
+    if ((rc = launch_verify_t<64>(p, tq, tk, tv, stream, num_sms)) != PA_OK) return rc;
+  }
+  return PA_OK;
 }
 
 }  // namespace pa

@@ -34,7 +34,7 @@ class _Event:
 class _Step:
     """The attributes bench.run_ours reads from GpuStep, on the CPU; append and attend do nothing."""
 
-    def __init__(self, w, device, fused=True, cascade=True, fp8=False):
+    def __init__(self, w, device, fused=True, cascade=True, fp8=False, plan=True):
         def t(a, dtype):
             return torch.from_numpy(np.ascontiguousarray(a).astype(dtype))
         self.w = w
@@ -47,6 +47,7 @@ class _Step:
         self.fused = self.decode and fused
         self.fp8 = fp8
         self.cascade = False
+        self.plan = None
         self.launches = 1 if self.fused else bench.step_launches(w)
         self.inputs = ["q", "k_new", "v_new", "block_tables", "context_lens"]
         if not self.fused:
@@ -75,7 +76,8 @@ def fake_device(monkeypatch):
 def _line(capsys, workload, **kw):
     args = argparse.Namespace(gpus=1, steps=4, warmup=3, workload=workload, impl="ours", cpu_seconds=0.2,
                               reference_seconds=1.0, no_cpu_baseline=True, kv_dtype="bf16", graph=False,
-                              cascade=False, separate_append=False)
+                              cascade=False, separate_append=False, no_plan=False, no_sub_records=True,
+                              sub_cpu_seconds=0.1)
     for k, v in kw.items():
         setattr(args, k, v)
     bench.run_ours(args, (6530.3, 1626.0, 1399.0, "measured"))
@@ -108,3 +110,19 @@ def test_small_workload_runs_with_l2_flushed_and_times_the_oracle(fake_device, c
     assert d["l2_warm"]["unit"] == "GB/s" and d["l2_warm"]["ms_per_step"] > 0
     cpu = d["cpu_baseline"]
     assert cpu["kind"] == "oracle" and cpu["unit"] == "GB/s" and cpu["value"] > 0 and cpu["cores"] >= 1
+
+
+def test_default_run_carries_the_other_workloads_as_sub_records(fake_device, capsys):
+    d = _line(capsys, 3, no_sub_records=False)
+    subs = d["workloads"]
+    assert set(subs) == {"grpo-shared-prefix", "grpo-shared-prefix-cascade", "mixed-chunk-decode",
+                         "llama3.3-70b-layer-decode-b128-fp8"}
+    for key, sub in subs.items():
+        for k in ("value", "unit", "ms_per_step", "dtype", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+            assert k in sub, (key, k)
+        assert sub["roofline"]["frac"] == pytest.approx(sub["roofline"]["achieved"] / sub["roofline"]["peak"],
+                                                        rel=1e-3)
+    assert subs["grpo-shared-prefix"]["config"]["l2"].startswith("flushed")
+    assert subs["mixed-chunk-decode"]["roofline_tensor"]["unit"] == "TFLOP/s"
+    assert "overlap_bound" in subs["mixed-chunk-decode"]
+    assert subs["llama3.3-70b-layer-decode-b128-fp8"]["dtype"].startswith("fp8")

@@ -335,3 +335,28 @@ def test_a_captured_step_replays_bit_identically(cfg):
         torch.cuda.synchronize()
         assert int(ds.status.item()) == 0
         assert torch.equal(ds.out.view(torch.int16), eager.view(torch.int16))
+
+
+def test_a_wait_that_runs_out_is_reported_and_the_context_stays_usable():
+    # The decode kernel's grid barrier waits (bounded, about 2 s) until every
+    # warp has arrived on the workspace counter, which the caller zero-fills.
+    # A counter left at -1 (the zero-fill skipped) never reaches the target:
+    # the wait runs out, the kernel sets the TIMEOUT bit and returns, and
+    # nothing faults.  After a zero-fill the next call is exact again.
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.custom([3000, 40, 1200], [1, 1, 1], 16, 2, 128, 16, seed=14, poison=True)
+    ds = DeviceStep(w)
+    ds.append()
+    kc, vc = oracle_after_append(w)
+    ref = _attend_ref(w, kc, vc)
+    ds.workspace.view(torch.int32)[0] = -1  # the barrier's arrival counter
+    ds.attend()
+    torch.cuda.synchronize()
+    assert int(ds.status.item()) & pa.status_bit(pa._binding.PA_ERR_TIMEOUT)
+    ds.status.zero_()
+    ds.workspace.zero_()
+    ds.out.fill_(0)
+    ds.attend()
+    torch.cuda.synchronize()
+    assert int(ds.status.item()) == 0
+    compare(ds.out.float().cpu().numpy(), ref, "after a timed-out call")

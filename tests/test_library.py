@@ -188,3 +188,21 @@ def test_a_missing_library_fails_loudly(tmp_path):
                        env={**os.environ, "PYTHONPATH": str(tmp_path)})
     assert r.returncode == 0, r.stderr
     assert "raised:" in r.stdout and "no CPU fallback" in r.stdout
+
+
+def test_plan_rejects_bad_arguments_before_touching_a_device():
+    import ctypes as C
+    from paged_kv_cache_445_b200 import _binding as b
+    qs = (C.c_int32 * 3)(0, 5, 6)
+    cl = (C.c_int32 * 2)(40, 7)
+    plan = b.Plan()
+    L = b._lib
+    assert L.pa_plan_batch(None, cl, 2, 8, 2, 128, 16, 8, C.byref(plan)) == b.PA_ERR_NULL
+    assert L.pa_plan_batch(qs, cl, 2, 8, 2, 128, 16, 8, None) == b.PA_ERR_NULL
+    assert L.pa_plan_batch(qs, cl, 2, 6, 4, 128, 16, 8, C.byref(plan)) == b.PA_ERR_SHAPE       # Hq % Hkv
+    assert L.pa_plan_batch(qs, cl, 2, 8, 2, 96, 16, 8, C.byref(plan)) == b.PA_ERR_UNSUPPORTED  # head_dim
+    assert L.pa_plan_batch(qs, cl, 2, 8, 2, 128, 24, 8, C.byref(plan)) == b.PA_ERR_UNSUPPORTED  # block size
+    bad = (C.c_int32 * 3)(1, 5, 6)  # query_start must start at 0
+    assert L.pa_plan_batch(bad, cl, 2, 8, 2, 128, 16, 8, C.byref(plan)) == b.PA_ERR_SHAPE
+    assert L.pa_prefill_chunk_planned(4096, 4096, None, 4096, 4096, 4096, 4, 4096, 2, 6, 8, 2, 128, 16, 10, 0.1,
+                                      4096, 1 << 20, C.byref(plan), None, None) == b.PA_ERR_NULL
