@@ -615,21 +615,39 @@ def measure(args, peaks, workload, rank, world, local, *, cascade, fp8, plan=Tru
 SUB_RECORDS = [  # (key, workload, cascade, fp8): the other workloads of the default run, at N = 1
     ("grpo-shared-prefix", 4, False, False),
     ("grpo-shared-prefix-cascade", 4, True, False),
+    ("grpo-long-prefix", 7, False, False),
+    ("grpo-long-prefix-cascade", 7, True, False),
     ("mixed-chunk-decode", 5, False, False),
     ("llama3.3-70b-layer-decode-b128-fp8", 3, False, True),
 ]
 
 
+def calibrate(args):
+    """Per-SM streaming rates for the decode split (pa_calibrate), once per run."""
+    if args.no_calibrate:
+        return {"weighted": False}
+    import paged_kv_cache_445_b200 as pa
+    t0 = time.time()
+    w = np.asarray(pa.pa_calibrate(), dtype=np.float64)
+    rel = w / np.median(w)
+    log(f"calibrated {len(w)} SMs in {time.time() - t0:.2f}s: shares {rel.min():.2f} .. {rel.max():.2f} of the median")
+    return {"weighted": True, "sms": int(len(w)), "share_vs_median": {"min": round(float(rel.min()), 3),
+                                                                      "max": round(float(rel.max()), 3)}}
+
+
 def run_ours(args, peaks):
     rank, world, local = dist_setup(args.gpus)
+    split = calibrate(args)
     line = measure(args, peaks, args.workload, rank, world, local, cascade=args.cascade,
                    fp8=args.kv_dtype == "fp8", plan=not args.no_plan)
+    line["config"]["sm_split"] = split
     if world == 1 and not args.no_sub_records and args.workload == 3 and args.kv_dtype == "bf16" \
             and not args.cascade and not args.graph:
         # the other workloads, each with its own roofline, clocks and short CPU baseline
         subs = {}
         for key, wl, casc, f8 in SUB_RECORDS:
             sub = measure(args, peaks, wl, rank, world, local, cascade=casc, fp8=f8, cpu_seconds=args.sub_cpu_seconds)
+            sub["config"]["sm_split"] = split
             for k in ("metric", "n_gpus", "steps", "warmup", "higher_is_better", "scaling", "vs_baseline", "data"):
                 sub.pop(k, None)
             subs[key] = sub
@@ -757,7 +775,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5, 6])
+    ap.add_argument("--workload", type=int, default=3, choices=[1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
@@ -769,6 +787,8 @@ def main(argv=None):
     ap.add_argument("--cascade", action="store_true",
                     help="shared-prefix batches: pa_decode_cascade (each shared prefix read once per group) "
                          "instead of plain decode")
+    ap.add_argument("--no-calibrate", action="store_true",
+                    help="leave out pa_calibrate: the decode kernel splits its work equally between warps")
     ap.add_argument("--no-plan", action="store_true",
                     help="varlen batches: pa_prefill_chunk without the host plan (every kernel launched, one after "
                          "the other on the whole GPU)")

@@ -193,6 +193,22 @@ PA_API int pa_decode_fp8(void* out, const void* q, const void* k_new, const void
                          size_t workspace_bytes, int* dev_status, void* stream);
 
 /*
+ * pa_prefill_chunk_fp8 -- pa_prefill_chunk over an FP8 (E4M3) cache, with the
+ * scales and code format of pa_decode_fp8: a varlen batch of prefill chunks,
+ * verification rows and decodes.  Every row runs on the decode kernel's E4M3
+ * path (each row of a sequence reads its keys; the tcgen05 chunk and
+ * verification kernels take bf16 caches only), so a long chunk costs one
+ * pass over its keys per row.  head_dim 128 or 256; workspace as for
+ * pa_prefill_chunk.
+ */
+PA_API int pa_prefill_chunk_fp8(void* out, const void* q, const int32_t* query_start, const void* k_cache,
+                                const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                                const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
+                                int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                                float k_scale, float v_scale, void* workspace, size_t workspace_bytes, int* dev_status,
+                                void* stream);
+
+/*
  * pa_decode_cascade -- pa_decode (optionally fused with the append, as
  * pa_decode_append) for a batch in which groups of sequences share a prefix of
  * the KV cache, as copy-on-write forks of one prompt do ("vLLM serving
@@ -336,6 +352,44 @@ PA_API int pa_decode_static_scratch(void* out, const void* q, const void* k_cach
                                     const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
                                     int head_dim, int block_size, int num_blocks, float scale, int* dev_status,
                                     void* stream);
+
+/*
+ * pa_calibrate -- per-SM shares for the decode kernel's split of the work,
+ * measured once on this device.
+ *
+ * The decode path is bound by HBM bandwidth and hands every warp a fixed
+ * contiguous share of the batch's key tiles before it starts (no claims at
+ * run time, so results do not depend on timing).  The SMs of a B200 do not
+ * stream equally fast under a full load (timed per warp: pairs of SMs at
+ * about 44, 51 and 59 GB/s, the same from launch to launch), so with equal
+ * shares the GPU waits for its slowest SMs.  pa_calibrate runs the decode
+ * kernel on a synthetic batch (128 sequences x 2048 tokens, 64 query / 8 KV
+ * heads, head_dim 128) held in `buffer`, times every SM's share, and adjusts
+ * per-SM weights over four rounds until the SMs finish together.  Every later
+ * decode launch on this device (pa_decode, pa_decode_append, pa_decode_fp8,
+ * pa_decode_cascade and the decode rows of pa_prefill_chunk*) gives each SM
+ * a share in proportion to its weight.  Not part of the pages' problem
+ * statement: a B200 scheduling aid.
+ *
+ * buffer: device memory of at least pa_calibrate_bytes() bytes (about
+ * 1.1 GB; 256-byte aligned), overwritten.  The call WAITS for its own work
+ * (the library's one synchronising call: a set-up step, about 20 ms).  Call
+ * it once per device, with nothing else running on the device, before the
+ * decode calls that should use it; decode calls that overlap it on other
+ * host threads keep the split they started with.  Results of decode calls
+ * before and after it differ in rounding (the split moves the places where
+ * partial sums are cut).  Returns PA_ERR_WORKSPACE for a small buffer,
+ * PA_ERR_UNSUPPORTED on a GPU with more than 160 SMs, PA_ERR_RANGE if some
+ * SM got no work to time (the equal split stays).
+ *
+ * pa_calibration -- the recorded weights of the current device (relative,
+ * largest 60000; one per SM; weights_out may be NULL): PA_ERR_RANGE if none.
+ * pa_calibration_clear -- forget every device's weights (equal split again).
+ */
+PA_API size_t pa_calibrate_bytes(void);
+PA_API int pa_calibrate(void* buffer, size_t bytes, int* dev_status, void* stream);
+PA_API int pa_calibration(int* num_sms, uint16_t* weights_out);
+PA_API void pa_calibration_clear(void);
 
 /* Human-readable name of a pa_status value (static storage). */
 PA_API const char* pa_status_string(int status);

@@ -15,6 +15,7 @@ __all__ = [
     "make_cascade_workspace", "pa_prefill_chunk", "pa_workspace_bytes", "pa_decode_static_scratch",
     "pa_status_string", "pa_last_cuda_error", "pa_last_cuda_error_string", "PAError", "library_path",
     "make_workspace", "status_bit", "pa_plan_batch", "pa_prefill_chunk_planned", "Plan",
+    "pa_calibrate", "pa_calibration", "pa_calibration_clear", "pa_prefill_chunk_fp8",
 ]
 
 

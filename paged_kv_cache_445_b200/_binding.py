@@ -44,6 +44,9 @@ _lib.pa_cache_append_fp8.restype = _ci
 _lib.pa_decode_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
 _lib.pa_decode_fp8.restype = _ci
+_lib.pa_prefill_chunk_fp8.argtypes = [_vp, _vp, _i32p, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci, _ci,
+                                      ctypes.c_float, ctypes.c_float, ctypes.c_float, _vp, ctypes.c_size_t, _vp, _vp]
+_lib.pa_prefill_chunk_fp8.restype = _ci
 _lib.pa_decode_static_scratch.argtypes = [_vp, _vp, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                           ctypes.c_float, _vp, _vp]
 _lib.pa_decode_static_scratch.restype = _ci
@@ -62,6 +65,14 @@ _lib.pa_plan_batch.restype = _ci
 _lib.pa_prefill_chunk_planned.argtypes = [_vp, _vp, _i32p, _vp, _vp, _i32p, _ci, _i32p, _ci, _ci, _ci, _ci, _ci, _ci,
                                           _ci, ctypes.c_float, _vp, ctypes.c_size_t, ctypes.POINTER(Plan), _vp, _vp]
 _lib.pa_prefill_chunk_planned.restype = _ci
+_lib.pa_calibrate_bytes.argtypes = []
+_lib.pa_calibrate_bytes.restype = ctypes.c_size_t
+_lib.pa_calibrate.argtypes = [_vp, ctypes.c_size_t, _vp, _vp]
+_lib.pa_calibrate.restype = _ci
+_lib.pa_calibration.argtypes = [ctypes.POINTER(_ci), _vp]
+_lib.pa_calibration.restype = _ci
+_lib.pa_calibration_clear.argtypes = []
+_lib.pa_calibration_clear.restype = None
 _lib.pa_last_cuda_error.argtypes = []
 _lib.pa_last_cuda_error.restype = _ci
 _lib.pa_last_cuda_error_string.argtypes = []
@@ -315,6 +326,29 @@ def _host_i32(a, name):
     return a
 
 
+def pa_prefill_chunk_fp8(out, q, query_start, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale,
+                         workspace, dev_status=None, stream=None) -> None:
+    """pa_prefill_chunk over E4M3 caches (uint8 [num_blocks, Hkv, block_size, d])
+    with per-tensor scales, as pa_decode_fp8."""
+    op = _dev(out, "out", torch.bfloat16, 3)
+    qp = _dev(q, "q", torch.bfloat16, 3)
+    kc = _dev(k_cache, "k_cache", torch.uint8, 4)
+    vc = _dev(v_cache, "v_cache", torch.uint8, 4)
+    bt = _dev(block_tables, "block_tables", torch.int32, 2)
+    cl = _dev(context_lens, "context_lens", torch.int32, 1)
+    qs = _dev(query_start, "query_start", torch.int32, 1)
+    ws = _dev(workspace, "workspace", torch.uint8, 1)
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or k_cache.shape[3] != q.shape[2]:
+        raise ValueError("out/q [Tq, Hq, d] and caches [num_blocks, Hkv, block_size, d] must agree")
+    if query_start.shape[0] != context_lens.shape[0] + 1 or block_tables.shape[0] != context_lens.shape[0]:
+        raise ValueError("query_start must have num_seqs + 1 entries, one table row per sequence")
+    nb, hkv, bs, d = k_cache.shape
+    _check(_lib.pa_prefill_chunk_fp8(op, qp, qs, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0],
+                                     q.shape[0], q.shape[1], hkv, d, bs, nb, float(scale), float(k_scale),
+                                     float(v_scale), ws, workspace.numel(), _status_ptr(dev_status),
+                                     _stream_ptr(stream)))
+
+
 def pa_plan_batch(query_start, context_lens, num_q_heads: int, num_kv_heads: int, head_dim: int, block_size: int,
                   max_blocks_per_seq: int) -> Plan:
     """Host plan of a varlen batch from HOST copies of query_start [B + 1] and
@@ -344,6 +378,39 @@ def pa_prefill_chunk_planned(out, q, query_start, k_cache, v_cache, block_tables
     _check(_lib.pa_prefill_chunk_planned(op, qp, qs, kc, vc, bt, block_tables.shape[1], cl, context_lens.shape[0],
                                          q.shape[0], q.shape[1], hkv, d, bs, nb, float(scale), ws, workspace.numel(),
                                          ctypes.byref(plan), _status_ptr(dev_status), _stream_ptr(stream)))
+
+
+def pa_calibrate(buffer: torch.Tensor | None = None, dev_status=None, stream=None) -> list[int]:
+    """Time the decode kernel on every SM of the current device and keep per-SM
+    weights for its split of the work; returns the weights.  ``buffer``: a
+    CUDA tensor of at least pa_calibrate_bytes() bytes (overwritten); one is
+    allocated for the call if None.  Waits for its own work."""
+    need = int(_lib.pa_calibrate_bytes())
+    if need == 0:
+        raise PAError(PA_ERR_CUDA, "no CUDA device")
+    if buffer is None:
+        buffer = torch.empty(need, dtype=torch.uint8, device="cuda")
+    if not buffer.is_cuda or not buffer.is_contiguous():
+        raise ValueError("buffer must be a contiguous CUDA tensor")
+    _check(_lib.pa_calibrate(buffer.data_ptr(), buffer.numel() * buffer.element_size(), _status_ptr(dev_status),
+                             _stream_ptr(stream)))
+    return pa_calibration()
+
+
+def pa_calibration() -> list[int]:
+    """The per-SM rates recorded for the current device ([] if none)."""
+    n = _ci(0)
+    rates = (ctypes.c_uint16 * 256)()
+    rc = _lib.pa_calibration(ctypes.byref(n), rates)
+    if rc == PA_ERR_RANGE:
+        return []
+    _check(rc)
+    return list(rates[:n.value])
+
+
+def pa_calibration_clear() -> None:
+    """Forget every device's rates: decode splits its work equally again."""
+    _lib.pa_calibration_clear()
 
 
 def pa_decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale, dev_status=None,
@@ -379,4 +446,5 @@ def exported_symbols() -> list[str]:
     return ["pa_cache_append", "pa_workspace_bytes", "pa_decode", "pa_decode_append", "pa_cache_append_fp8",
             "pa_decode_fp8", "pa_cascade_workspace_bytes", "pa_decode_cascade", "pa_prefill_chunk",
             "pa_decode_static_scratch", "pa_status_string", "pa_last_cuda_error", "pa_last_cuda_error_string",
-            "pa_plan_batch", "pa_prefill_chunk_planned"]
+            "pa_plan_batch", "pa_prefill_chunk_planned", "pa_prefill_chunk_fp8", "pa_calibrate_bytes", "pa_calibrate", "pa_calibration",
+            "pa_calibration_clear"]

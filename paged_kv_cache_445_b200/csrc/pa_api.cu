@@ -170,7 +170,7 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                          void* workspace, size_t workspace_bytes, int* dev_status, void* stream,
                          const void* k_new, const void* v_new, const int32_t* group_start,
                          const int32_t* group_prefix, int num_groups, int kv_fp8, float k_scale, float v_scale,
-                         const int32_t* plan) {
+                         const int32_t* plan, const RowsOverride* ovr) {
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace) return PA_ERR_NULL;
   if ((k_new == nullptr) != (v_new == nullptr)) return PA_ERR_NULL;
   if (k_new && query_start) return PA_ERR_UNSUPPORTED;  // the fused append serves one-row (decode) batches
@@ -242,6 +242,20 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
     p.v_inv_scale = 1.f / v_scale;
   }
   rows_workspace_layout(workspace, total_q_tokens, num_q_heads, num_kv_heads, head_dim, max_keys, di.num_sms, &p);
+  p.num_sms = di.num_sms;
+  p.weighted = di.num_sms <= PA_MAX_WEIGHTED_SMS && sm_rates_snapshot(p.sm_rate, di.num_sms) ? 1 : 0;
+  if (ovr) {
+    p.trace = ovr->trace;
+    if (ovr->weighted == 0) p.weighted = 0;
+    if (ovr->weighted == 1 && ovr->sm_rate && di.num_sms <= PA_MAX_WEIGHTED_SMS) {
+      p.weighted = 1;
+      for (int i = 0; i < di.num_sms; ++i) p.sm_rate[i] = ovr->sm_rate[i];
+    }
+  }
+  if (p.weighted) {  // prefix sums for a whole-GPU launch: each CTA then needs two words
+    p.sm_prefix[0] = 0;
+    for (int i = 0; i < di.num_sms; ++i) p.sm_prefix[i + 1] = p.sm_prefix[i] + p.sm_rate[i];
+  }
   p.status = dev_status;
   p.k_new = k_new;
   p.v_new = v_new;
@@ -352,14 +366,15 @@ size_t decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, i
 
 namespace {
 // Per-SM rates of the kernels on a B200, used only to share the SMs between
-// the decode rows and the chunk rows of one batch (measured: an 8-warp decode
-// CTA streams about 150 GB/s of KV when few SMs load HBM, the decode rows of
-// a whole GPU about 6.2 TB/s, the tcgen05 chunk kernel about 6.5 TFLOP/s per
-// SM).  A split is used when its model time beats running the two kernels
-// one after the other on the whole GPU by 5 %.
-constexpr double DECODE_BYTES_PER_S_PER_SM = 150e9;
+// the decode rows and the chunk rows of one batch (measured beside each
+// other on the mixed 512-token chunk + 127 decodes batch: an 8-warp decode
+// CTA streams about 65 GB/s of KV, the tcgen05 chunk kernel about 6.8
+// TFLOP/s per SM; the decode rows of a whole GPU about 6.2 TB/s).  A split
+// is used when its model time beats running the two kernels one after the
+// other on the whole GPU by 5 %.
+constexpr double DECODE_BYTES_PER_S_PER_SM = 65e9;
 constexpr double DECODE_BYTES_PER_S_ALL = 6.2e12;
-constexpr double CHUNK_FLOPS_PER_S_PER_SM = 6.5e12;
+constexpr double CHUNK_FLOPS_PER_S_PER_SM = 6.8e12;
 
 int plan_split(double decode_bytes, double chunk_flops, int num_sms) {
   const double serial = decode_bytes / DECODE_BYTES_PER_S_ALL + chunk_flops / (num_sms * CHUNK_FLOPS_PER_S_PER_SM);
@@ -545,6 +560,18 @@ int pa_decode_fp8(void* out, const void* q, const void* k_new, const void* v_new
                            num_seqs, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                            workspace, workspace_bytes, dev_status, stream, k_new, v_new, nullptr, nullptr, 0, 1,
                            k_scale, v_scale);
+}
+
+int pa_prefill_chunk_fp8(void* out, const void* q, const int32_t* query_start, const void* k_cache,
+                         const void* v_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                         const int32_t* context_lens, int num_seqs, int total_q_tokens, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, float k_scale,
+                         float v_scale, void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  if (!query_start) return PA_ERR_NULL;
+  return pa::run_attention(out, q, query_start, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                           num_seqs, total_q_tokens, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                           scale, workspace, workspace_bytes, dev_status, stream, nullptr, nullptr, nullptr, nullptr,
+                           0, 1, k_scale, v_scale);
 }
 
 int pa_prefill_chunk(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,

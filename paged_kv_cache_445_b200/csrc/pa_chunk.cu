@@ -75,6 +75,7 @@ constexpr uint32_t TMEM_COLS = 512;                           // S_A, S_B, O_A, 
 constexpr uint32_t TMEM_O = 256;                              // O of M-tile w at TMEM_O + 128 w
 constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when the max rises by > 2^8
 constexpr int SLOT_STRIDE = CH_D + 4;  // piece slot row: O[128], m, l, 2 floats of padding
+constexpr int MIN_UNITS_PER_CTA = 4;   // key tiles
 // Register split (setmaxnreg): the launch gives 168 per thread (65,536 / 384,
 // rounded down to 8); warpgroup 0 drops to 80, the softmax warpgroups rise to
 // 208: 128 x 80 + 256 x 208 = 63,488 <= 384 x 168 = 64,512, the launch's total
@@ -247,9 +248,13 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
   if (!p.dep_at_end) grid_dependency_wait();
 
   // this CTA's contiguous range [ua, ub) of the batch's (item, key tile) units
+  // (at least MIN_UNITS_PER_CTA units per CTA: a small batch on fewer CTAs,
+  // so that its items are not cut into one-tile pieces; the others idle)
   const int units = sh.units;
-  const int ncta = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
-  const int ua = cta_range_start(units, cta, ncta), ub = cta_range_start(units, cta + 1, ncta);
+  const int ncta = max(1, min(static_cast<int>(gridDim.x), units / MIN_UNITS_PER_CTA));
+  const int cta = static_cast<int>(blockIdx.x);
+  const int ua = cta < ncta ? cta_range_start(units, cta, ncta) : units;
+  const int ub = cta < ncta ? cta_range_start(units, cta + 1, ncta) : units;
   if (warp < 4) {
     // ================================================================ warpgroup 0
     regs_dec<REGS_PRODUCER>();
@@ -454,14 +459,18 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       const bool row_valid = tok < it.qlen && last_key >= 0;
       const int tile_last = it.p0 + it.tp * PAIR + w * TOK;   // first row of this M-tile: keys beyond it are
                                                               // masked for some row of the tile
-      // a cut item: the CTAs c_first .. c_last hold its pieces; c_first's is
-      // the last piece of its range (slot 1) unless its range starts with it
+      // a cut item: the CTAs c_first .. c_last with a non-empty range hold its
+      // pieces (with more CTAs than units some ranges are empty); c_first's
+      // is the last piece of its range (slot 1) unless its range starts with
+      // the item, every later one is the first piece of its range (slot 0)
       const bool whole = j0 == 0 && j1 == nt;
-      int c_first = 0, c_last = 0, first_slot = 0;
+      int c_first = 0, c_last = 0, first_slot = 0, npieces = 0;
       if (!whole) {
         c_first = cta_of_unit(units, ubase, ncta);
         c_last = cta_of_unit(units, ubase + nt - 1, ncta);
         first_slot = cta_range_start(units, c_first, ncta) == ubase ? 0 : 1;
+        for (int c = c_first; c <= c_last; ++c)
+          npieces += cta_range_start(units, c + 1, ncta) > cta_range_start(units, c, ncta);
       }
       const int my_slot = (ubase + j0 == ua) ? 0 : 1;  // this CTA's first piece, or its last
       int* const cnt = p.counters + static_cast<long long>(idx) * (2 * CH_M) + w * CH_M + row;
@@ -628,17 +637,19 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       // One count per (item, row): the thread that lands a row's last piece
       // merges that row, with no wait on any other thread.
       __threadfence();
-      if (atomicAdd(cnt, 1) != c_last - c_first) continue;
+      if (atomicAdd(cnt, 1) != npieces - 1) continue;
       *cnt = 0;  // every piece of this row has arrived: back to zero for the next call
       __threadfence();
       // merge in CTA order: m = max m_k, out = sum_k 2^(m_k - m) O_k / sum_k 2^(m_k - m) l_k
       float mmax = -INFINITY, lsum = 0.f;
       for (int c = c_first; c <= c_last; ++c) {
+        if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
         const int sl = c == c_first ? first_slot : 0;
         const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
         mmax = fmaxf(mmax, __ldcg(src + CH_D));
       }
       for (int c = c_first; c <= c_last; ++c) {
+        if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
         const int sl = c == c_first ? first_slot : 0;
         const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
         const float2 ml = __ldcg(reinterpret_cast<const float2*>(src + CH_D));
@@ -652,6 +663,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) acc[i] = 0.f;
         for (int c = c_first; c <= c_last; ++c) {
+          if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
           const int sl = c == c_first ? first_slot : 0;
           const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
           const float mk = __ldcg(src + CH_D);

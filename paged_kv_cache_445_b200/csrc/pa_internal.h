@@ -55,6 +55,14 @@ int per_device(PerDevice& cache, Setup setup, int* out) {
   return PA_OK;
 }
 
+// SMs whose rates a decode launch can carry in its parameters.
+constexpr int PA_MAX_WEIGHTED_SMS = 160;
+
+// The per-SM rates pa_calibrate recorded for the current device (false if
+// none, or recorded for another SM count).
+bool sm_rates_snapshot(uint16_t* out, int num_sms);
+void sm_rates_clear();
+
 // Batch size up to which the rows kernel keeps per-sequence prefix sums of
 // tile counts in shared memory (larger batches scan context_lens instead).
 constexpr int ROWS_SMEM_SEQS_HOST = 1024;
@@ -87,6 +95,17 @@ struct RowsParams {
   int total_warps;
   int tile_shift;   // log2 of the keys per work unit (16, or 32 for the E4M3 kernel with one head tile)
   int trigger_early;  // 1: release the dependent grid (the chunk kernel beside this one) once the append is visible
+  // Split of the tiles by SM rate (pa_calibrate): each SM takes a share in
+  // proportion to sm_rate[smid], cut equally between its warps.
+  int weighted;
+  int num_sms;
+  int* sm_slots;          // workspace: CTAs that have taken their SM's share, per SM; zero between calls
+  unsigned* sm_mask;      // workspace: SMs of a launch on part of the GPU (8 words); zero between calls
+  uint16_t sm_rate[PA_MAX_WEIGHTED_SMS];
+  uint32_t sm_prefix[PA_MAX_WEIGHTED_SMS + 1];  // sm_prefix[s] = sum of sm_rate[0 .. s-1] (a whole-GPU launch)
+  // Calibration only (nullptr otherwise): per range r, {SM id, units, time of
+  // the first copy, time the last tile was consumed} (globaltimer ns).
+  unsigned long long* trace;
   // Fused cache append (decode only; nullptr: none).  Row s of k_new / v_new
   // ([B, Hkv, D] bf16) is sequence s's newest token: the kernel writes it to
   // position context_lens[s] - 1 through the block table and attends to it
@@ -276,6 +295,13 @@ enum PlanWord {
 constexpr int32_t PLAN_MAGIC_VALUE = 0x50414e31;  // "PAN1"
 constexpr int32_t PLAN_VERIFY32 = 1, PLAN_VERIFY64 = 2, PLAN_CHUNK = 4, PLAN_ROWS = 8;
 
+// What a calibration run of the decode kernel overrides.
+struct RowsOverride {
+  unsigned long long* trace;  // RowsParams::trace
+  int weighted;               // -1: the recorded rates, 0: equal split, 1: the rates below
+  const uint16_t* sm_rate;
+};
+
 // Argument checks, tensor maps and kernel dispatch shared by the attention
 // entry points (query_start == nullptr: one query row per sequence).
 int run_attention(void* out, const void* q, const int32_t* query_start, const void* k_cache, const void* v_cache,
@@ -284,7 +310,8 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
                   int num_blocks, float scale, void* workspace, size_t workspace_bytes, int* dev_status,
                   void* stream, const void* k_new = nullptr, const void* v_new = nullptr,
                   const int32_t* group_start = nullptr, const int32_t* group_prefix = nullptr, int num_groups = 0,
-                  int kv_fp8 = 0, float k_scale = 1.f, float v_scale = 1.f, const int32_t* plan = nullptr);
+                  int kv_fp8 = 0, float k_scale = 1.f, float v_scale = 1.f, const int32_t* plan = nullptr,
+                  const RowsOverride* ovr = nullptr);
 // Bytes of workspace a decode call (one query row per sequence) needs: the
 // rows kernel's part of pa_workspace_bytes.
 size_t decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,

@@ -537,7 +537,7 @@ constexpr int rows_ctas_per_sm() {
 template <int D, int NT, int R, bool F8, int TK, int NW>
 __global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 3 ? 3 : 1)
     rows_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
-                const RowsParams p) {
+                const __grid_constant__ RowsParams p) {
   static_assert(TK == TILE_KEYS || (TK == 2 * TILE_KEYS && F8 && D == 128 && NT == 1), "32-key tiles: E4M3, D 128, G <= 8");
   using S = RowsShape<D, NT, F8, TK>;
   constexpr int KT = S::KT;
@@ -552,6 +552,24 @@ __global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 
   uint8_t* base = align1024(smem_raw);
   const bool use_pfx = p.num_seqs <= ROWS_SMEM_SEQS;
   long long* pfx = use_pfx ? reinterpret_cast<long long*>(base + NW * R * S::STAGE_BYTES) : nullptr;
+
+  // Split by SM rate: this CTA's SM, registered at once so that the atomics'
+  // round trips overlap the prologue (their results are read after it).
+  const bool partial = p.weighted && static_cast<int>(gridDim.x) < p.num_sms;  // one CTA on each of some SMs
+  unsigned sm_id = 0;
+  int sm_claim = 0;
+  if (p.weighted && threadIdx.x == 0) {
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(sm_id));
+    if (sm_id < static_cast<unsigned>(p.num_sms)) {
+      if (partial) {
+        atomicOr(p.sm_mask + (sm_id >> 5), 1u << (sm_id & 31));
+        __threadfence();
+        atomicAdd(p.sched + 2, 1);
+      } else {
+        sm_claim = atomicAdd(p.sm_slots + sm_id, 1);  // which of the SM's CTAs this one is
+      }
+    }
+  }
 
   // ---- prologue: tiles of every sequence, their prefix sums, the total T.
   // Rows without a key are written as zeros here (each by one thread).
@@ -596,14 +614,92 @@ __global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 
     T = 0;
   }
 
-  const long long W = T < p.total_warps ? T : p.total_warps;
+  // ---- this warp's contiguous range [a, e) of the T units, and its index r
+  // among the ranges (its partial-result slots are 2r and 2r + 1)
+  long long ra = 0, re = 0;
+  int r_index = gw;
+  if (p.weighted && T > 0) {
+    // each SM takes a share of the units in proportion to its rate, cut
+    // equally between the warps of its CTAs; which CTA of an SM takes which
+    // part is decided by arrival (the parts, hence the result, do not depend
+    // on it)
+    __shared__ int sm_local, sm_ok;
+    __shared__ long long sm_lo, sm_all;
+    if (threadIdx.x == 0) {
+      const unsigned smid = sm_id;
+      sm_ok = smid < static_cast<unsigned>(p.num_sms);
+      if (partial && sm_ok) {  // wait (bounded) until every CTA has registered its SM
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(p.sched + 2) < static_cast<int>(gridDim.x)) {
+          if (globaltimer_ns() - t0 > WAIT_NS) {
+            set_status(p.status, PA_STATUS_BIT(PA_ERR_TIMEOUT));
+            sm_ok = 0;
+            break;
+          }
+          __nanosleep(64);
+        }
+      }
+      sm_local = (partial ? 0 : sm_claim) * 65536 + static_cast<int>(smid);  // (local index, SM id)
+      if (!partial && sm_ok) {  // a whole-GPU launch: the host's prefix sums
+        sm_lo = p.sm_prefix[smid];
+        sm_all = p.sm_prefix[p.num_sms];
+      }
+    }
+    if (partial) {  // the rates of the registered SMs only: a reduction over the CTA's threads
+      __syncthreads();
+      const unsigned me = static_cast<unsigned>(sm_local & 65535);
+      long long lo = 0, all = 0;
+      for (int q = threadIdx.x; q < p.num_sms; q += ROWS_THREADS) {
+        if (!((__ldcg(p.sm_mask + (q >> 5)) >> (q & 31)) & 1u)) continue;
+        all += p.sm_rate[q];
+        if (static_cast<unsigned>(q) < me) lo += p.sm_rate[q];
+      }
+      lo = warp_sum64(lo);
+      all = warp_sum64(all);
+      __shared__ long long red[2][NW];
+      if (lane == 0) {
+        red[0][warp] = lo;
+        red[1][warp] = all;
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        long long a0 = 0, a1 = 0;
+        for (int k = 0; k < NW; ++k) {
+          a0 += red[0][k];
+          a1 += red[1][k];
+        }
+        sm_lo = a0;
+        sm_all = a1;
+      }
+    }
+    __syncthreads();
+    if (sm_ok && sm_all > 0) {
+      const int smid = sm_local & 65535, local = sm_local >> 16;
+      const int cps = partial ? 1 : static_cast<int>(gridDim.x) / p.num_sms;  // CTAs on every SM
+      const int nsub = cps * NW, k = local * NW + warp;
+      const long long lo = T * sm_lo / sm_all, hi = T * (sm_lo + p.sm_rate[smid]) / sm_all;
+      ra = lo + (hi - lo) * k / nsub;
+      re = lo + (hi - lo) * (k + 1) / nsub;
+      r_index = smid * nsub + k;
+    } else {  // an SM outside the table (cannot happen on the device that recorded it): no share
+      ra = re = 0;
+      r_index = gw;
+      if (threadIdx.x == 0) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
+    }
+  } else {
+    const long long W = T < p.total_warps ? T : p.total_warps;
+    if (gw < W) {
+      ra = range_start(gw, T, W);
+      re = range_start(gw + 1, T, W);
+    }
+  }
   uint64_t* bar = bars[warp];
   TileMeta* meta = metas[warp];
   uint8_t* ring = base + static_cast<size_t>(warp) * R * S::STAGE_BYTES;
   long long issued = 0, stopped_at = -1;
   int nslots = 0;
 
-  if (gw < W) {
+  if (ra < re) {
     if (lane == 0) {
       prefetch_tmap(&tmk);
       prefetch_tmap(&tmv);
@@ -615,9 +711,10 @@ __global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 
     const uint64_t pol = policy_evict_first();
 
     // ---- producer: the load cursor walks the warp's range [a, e)
-    const long long a = range_start(gw, T, W), e = range_start(gw + 1, T, W);
+    const long long a = ra, e = re;
     Cursor lc;
     seek(p, pfx, a, lane, lc);
+    const unsigned long long t_first = p.trace ? globaltimer_ns() : 0;
     bool loading = true;
     BtWindow win;
     win.s = -1;
@@ -1125,7 +1222,7 @@ __global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 
         } else if (began && tm.t == tm.n - 1) {
           store_output<D, NT, F8>(p, o, l, tm.row, tm.h, lane);
         } else if (nslots < ROWS_SLOTS_PER_WARP) {
-          const long long slot = static_cast<long long>(gw) * ROWS_SLOTS_PER_WARP + nslots++;
+          const long long slot = static_cast<long long>(r_index) * ROWS_SLOTS_PER_WARP + nslots++;
           float* ps = p.partials + slot * S::SLOT_FLOATS;
 #pragma unroll
           for (int mt = 0; mt < KT; ++mt)
@@ -1156,15 +1253,34 @@ __global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 
       }
     }
 
+    if (p.trace && lane == 0) {  // calibration: when this warp's range streamed, and on which SM
+      unsigned smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      unsigned long long* tr = p.trace + static_cast<long long>(r_index) * 4;
+      tr[0] = smid;
+      tr[1] = static_cast<unsigned long long>(e - a);
+      tr[2] = t_first;
+      tr[3] = globaltimer_ns();
+    }
     if (stopped_at >= 0) {  // let copies still in flight land before the shared memory goes away
       for (long long j = stopped_at + 1; j < issued; ++j) mbar_wait(&bar[j % R], static_cast<uint32_t>((j / R) & 1));
     }
   }
 
-  if (gw >= W && p.k_new)  // warps without tiles still take their share of the fused append
+  if (!(ra < re) && p.k_new)  // warps without tiles still take their share of the fused append
     fused_append<D, F8>(p, static_cast<long long>(blockIdx.x) * ROWS_THREADS + threadIdx.x,
                     static_cast<long long>(gridDim.x) * ROWS_THREADS);
-  if (T == 0) return;  // no tile anywhere (every CTA sees the same T): nothing to merge, no barrier
+  if (T == 0) {  // no tile anywhere (every CTA sees the same T): nothing to merge, no barrier
+    if (p.weighted && threadIdx.x == 0 && sm_id < static_cast<unsigned>(p.num_sms)) {  // undo the registration
+      if (partial) {
+        atomicAnd(p.sm_mask + (sm_id >> 5), ~(1u << (sm_id & 31)));
+        atomicSub(p.sched + 2, 1);
+      } else {
+        atomicSub(p.sm_slots + sm_id, 1);
+      }
+    }
+    return;
+  }
 
   // ---- grid barrier: every partial and table entry is stored before any merge reads it
   __syncwarp();
@@ -1199,6 +1315,11 @@ __global__ void __launch_bounds__(NW * 32, rows_ctas_per_sm<D, NT, F8, TK>() == 
     if (out == p.total_warps - 1) {
       p.sched[0] = 0;
       p.sched[1] = 0;
+      if (p.weighted) {
+        p.sched[2] = 0;
+        for (int q = 0; q < 8; ++q) p.sm_mask[q] = 0;
+        for (int q = 0; q < p.num_sms; ++q) p.sm_slots[q] = 0;
+      }
     }
   }
 }
@@ -1264,7 +1385,10 @@ int rows_supported(int group, int head_dim) {
 
 namespace {
 size_t round256(size_t n) { return (n + 255) / 256 * 256; }
-constexpr size_t SCHED_BYTES = 256;
+// [0] warps at the barrier, [1] warps done, [2] CTAs of a partial launch that
+// have registered their SM, [8..15] their SM mask, [16..16 + 256) CTAs per SM
+// that have taken their share
+constexpr size_t SCHED_BYTES = 2048;
 size_t slot_bytes(int group, int head_dim) {
   const int nt = group > 8 ? 2 : 1;
   const size_t o = static_cast<size_t>(head_dim / 16) * nt * 32 * 4;
@@ -1304,6 +1428,8 @@ void rows_workspace_layout(void* ws, int num_rows, int num_q_heads, int num_kv_h
   (void)head_dim;
   uint8_t* b = static_cast<uint8_t*>(ws);
   p->sched = reinterpret_cast<int*>(b);
+  p->sm_mask = reinterpret_cast<unsigned*>(b) + 8;
+  p->sm_slots = reinterpret_cast<int*>(b) + 16;
   b += SCHED_BYTES;
   p->verify_counters = reinterpret_cast<int*>(b);
   b += verify_counter_bytes(num_sms);

@@ -164,6 +164,9 @@ def _lengths(cfg: int, rng: np.random.Generator):
     if cfg == 6:  # the 70B-like length mix, each sequence verifying 4 draft tokens
         ctx = np.clip(np.round(rng.lognormal(math.log(1500.0), 0.8, size=128)), 16, 8192).astype(np.int64)
         return tuple(ctx - 4), (4,) * 128
+    if cfg == 7:  # GRPO with long prompts: 8 prompts x 16 rollouts, 8192-token shared prefixes
+        tails = rng.integers(0, 1024, size=128, endpoint=True)
+        return tuple(8192 + tails), (1,) * 128
     raise ValueError(f"unknown workload {cfg}")
 
 
@@ -172,7 +175,9 @@ def standard_spec(cfg: int, seed: int | None = None) -> Spec:
     3 Llama-3.3-70B-like decode at concurrency 128, 4 GRPO shared-prefix decode,
     5 mixed 512-token prefill chunk + 127 decodes, 6 the workload-3 layer
     verifying 4 draft tokens per sequence, as speculative decoding does --
-    "Inference optimization", section "Speculative decoding")."""
+    "Inference optimization", section "Speculative decoding"; 7 the GRPO
+    shape with 8 prompts of 8192 tokens x 16 rollouts, whose shared prefixes
+    (268 MB of KV) no longer fit in the 126 MB L2)."""
     seed = 445 + cfg if seed is None else seed
     rng = np.random.Generator(np.random.PCG64(seed))
     prefix, new = _lengths(cfg, rng)
@@ -188,6 +193,9 @@ def standard_spec(cfg: int, seed: int | None = None) -> Spec:
                     share=groups, share_tokens=2048)
     if cfg == 5:
         return Spec("mixed-prefill512-plus-127-decodes", 64, 8, 128, 16, prefix, new)
+    if cfg == 7:
+        groups = tuple(tuple(range(16 * g, 16 * g + 16)) for g in range(8))
+        return Spec("grpo-long-prefix-decode-8x16", 24, 4, 256, 32, prefix, new, share=groups, share_tokens=8192)
     return Spec("llama3.3-70b-layer-verify4-b128", 64, 8, 128, 16, prefix, new, q_std=0.5)
 
 

@@ -76,7 +76,7 @@ def fake_device(monkeypatch):
 def _line(capsys, workload, **kw):
     args = argparse.Namespace(gpus=1, steps=4, warmup=3, workload=workload, impl="ours", cpu_seconds=0.2,
                               reference_seconds=1.0, no_cpu_baseline=True, kv_dtype="bf16", graph=False,
-                              cascade=False, separate_append=False, no_plan=False, no_sub_records=True,
+                              cascade=False, separate_append=False, no_plan=False, no_sub_records=True, no_calibrate=True,
                               sub_cpu_seconds=0.1)
     for k, v in kw.items():
         setattr(args, k, v)
@@ -115,8 +115,8 @@ def test_small_workload_runs_with_l2_flushed_and_times_the_oracle(fake_device, c
 def test_default_run_carries_the_other_workloads_as_sub_records(fake_device, capsys):
     d = _line(capsys, 3, no_sub_records=False)
     subs = d["workloads"]
-    assert set(subs) == {"grpo-shared-prefix", "grpo-shared-prefix-cascade", "mixed-chunk-decode",
-                         "llama3.3-70b-layer-decode-b128-fp8"}
+    assert set(subs) == {"grpo-shared-prefix", "grpo-shared-prefix-cascade", "grpo-long-prefix",
+                         "grpo-long-prefix-cascade", "mixed-chunk-decode", "llama3.3-70b-layer-decode-b128-fp8"}
     for key, sub in subs.items():
         for k in ("value", "unit", "ms_per_step", "dtype", "config", "roofline", "e2e", "gpu_launches", "clocks"):
             assert k in sub, (key, k)

@@ -115,3 +115,13 @@ def test_cascade_reports_a_context_inside_the_shared_prefix():
                          i32(gs), i32(gp), ws, dev_status=ds.status)
     torch.cuda.synchronize()
     assert int(ds.status.item()) & pa.status_bit(pa._binding.PA_ERR_RANGE)
+
+
+def test_long_prefix_grpo_workload_matches_oracle():
+    # 8 prompts x 16 rollouts sharing 8192-token prefixes (268 MB of shared
+    # KV, more than the L2 holds): every row against the oracle
+    w = workloads.standard(7, poison=True)
+    ds = DeviceStep(w)
+    _cascade(ds, fused=True)
+    assert int(ds.status.item()) == 0
+    compare(ds.out.float().cpu().numpy(), _ref(w), "long-prefix GRPO cascade")

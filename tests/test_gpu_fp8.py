@@ -129,3 +129,45 @@ def test_fp8_rejects_what_it_does_not_support():
     with pytest.raises(pa.PAError) as e:
         st.decode()
     assert e.value.code == pa._binding.PA_ERR_SHAPE
+
+
+FP8_VARLEN = [  # prefix list, qlen list, Hq, Hkv, d, bs
+    ([1000, 40, 300], [130, 1, 4], 16, 2, 128, 16),     # a chunk, a decode and a 4-row verification
+    ([0, 500, 17], [200, 1, 2], 8, 1, 128, 32),         # a prompt from position 0
+    ([700, 33], [64, 1], 12, 2, 256, 16),               # head_dim 256
+    ([64, 2000, 9], [3, 7, 1], 16, 1, 128, 16),         # G 16: two head tiles
+]
+
+
+@pytest.mark.parametrize("case", FP8_VARLEN, ids=lambda c: f"Hq{c[2]}-Hkv{c[3]}-d{c[4]}-q{max(c[1])}")
+def test_fp8_varlen_batches_match_the_oracle(case):
+    import paged_kv_cache_445_b200 as pa
+    prefix, qlen, hq, hkv, d, bs = case
+    w = workloads.custom(prefix, qlen, hq, hkv, d, bs, seed=sum(prefix) + d, poison=True)
+    st = Fp8Step(w, seed=9)
+    st.append()
+    d_ = st.ds
+    pa.pa_prefill_chunk_fp8(d_.out, d_.q, d_.query_start, st.kc, st.vc, d_.block_tables, d_.context_lens, w.scale,
+                            st.k_scale, st.v_scale, d_.workspace, d_.status)
+    torch.cuda.synchronize()
+    assert int(d_.status.item()) == 0
+    kc, vc = st.oracle_caches()
+    ref = oracle.paged_attention_fp8(w.q, kc, vc, w.block_tables, w.context_lens, w.query_start, w.scale,
+                                     st.k_scale, st.v_scale)
+    compare(d_.out.float().cpu().numpy(), ref, f"fp8 varlen {case}")
+
+
+def test_fp8_verify4_layer_matches_the_oracle_on_every_row():
+    import paged_kv_cache_445_b200 as pa
+    w = workloads.standard(6, poison=True)
+    st = Fp8Step(w, seed=6)
+    st.append()
+    d_ = st.ds
+    pa.pa_prefill_chunk_fp8(d_.out, d_.q, d_.query_start, st.kc, st.vc, d_.block_tables, d_.context_lens, w.scale,
+                            st.k_scale, st.v_scale, d_.workspace, d_.status)
+    torch.cuda.synchronize()
+    assert int(d_.status.item()) == 0
+    kc, vc = st.oracle_caches()
+    ref = oracle.paged_attention_fp8(w.q, kc, vc, w.block_tables, w.context_lens, w.query_start, w.scale,
+                                     st.k_scale, st.v_scale)
+    compare(d_.out.float().cpu().numpy(), ref, "fp8 verify-4 layer")

@@ -206,3 +206,22 @@ def test_plan_rejects_bad_arguments_before_touching_a_device():
     assert L.pa_plan_batch(bad, cl, 2, 8, 2, 128, 16, 8, C.byref(plan)) == b.PA_ERR_SHAPE
     assert L.pa_prefill_chunk_planned(4096, 4096, None, 4096, 4096, 4096, 4, 4096, 2, 6, 8, 2, 128, 16, 10, 0.1,
                                       4096, 1 << 20, C.byref(plan), None, None) == b.PA_ERR_NULL
+
+
+def test_calibrate_rejects_bad_arguments_before_touching_a_device():
+    from paged_kv_cache_445_b200 import _binding as b
+    L = b._lib
+    assert L.pa_calibrate(None, 1 << 31, None, None) == b.PA_ERR_NULL
+    assert L.pa_calibrate(4096 + 16, 1 << 31, None, None) == b.PA_ERR_SHAPE  # not 256-byte aligned
+
+
+def test_fp8_varlen_rejects_bad_arguments_before_touching_a_device():
+    from paged_kv_cache_445_b200 import _binding as b
+    L, f = b._lib, 4096
+
+    def call(qs=f, d=128, ks=0.5):
+        return L.pa_prefill_chunk_fp8(f, f, qs, f, f, f, 4, f, 2, 6, 8, 2, d, 16, 10, 0.1, ks, 0.25, f, 1 << 20,
+                                      None, None)
+    assert call(qs=None) == b.PA_ERR_NULL
+    assert call(d=64) == b.PA_ERR_UNSUPPORTED
+    assert call(ks=0.0) == b.PA_ERR_SHAPE
