@@ -365,11 +365,14 @@ PA_API int pa_decode_static_scratch(void* out, const void* q, const void* k_cach
  * shares the GPU waits for its slowest SMs.  pa_calibrate runs the decode
  * kernel on a synthetic batch (128 sequences x 2048 tokens, 64 query / 8 KV
  * heads, head_dim 128) held in `buffer`, times every SM's share, and adjusts
- * per-SM weights over four rounds until the SMs finish together.  Every later
- * decode launch on this device (pa_decode, pa_decode_append, pa_decode_fp8,
- * pa_decode_cascade and the decode rows of pa_prefill_chunk*) gives each SM
- * a share in proportion to its weight.  Not part of the pages' problem
- * statement: a B200 scheduling aid.
+ * per-SM weights over four rounds until the SMs finish together.  Later
+ * launches of the kernel variant that was timed (bf16 cache, head_dim 128, up
+ * to 8 query heads per KV head, spread over the whole GPU: pa_decode,
+ * pa_decode_append, pa_decode_cascade's private keys and the decode rows of
+ * an unplanned pa_prefill_chunk on such shapes) give each SM a share in
+ * proportion to its weight; the other variants keep equal shares (the
+ * weights made them slower).  Not part of the pages' problem statement: a
+ * B200 scheduling aid.
  *
  * buffer: device memory of at least pa_calibrate_bytes() bytes (about
  * 1.1 GB; 256-byte aligned), overwritten.  The call WAITS for its own work

@@ -1351,6 +1351,11 @@ static int launch_rows_t(const RowsParams& p0, const CUtensorMap& tmk, const CUt
   if (rc_setup != PA_OK) return rc_setup;
   RowsParams p = p0;
   p.tile_shift = TK == 32 ? 5 : 4;
+  // The per-SM weights hold for the variant they were measured with (bf16,
+  // head_dim 128, one head tile, two 4-warp CTAs per SM over the whole GPU):
+  // on the other variants they made steps slower (head_dim 256 by 10 %, the
+  // E4M3 kernel by 4 %), so those split equally.
+  if (!(D == 128 && NT == 1 && !F8 && NW == ROWS_WARPS && ctas <= 0)) p.weighted = 0;
   // ctas > 0: a launch on part of the GPU (one CTA per SM, the rest of the
   // SMs left to a kernel that runs beside it)
   const int grid = ctas > 0 ? (ctas < num_sms * blocks_per_sm ? ctas : num_sms * blocks_per_sm)

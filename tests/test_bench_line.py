@@ -62,13 +62,21 @@ class _Step:
         pass
 
 
+class _Stream:
+    def wait_event(self, ev):
+        pass
+
+
 @pytest.fixture
 def fake_device(monkeypatch):
+    import contextlib
     monkeypatch.setattr(bench, "dist_setup", lambda n: (0, 1, 0))
     monkeypatch.setattr(bench, "GpuStep", _Step)
     monkeypatch.setattr(torch.cuda, "Event", _Event)
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
-    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: None)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a, **k: _Stream())
+    monkeypatch.setattr(torch.cuda, "Stream", lambda *a, **k: _Stream())
+    monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
     monkeypatch.setattr(torch.Tensor, "pin_memory", lambda self: self)
     monkeypatch.setattr(bench, "FLUSH_BYTES", 1 << 20)
 
