@@ -76,6 +76,8 @@ constexpr uint32_t TMEM_O = 256;                              // O of M-tile w a
 constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when the max rises by > 2^8
 constexpr int SLOT_STRIDE = CH_D + 4;  // piece slot row: O[128], m, l, 2 floats of padding
 constexpr int MIN_UNITS_PER_CTA = 4;   // key tiles
+// What a CTA reads or writes once (Q tiles, piece slots) goes into L2 as
+// first to be evicted, ahead of the K/V tiles the other items re-read.
 // Register split (setmaxnreg): the launch gives 168 per thread (65,536 / 384,
 // rounded down to 8); warpgroup 0 drops to 80, the softmax warpgroups rise to
 // 208: 128 x 80 + 256 x 208 = 63,488 <= 384 x 168 = 64,512, the launch's total
@@ -98,6 +100,8 @@ struct Shared {
   int abort;
   int merge;        // this CTA landed the last piece of the item being finished
   int units;  // (item, key tile) units of the batch
+  int items;  // items with at least one key tile
+  int my_lo, my_hi;  // with no more items than CTAs: this CTA's item, as a unit range
 };
 
 }  // namespace
@@ -170,6 +174,32 @@ __device__ __forceinline__ bool chunk_unit_item(const ChunkParams& p, int pair_t
   return false;
 }
 
+// Items with at least one key tile, and the unit range of the c-th of them
+// (lo = hi = units if there is none).
+__device__ __forceinline__ void chunk_items(const ChunkParams& p, int pair_tok, int c, int& count, int& lo, int& hi) {
+  count = 0;
+  int base = 0;
+  lo = hi = -1;
+  const int cap = p.max_blocks * p.block_size;
+  for (int s = 0; s < p.num_seqs; ++s) {
+    const int q0 = __ldg(p.query_start + s), qlen = __ldg(p.query_start + s + 1) - q0;
+    if (qlen < p.min_qlen) continue;
+    const int ctx = min(__ldg(p.context_lens + s), cap);
+    for (int tp = 0; tp * pair_tok < qlen; ++tp) {
+      Item it;
+      fill_item(s, q0, qlen, ctx, tp, it);
+      const int n = item_tiles(it, pair_tok);
+      if (n == 0) continue;
+      for (int h = 0; h < p.num_kv_heads; ++h, ++count, base += n)
+        if (count == c) {
+          lo = base;
+          hi = base + n;
+        }
+    }
+  }
+  if (lo < 0) lo = hi = base;
+}
+
 // First unit of CTA c's range, and the CTA whose range holds unit u.
 __device__ __forceinline__ int cta_range_start(int units, int c, int ncta) {
   return static_cast<int>(static_cast<long long>(units) * c / ncta);
@@ -193,6 +223,62 @@ __device__ __forceinline__ bool ch_wait(Shared& sh, uint64_t* bar, uint32_t phas
         set_status(status, PA_STATUS_BIT(PA_ERR_TIMEOUT));
         return false;
       }
+    }
+  }
+}
+
+// Merge the pieces of one row of a cut item, held by the CTAs c_first ..
+// c_last with a non-empty range (slot first_slot for c_first, 0 for the
+// others), in CTA order: m = max m_k, out = sum_k 2^(m_k - m) O_k /
+// sum_k 2^(m_k - m) l_k; then write the bf16 row (orow == nullptr: a row past
+// the chunk, nothing to write).  Kept out of line: the rare path's registers
+// stay out of the softmax loop's allocation.
+__device__ __noinline__ void merge_row(const float* __restrict__ partials, int units, int ncta, int ubase, int c_first,
+                                       int c_last, int first_slot, int wrow, __nv_bfloat16* orow) {
+  float mmax = -INFINITY, lsum = 0.f;
+  for (int c = c_first; c <= c_last; ++c) {
+    if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
+    const int sl = c == c_first ? first_slot : 0;
+    const float* src = partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
+    mmax = fmaxf(mmax, __ldcg(src + CH_D));
+  }
+  for (int c = c_first; c <= c_last; ++c) {
+    if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;
+    const int sl = c == c_first ? first_slot : 0;
+    const float* src = partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(src + CH_D));
+    lsum += ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mmax) * ml.y;
+  }
+  if (!orow) return;
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll 1
+  for (int cc = 0; cc < CH_D / 32; ++cc) {
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    for (int c = c_first; c <= c_last; ++c) {
+      if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;
+      const int sl = c == c_first ? first_slot : 0;
+      const float* src = partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
+      const float mk = __ldcg(src + CH_D);
+      const float wk = mk == -INFINITY ? 0.f : fast_exp2(mk - mmax);
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src + cc * 32 + i));
+        acc[i] += wk * v4.x;
+        acc[i + 1] += wk * v4.y;
+        acc[i + 2] += wk * v4.z;
+        acc[i + 3] += wk * v4.w;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+      uint4 u4;
+      u4.x = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+      u4.y = pack_bf16x2(acc[i + 2] * inv, acc[i + 3] * inv);
+      u4.z = pack_bf16x2(acc[i + 4] * inv, acc[i + 5] * inv);
+      u4.w = pack_bf16x2(acc[i + 6] * inv, acc[i + 7] * inv);
+      *reinterpret_cast<uint4*>(orow + cc * 32 + i) = u4;
     }
   }
 }
@@ -230,6 +316,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
     const long long u_all = chunk_units(p, PAIR);
     if (u_all > 0x7fffffffLL) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));  // far beyond any real batch
     sh.units = u_all > 0x7fffffffLL ? 0 : static_cast<int>(u_all);
+    // with no more items than CTAs every CTA takes one whole item: no item is
+    // cut, and the CTAs of a KV head walk its key tiles in step (each tile
+    // crosses HBM once and is then read from L2 by the others)
+    chunk_items(p, PAIR, static_cast<int>(blockIdx.x), sh.items, sh.my_lo, sh.my_hi);
     fence_mbar_init();
   }
   if (warp == 1) {  // tensor memory: S_A, S_B, O_A, O_B
@@ -251,10 +341,11 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
   // (at least MIN_UNITS_PER_CTA units per CTA: a small batch on fewer CTAs,
   // so that its items are not cut into one-tile pieces; the others idle)
   const int units = sh.units;
+  const bool whole_items = sh.items <= static_cast<int>(gridDim.x);
   const int ncta = max(1, min(static_cast<int>(gridDim.x), units / MIN_UNITS_PER_CTA));
   const int cta = static_cast<int>(blockIdx.x);
-  const int ua = cta < ncta ? cta_range_start(units, cta, ncta) : units;
-  const int ub = cta < ncta ? cta_range_start(units, cta + 1, ncta) : units;
+  const int ua = whole_items ? sh.my_lo : cta < ncta ? cta_range_start(units, cta, ncta) : units;
+  const int ub = whole_items ? sh.my_hi : cta < ncta ? cta_range_start(units, cta + 1, ncta) : units;
   if (warp < 4) {
     // ================================================================ warpgroup 0
     regs_dec<REGS_PRODUCER>();
@@ -296,10 +387,11 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       if (lane == 0) {
         const int t0 = it.q0 + it.tp * PAIR;
         mbar_arrive_expect_tx(&sh.q_full, 2 * Q_BYTES);
-        tma_load_3d(smem + SMEM_Q, &tmq, &sh.q_full, 0, it.kvh * G, t0);
-        tma_load_3d(smem + SMEM_Q + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0);
-        tma_load_3d(smem + SMEM_Q + Q_BYTES, &tmq, &sh.q_full, 0, it.kvh * G, t0 + TOK);
-        tma_load_3d(smem + SMEM_Q + Q_BYTES + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0 + TOK);
+        const uint64_t qpol = policy_evict_first();
+        tma_load_3d_hint(smem + SMEM_Q, &tmq, &sh.q_full, 0, it.kvh * G, t0, qpol);
+        tma_load_3d_hint(smem + SMEM_Q + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0, qpol);
+        tma_load_3d_hint(smem + SMEM_Q + Q_BYTES, &tmq, &sh.q_full, 0, it.kvh * G, t0 + TOK, qpol);
+        tma_load_3d_hint(smem + SMEM_Q + Q_BYTES + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0 + TOK, qpol);
       }
       auto load_tile = [&](const CUtensorMap* tm, uint64_t* bars_full, uint64_t* bars_empty, int nst, int base_off,
                            uint32_t t, int blk, int y) -> bool {
@@ -459,21 +551,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       const bool row_valid = tok < it.qlen && last_key >= 0;
       const int tile_last = it.p0 + it.tp * PAIR + w * TOK;   // first row of this M-tile: keys beyond it are
                                                               // masked for some row of the tile
-      // a cut item: the CTAs c_first .. c_last with a non-empty range hold its
-      // pieces (with more CTAs than units some ranges are empty); c_first's
-      // is the last piece of its range (slot 1) unless its range starts with
-      // the item, every later one is the first piece of its range (slot 0)
-      const bool whole = j0 == 0 && j1 == nt;
-      int c_first = 0, c_last = 0, first_slot = 0, npieces = 0;
-      if (!whole) {
-        c_first = cta_of_unit(units, ubase, ncta);
-        c_last = cta_of_unit(units, ubase + nt - 1, ncta);
-        first_slot = cta_range_start(units, c_first, ncta) == ubase ? 0 : 1;
-        for (int c = c_first; c <= c_last; ++c)
-          npieces += cta_range_start(units, c + 1, ncta) > cta_range_start(units, c, ncta);
-      }
-      const int my_slot = (ubase + j0 == ua) ? 0 : 1;  // this CTA's first piece, or its last
-      int* const cnt = p.counters + static_cast<long long>(idx) * (2 * CH_M) + w * CH_M + row;
+
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = j0; j < j1 && ok; ++j) {
@@ -590,7 +668,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       tc_fence_after();
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
                             (static_cast<long long>(it.q0 + tok) * p.num_q_heads + it.kvh * G + head_in_group) * CH_D;
-      if (whole) {  // the whole item: O / l -> bf16 -> out
+      if (j0 == 0 && j1 == nt) {  // the whole item: O / l -> bf16 -> out
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
         for (int c = 0; c < CH_D / 32; ++c) {
@@ -619,9 +697,15 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         continue;
       }
       // ---- a piece of a cut item: the unnormalised (O, m, l) of this row go
-      // to this CTA's slot (0: the first piece of its range, 1: the last)
+      // to this CTA's slot (0: the first piece of its range, 1: the last).
+      // The CTAs c_first .. c_last with a non-empty range hold the item's
+      // pieces (with more CTAs than units some ranges are empty); c_first's is
+      // the last piece of its range (slot 1) unless its range starts with the
+      // item, every later one the first piece of its range (slot 0).
+      const int my_slot = (ubase + j0 == ua) ? 0 : 1;
       const int wrow = w * CH_M + row;  // row of the item (both M-tiles)
       float* dst = p.partials + ((static_cast<long long>(cta) * 2 + my_slot) * 2 * CH_M + wrow) * SLOT_STRIDE;
+      const uint64_t spol = policy_evict_first();
 #pragma unroll
       for (int c = 0; c < CH_D / 32; ++c) {
         float v[32];
@@ -629,7 +713,8 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
-          __stcg(reinterpret_cast<float4*>(dst + c * 32 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+          st_global_hint(reinterpret_cast<float4*>(dst + c * 32 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]),
+                         spol);
       }
       __stcg(reinterpret_cast<float2*>(dst + CH_D), make_float2(m_ref, l));
       tc_fence_before();
@@ -637,56 +722,16 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       // One count per (item, row): the thread that lands a row's last piece
       // merges that row, with no wait on any other thread.
       __threadfence();
+      const int c_first = cta_of_unit(units, ubase, ncta), c_last = cta_of_unit(units, ubase + nt - 1, ncta);
+      const int first_slot = cta_range_start(units, c_first, ncta) == ubase ? 0 : 1;
+      int npieces = 0;
+      for (int c = c_first; c <= c_last; ++c)
+        npieces += cta_range_start(units, c + 1, ncta) > cta_range_start(units, c, ncta);
+      int* const cnt = p.counters + static_cast<long long>(idx) * (2 * CH_M) + wrow;
       if (atomicAdd(cnt, 1) != npieces - 1) continue;
       *cnt = 0;  // every piece of this row has arrived: back to zero for the next call
       __threadfence();
-      // merge in CTA order: m = max m_k, out = sum_k 2^(m_k - m) O_k / sum_k 2^(m_k - m) l_k
-      float mmax = -INFINITY, lsum = 0.f;
-      for (int c = c_first; c <= c_last; ++c) {
-        if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
-        const int sl = c == c_first ? first_slot : 0;
-        const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
-        mmax = fmaxf(mmax, __ldcg(src + CH_D));
-      }
-      for (int c = c_first; c <= c_last; ++c) {
-        if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
-        const int sl = c == c_first ? first_slot : 0;
-        const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(src + CH_D));
-        lsum += ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mmax) * ml.y;
-      }
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-      if (!row_valid) continue;
-#pragma unroll 1
-      for (int cc = 0; cc < CH_D / 32; ++cc) {
-        float acc[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-        for (int c = c_first; c <= c_last; ++c) {
-          if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
-          const int sl = c == c_first ? first_slot : 0;
-          const float* src = p.partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
-          const float mk = __ldcg(src + CH_D);
-          const float wk = mk == -INFINITY ? 0.f : fast_exp2(mk - mmax);
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 v4 = __ldcg(reinterpret_cast<const float4*>(src + cc * 32 + i));
-            acc[i] += wk * v4.x;
-            acc[i + 1] += wk * v4.y;
-            acc[i + 2] += wk * v4.z;
-            acc[i + 3] += wk * v4.w;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          uint4 u4;
-          u4.x = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
-          u4.y = pack_bf16x2(acc[i + 2] * inv, acc[i + 3] * inv);
-          u4.z = pack_bf16x2(acc[i + 4] * inv, acc[i + 5] * inv);
-          u4.w = pack_bf16x2(acc[i + 6] * inv, acc[i + 7] * inv);
-          *reinterpret_cast<uint4*>(orow + cc * 32 + i) = u4;
-        }
-      }
+      merge_row(p.partials, units, ncta, ubase, c_first, c_last, first_slot, wrow, row_valid ? orow : nullptr);
     }
   }
 

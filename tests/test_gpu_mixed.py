@@ -57,23 +57,35 @@ def test_planned_mixed_batch_shares_the_gpu_and_matches_the_oracle_on_every_row(
     assert torch.equal(first.view(torch.int16), ds.out.view(torch.int16))
 
 
-def test_one_chunk_item_cut_into_many_pieces_merges_exactly():
-    # one item (a 128-token chunk at G 8 is one pair of M-tiles) over 20,000
-    # keys = 157 key tiles, on the whole GPU: nearly every CTA holds one piece
+def test_chunk_items_cut_between_ctas_merge_exactly():
+    # more items than CTAs: 20 pairs of M-tiles x 8 KV heads = 160 items of
+    # about 13 key tiles on the whole GPU, split into equal unit ranges, so
+    # items are cut at CTA boundaries and merged from their pieces
+    w = workloads.custom([1000], [640], 64, 8, 128, 16, seed=61, poison=True)
+    ds = DeviceStep(w)
+    ds.append()
+    ref = _ref(w)
+    outs = []
+    for _ in range(3):
+        ds.attend()
+        torch.cuda.synchronize()
+        assert int(ds.status.item()) == 0
+        outs.append(ds.out.clone())
+    compare(outs[0].float().cpu().numpy(), ref, "160 items cut between CTAs")
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
+def test_fewer_items_than_ctas_run_whole():
+    # one or two items over 20,000 keys (157 key tiles): each on one CTA
     for hkv in (1, 2):
         w = workloads.custom([20000 - 128], [128], 8 * hkv, hkv, 128, 16, seed=51 + hkv, poison=True)
         ds = DeviceStep(w)
         ds.append()
-        ref = _ref(w)
-        outs = []
-        for _ in range(3):
-            ds.attend()
-            torch.cuda.synchronize()
-            assert int(ds.status.item()) == 0
-            outs.append(ds.out.clone())
-        compare(outs[0].float().cpu().numpy(), ref, f"one item in many pieces, Hkv {hkv}")
-        for o in outs[1:]:
-            assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+        ds.attend()
+        torch.cuda.synchronize()
+        assert int(ds.status.item()) == 0
+        compare(ds.out.float().cpu().numpy(), _ref(w), f"whole items, Hkv {hkv}")
 
 
 PLANNED = [  # prefix list, qlen list, Hq, Hkv, d, bs
