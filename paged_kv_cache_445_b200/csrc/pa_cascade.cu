@@ -124,6 +124,12 @@ __device__ __forceinline__ bool cs_wait(CShared& sh, uint64_t* bar, uint32_t pha
   }
 }
 
+// The MMA warp's waits: one answer for the whole warp, which stays converged
+// for the predicated MMA issue.
+__device__ __forceinline__ bool cs_wait_warp(CShared& sh, uint64_t* bar, uint32_t phase, int* status) {
+  return __all_sync(FULL_MASK, cs_wait(sh, bar, phase, status));
+}
+
 template <int D>
 __global__ void __launch_bounds__(CS_THREADS, 1)
     cascade_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -242,10 +248,10 @@ __global__ void __launch_bounds__(CS_THREADS, 1)
       CItem it;
       if (!cascade_item(p, tokm, idx, it, nullptr)) break;
       const int nt = it.nt;
-      if (!cs_wait(sh, &sh.q_full, q_phase, p.status)) break;
+      if (!cs_wait_warp(sh, &sh.q_full, q_phase, p.status)) break;
       q_phase ^= 1;
       if (!first_item) {  // the epilogue of the previous item has read O
-        if (!cs_wait(sh, &sh.o_empty, o_phase, p.status)) break;
+        if (!cs_wait_warp(sh, &sh.o_empty, o_phase, p.status)) break;
         o_phase ^= 1;
       }
       first_item = false;
@@ -253,40 +259,34 @@ __global__ void __launch_bounds__(CS_THREADS, 1)
       // it handed over P(j - 2), and no MMA reads S
       auto qk = [&](int j) -> bool {
         const int stage = (kv_count + j) % CS_KST;
-        if (!cs_wait(sh, &sh.k_full[stage], ((kv_count + j) / CS_KST) & 1, p.status)) return false;
+        if (!cs_wait_warp(sh, &sh.k_full[stage], ((kv_count + j) / CS_KST) & 1, p.status)) return false;
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sk = smem_u32(smem + S::SMEM_K + stage * S::KV_BYTES);
+        const uint32_t sk = smem_u32(smem + S::SMEM_K + stage * S::KV_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_f16(tmem + (j & 1) * CS_N, umma_desc(sq + (kk >> 2) * S::Q_PANEL + (kk & 3) * 32, 16, 1024),
-                     umma_desc(sk + (kk >> 2) * S::KV_PANEL + (kk & 3) * 32, 16, 1024), idesc_qk, kk > 0);
-          umma_commit(&sh.s_full[j & 1]);
-          umma_commit(&sh.k_empty[stage]);
-          if (j == nt - 1) umma_commit(&sh.q_empty);
-        }
-        __syncwarp();
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_f16(tmem + (j & 1) * CS_N, umma_desc(sq + (kk >> 2) * S::Q_PANEL + (kk & 3) * 32, 16, 1024),
+                   umma_desc(sk + (kk >> 2) * S::KV_PANEL + (kk & 3) * 32, 16, 1024), idesc_qk, kk > 0);
+        umma_commit(&sh.s_full[j & 1]);
+        umma_commit(&sh.k_empty[stage]);
+        if (j == nt - 1) umma_commit(&sh.q_empty);
         return true;
       };
       auto pv = [&](int j) -> bool {
-        if (!cs_wait(sh, &sh.p_full, p_phase, p.status)) return false;
+        if (!cs_wait_warp(sh, &sh.p_full, p_phase, p.status)) return false;
         p_phase ^= 1;
         const int stage = (kv_count + j) % CS_VST;
-        if (!cs_wait(sh, &sh.v_full[stage], ((kv_count + j) / CS_VST) & 1, p.status)) return false;
+        if (!cs_wait_warp(sh, &sh.v_full[stage], ((kv_count + j) / CS_VST) & 1, p.status)) return false;
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sv = smem_u32(smem + S::SMEM_V + stage * S::KV_BYTES);
+        const uint32_t sv = smem_u32(smem + S::SMEM_V + stage * S::KV_BYTES);
 #pragma unroll
-          for (int nb = 0; nb < D / PV_N; ++nb)  // O columns [PV_N nb, PV_N (nb + 1)): V panels 2 nb, 2 nb + 1
+        for (int nb = 0; nb < D / PV_N; ++nb)  // O columns [PV_N nb, PV_N (nb + 1)): V panels 2 nb, 2 nb + 1
 #pragma unroll
-            for (int kk = 0; kk < CS_N / 16; ++kk)  // keys 16kk..: P columns 8kk.., V rows 16kk..
-              umma_f16_ts(tmem + S::TMEM_O + nb * PV_N, tmem + S::TMEM_P + (j & 1) * (CS_N / 2) + 8 * kk,
-                          umma_desc(sv + nb * (PV_N / 64) * S::KV_PANEL + kk * 16 * 128, S::KV_PANEL, 1024),
-                          idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&sh.pv_done);
-          umma_commit(&sh.v_empty[stage]);
-        }
-        __syncwarp();
+          for (int kk = 0; kk < CS_N / 16; ++kk)  // keys 16kk..: P columns 8kk.., V rows 16kk..
+            umma_f16_ts(tmem + S::TMEM_O + nb * PV_N, tmem + S::TMEM_P + (j & 1) * (CS_N / 2) + 8 * kk,
+                        umma_desc(sv + nb * (PV_N / 64) * S::KV_PANEL + kk * 16 * 128, S::KV_PANEL, 1024), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&sh.pv_done);
+        umma_commit(&sh.v_empty[stage]);
         return true;
       };
       bool ok = qk(0);
@@ -418,8 +418,8 @@ __global__ void __launch_bounds__(CS_THREADS, 1)
 
   // ---- teardown: drain this CTA's tensor-core work, then free tensor memory
   if (warp == 1) {
-    if (lane == 0) umma_commit(&sh.drain);
     __syncwarp();
+    umma_commit(&sh.drain);  // arrives once every MMA issued by lane 0 has completed
     mbar_wait(&sh.drain, 0);
   }
   tc_fence_before();

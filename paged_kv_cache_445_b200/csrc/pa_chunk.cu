@@ -79,10 +79,10 @@ constexpr int MIN_UNITS_PER_CTA = 4;   // key tiles
 // What a CTA reads or writes once (Q tiles, piece slots) goes into L2 as
 // first to be evicted, ahead of the K/V tiles the other items re-read.
 // Register split (setmaxnreg): the launch gives 168 per thread (65,536 / 384,
-// rounded down to 8); warpgroup 0 drops to 80, the softmax warpgroups rise to
-// 208: 128 x 80 + 256 x 208 = 63,488 <= 384 x 168 = 64,512, the launch's total
-// (a larger sum would make setmaxnreg.inc wait forever).
-constexpr int REGS_LAUNCH = 168, REGS_PRODUCER = 80, REGS_SOFTMAX = 208;
+// rounded down to 8); warpgroup 0 drops to 104, the softmax warpgroups rise to
+// 200: 128 x 104 + 256 x 200 = 64,512 = 384 x 168, the launch's total (a
+// larger sum would make setmaxnreg.inc wait forever).  Neither side spills.
+constexpr int REGS_LAUNCH = 168, REGS_PRODUCER = 104, REGS_SOFTMAX = 200;
 static_assert(128 * REGS_PRODUCER + 256 * REGS_SOFTMAX <= CH_THREADS * REGS_LAUNCH, "register split");
 
 struct Item {
@@ -225,6 +225,12 @@ __device__ __forceinline__ bool ch_wait(Shared& sh, uint64_t* bar, uint32_t phas
       }
     }
   }
+}
+
+// The MMA warp's waits: every lane polls, and the warp takes one answer (so
+// the warp stays converged for the predicated MMA issue that follows).
+__device__ __forceinline__ bool ch_wait_warp(Shared& sh, uint64_t* bar, uint32_t phase, int* status) {
+  return __all_sync(FULL_MASK, ch_wait(sh, bar, phase, status));
 }
 
 // Merge the pieces of one row of a cut item, held by the CTAs c_first ..
@@ -451,21 +457,19 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       const int j0 = u - ubase;
       const int j1 = ub - ubase < nt ? ub - ubase : nt;
       u = ubase + j1;
-      if (!ch_wait(sh, &sh.q_full, q_phase, p.status)) break;
+      if (!ch_wait_warp(sh, &sh.q_full, q_phase, p.status)) break;
       q_phase ^= 1;
       if (!first_item) {  // both epilogues of the previous item have read O
-        if (!ch_wait(sh, &sh.o_empty[0], o_phase, p.status) || !ch_wait(sh, &sh.o_empty[1], o_phase, p.status))
+        if (!ch_wait_warp(sh, &sh.o_empty[0], o_phase, p.status) ||
+            !ch_wait_warp(sh, &sh.o_empty[1], o_phase, p.status))
           break;
         o_phase ^= 1;
       }
       first_item = false;
       if (j1 <= j0) {  // nothing to multiply: Q is free, and each epilogue gets its one P V completion
-        if (lane == 0) {
-          umma_commit(&sh.q_empty);
-          umma_commit(&sh.pv_done[0]);
-          umma_commit(&sh.pv_done[1]);
-        }
-        __syncwarp();
+        umma_commit(&sh.q_empty);
+        umma_commit(&sh.pv_done[0]);
+        umma_commit(&sh.pv_done[1]);
         ++pv_commits[0];
         ++pv_commits[1];
         continue;
@@ -476,46 +480,39 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       auto qk = [&](int w, int j) -> bool {
         const uint32_t t = kv_count + (j - j0);  // tiles this CTA has taken so far
         const int stage = t % KST;
-        if (w == 0 && !ch_wait(sh, &sh.k_full[stage], (t / KST) & 1, p.status)) return false;
-        if (j > j0 && !ch_wait(sh, &sh.pv_done[w], (pv_commits[w] - 1) & 1, p.status)) return false;
+        if (w == 0 && !ch_wait_warp(sh, &sh.k_full[stage], (t / KST) & 1, p.status)) return false;
+        if (j > j0 && !ch_wait_warp(sh, &sh.pv_done[w], (pv_commits[w] - 1) & 1, p.status)) return false;
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sk = smem_u32(smem + SMEM_K + stage * KV_BYTES);
-          const uint32_t qw = sq + w * Q_BYTES;
+        const uint32_t sk = smem_u32(smem + SMEM_K + stage * KV_BYTES);
+        const uint32_t qw = sq + w * Q_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < CH_D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
-            umma_f16(tmem + w * CH_N, umma_desc(qw + off, 16, 1024), umma_desc(sk + off, 16, 1024), idesc_qk,
-                     kk > 0);
-          }
-          umma_commit(&sh.s_full[w]);
-          if (w == 1) {
-            umma_commit(&sh.k_empty[stage]);
-            if (j == j1 - 1) umma_commit(&sh.q_empty);
-          }
+        for (int kk = 0; kk < CH_D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
+          umma_f16(tmem + w * CH_N, umma_desc(qw + off, 16, 1024), umma_desc(sk + off, 16, 1024), idesc_qk, kk > 0);
         }
-        __syncwarp();
+        umma_commit(&sh.s_full[w]);
+        if (w == 1) {
+          umma_commit(&sh.k_empty[stage]);
+          if (j == j1 - 1) umma_commit(&sh.q_empty);
+        }
         return true;
       };
       // O_w += P_w(j) V(j), P_w(j) in the first 64 columns of S_w
       auto pv = [&](int w, int j) -> bool {
-        if (!ch_wait(sh, &sh.p_full[w], p_phase[w], p.status)) return false;
+        if (!ch_wait_warp(sh, &sh.p_full[w], p_phase[w], p.status)) return false;
         p_phase[w] ^= 1;
         const uint32_t t = kv_count + (j - j0);
         const int stage = t % VST;
-        if (w == 0 && !ch_wait(sh, &sh.v_full[stage], (t / VST) & 1, p.status)) return false;
+        if (w == 0 && !ch_wait_warp(sh, &sh.v_full[stage], (t / VST) & 1, p.status)) return false;
         tc_fence_after();
-        if (lane == 0) {
-          const uint32_t sv = smem_u32(smem + SMEM_V + stage * KV_BYTES);
-          const uint32_t pt = tmem + w * CH_N;
+        const uint32_t sv = smem_u32(smem + SMEM_V + stage * KV_BYTES);
+        const uint32_t pt = tmem + w * CH_N;
 #pragma unroll
-          for (int kk = 0; kk < CH_N / 16; ++kk)  // keys 16kk.. = P columns 8kk..; V rows 16kk.., both panels
-            umma_f16_ts(tmem + TMEM_O + w * CH_N, pt + 8 * kk, umma_desc(sv + kk * 16 * 128, PANEL, 1024),
-                        idesc_pv, (j > j0 || kk > 0) ? 1u : 0u);
-          umma_commit(&sh.pv_done[w]);
-          if (w == 1) umma_commit(&sh.v_empty[stage]);
-        }
-        __syncwarp();
+        for (int kk = 0; kk < CH_N / 16; ++kk)  // keys 16kk.. = P columns 8kk..; V rows 16kk.., both panels
+          umma_f16_ts(tmem + TMEM_O + w * CH_N, pt + 8 * kk, umma_desc(sv + kk * 16 * 128, PANEL, 1024), idesc_pv,
+                      (j > j0 || kk > 0) ? 1u : 0u);
+        umma_commit(&sh.pv_done[w]);
+        if (w == 1) umma_commit(&sh.v_empty[stage]);
         ++pv_commits[w];
         return true;
       };
@@ -738,8 +735,8 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
 
   // ---- teardown: drain this CTA's tensor-core work, then free tensor memory
   if (warp == 1) {
-    if (lane == 0) umma_commit(&sh.drain);  // arrives once every MMA issued by this thread has completed
     __syncwarp();
+    umma_commit(&sh.drain);  // arrives once every MMA issued by lane 0 has completed
     mbar_wait(&sh.drain, 0);
   }
   tc_fence_before();

@@ -413,20 +413,17 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         rdy = __shfl_sync(FULL_MASK, rdy, 0);
         if (rdy) {
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sk = sbase + L::K_OFF + ks * VF_KV_BYTES;
-            const uint32_t sq = sbase + L::Q_OFF + qb * L::QBUF;
+          const uint32_t sk = sbase + L::K_OFF + ks * VF_KV_BYTES;
+          const uint32_t sq = sbase + L::Q_OFF + qb * L::QBUF;
 #pragma unroll
-            for (int kk = 0; kk < VF_D / 16; ++kk) {
-              const uint32_t offk = (kk >> 2) * VF_PANEL + (kk & 3) * 32, offq = (kk >> 2) * L::QP + (kk & 3) * 32;
-              umma_f16(tmem + b * NCOL, umma_desc(sk + offk, 16, 1024), umma_desc(sq + offq, 16, 1024), idesc_s,
-                       kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&sh.s_full[b]);
-            umma_commit(&sh.k_empty[ks]);
-            if (j == it.t1 - 1) umma_commit(&sh.q_empty[qb]);
+          for (int kk = 0; kk < VF_D / 16; ++kk) {
+            const uint32_t offk = (kk >> 2) * VF_PANEL + (kk & 3) * 32, offq = (kk >> 2) * L::QP + (kk & 3) * 32;
+            umma_f16(tmem + b * NCOL, umma_desc(sk + offk, 16, 1024), umma_desc(sq + offq, 16, 1024), idesc_s,
+                     kk > 0 ? 1u : 0u);
           }
-          __syncwarp();
+          umma_commit(&sh.s_full[b]);
+          umma_commit(&sh.k_empty[ks]);
+          if (j == it.t1 - 1) umma_commit(&sh.q_empty[qb]);
           job_item[gs % RING] = is;
           job_first[gs % RING] = o_first;
           o_first = false;
@@ -454,17 +451,14 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
         rdy = __shfl_sync(FULL_MASK, rdy, 0);
         if (rdy) {
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sp = sbase + L::P_OFF;
-            const uint32_t sv = sbase + L::V_OFF + vs * VF_KV_BYTES;
+          const uint32_t sp = sbase + L::P_OFF;
+          const uint32_t sv = sbase + L::V_OFF + vs * VF_KV_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < VF_N / 16; ++kk)  // keys 16 kk .. + 15: P columns of panel kk / 4, V rows 16 kk ..
-              umma_f16(tmem + VF_TMEM_O + os * 128, umma_desc(sp + (kk >> 2) * L::PP + (kk & 3) * 32, 16, 1024),
-                       umma_desc(sv + kk * 16 * 128, VF_PANEL, 1024), idesc_o, (!first || kk > 0) ? 1u : 0u);
-            umma_commit(&sh.pv_done[b]);
-            umma_commit(&sh.v_empty[vs]);
-          }
-          __syncwarp();
+          for (int kk = 0; kk < VF_N / 16; ++kk)  // keys 16 kk .. + 15: P columns of panel kk / 4, V rows 16 kk ..
+            umma_f16(tmem + VF_TMEM_O + os * 128, umma_desc(sp + (kk >> 2) * L::PP + (kk & 3) * 32, 16, 1024),
+                     umma_desc(sv + kk * 16 * 128, VF_PANEL, 1024), idesc_o, (!first || kk > 0) ? 1u : 0u);
+          umma_commit(&sh.pv_done[b]);
+          umma_commit(&sh.v_empty[vs]);
           ++gp;
           prog = true;
         }
@@ -821,8 +815,8 @@ __global__ void __launch_bounds__(VF_THREADS, 1)
 
   // ---- teardown: drain this CTA's tensor-core work, then free tensor memory
   if (warp == 1) {
-    if (lane == 0) umma_commit(&sh.drain);  // arrives once every MMA issued by this thread has completed
     __syncwarp();
+    umma_commit(&sh.drain);  // arrives once every MMA issued by lane 0 has completed
     mbar_wait(&sh.drain, 0);
   }
   tc_fence_before();
