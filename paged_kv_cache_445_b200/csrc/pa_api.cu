@@ -367,14 +367,15 @@ size_t decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, i
 namespace {
 // Per-SM rates of the kernels on a B200, used only to share the SMs between
 // the decode rows and the chunk rows of one batch (measured beside each
-// other on the mixed 512-token chunk + 127 decodes batch: an 8-warp decode
-// CTA streams about 65 GB/s of KV, the tcgen05 chunk kernel about 6.8
-// TFLOP/s per SM; the decode rows of a whole GPU about 6.2 TB/s).  A split
-// is used when its model time beats running the two kernels one after the
-// other on the whole GPU by 5 %.
-constexpr double DECODE_BYTES_PER_S_PER_SM = 65e9;
+// other on the mixed 512-token chunk + 127 decodes batch, where a sweep of
+// the split put both sides' end together at 60 decode SMs: an 8-warp decode
+// CTA streams about 66 GB/s of KV, the tcgen05 chunk kernel on stream-K
+// ranges about 6.0 TFLOP/s per SM; the decode rows of a whole GPU about 6.2
+// TB/s).  A split is used when its model time beats running the two kernels
+// one after the other on the whole GPU by 5 %.
+constexpr double DECODE_BYTES_PER_S_PER_SM = 66e9;
 constexpr double DECODE_BYTES_PER_S_ALL = 6.2e12;
-constexpr double CHUNK_FLOPS_PER_S_PER_SM = 6.8e12;
+constexpr double CHUNK_FLOPS_PER_S_PER_SM = 6.0e12;
 
 int plan_split(double decode_bytes, double chunk_flops, int num_sms) {
   const double serial = decode_bytes / DECODE_BYTES_PER_S_ALL + chunk_flops / (num_sms * CHUNK_FLOPS_PER_S_PER_SM);
