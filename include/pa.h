@@ -95,8 +95,8 @@ PA_API int pa_cache_append(const void* k_new, const void* v_new, void* k_cache, 
  * tables are `max_blocks_per_seq` wide, on the CURRENT device (the figure
  * depends on its SM count).  Returns 0 for invalid sizes.
  *
- * It covers every call the batch may take: at head_dim 128 with a group the
- * tcgen05 kernels support it includes the prefill chunk kernel's piece area
+ * It covers every call the batch may take: at head_dim 64 or 128 with a group
+ * the tcgen05 chunk kernel supports it includes that kernel's piece area
  * (two slots of 256 rows x 132 floats per SM, about 40 MB on a 148-SM GPU),
  * which decode calls do not use.
  *
@@ -263,8 +263,10 @@ PA_API int pa_decode_cascade(void* out, const void* q, const void* k_new, const 
  * another on `stream`: a tcgen05 kernel for sequences with 2 .. 64/G rows
  * (speculative verification: the "Speculative decoding" section of
  * "Inference optimization"; batches of at most 512 sequences), the tcgen05
- * chunk kernel for longer chunks, and the decode path for qlen = 1.  Other
- * head dims run every row on the decode path.  A row with no key (p < 0)
+ * chunk kernel for longer chunks, and the decode path for qlen = 1.  At
+ * head_dim 64 (same groups) the tcgen05 chunk kernel takes every sequence of
+ * 2 or more rows.  Other head dims and groups run every row on the decode
+ * path.  A row with no key (p < 0)
  * produces zeros.  Workspace: pa_workspace_bytes(total_q_tokens, ...), under
  * its contract (zero-filled once; the call leaves its counters at zero).
  */

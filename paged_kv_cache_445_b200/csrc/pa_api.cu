@@ -330,6 +330,7 @@ int run_attention(void* out, const void* q, const int32_t* query_start, const vo
     c.num_q_heads = num_q_heads;
     c.num_kv_heads = num_kv_heads;
     c.group = p.group;
+    c.head_dim = head_dim;
     c.block_size = block_size;
     c.num_blocks = num_blocks;
     c.scale_log2 = p.scale_log2;
@@ -372,7 +373,10 @@ namespace {
 // CTA streams about 66 GB/s of KV, the tcgen05 chunk kernel on stream-K
 // ranges about 6.0 TFLOP/s per SM; the decode rows of a whole GPU about 6.2
 // TB/s).  A split is used when its model time beats running the two kernels
-// one after the other on the whole GPU by 5 %.
+// one after the other on the whole GPU by 5 %.  The decode side takes an
+// even number of SMs: SMs come in pairs, and a pair shared by a decode CTA
+// and a chunk CTA slowed the step by about 12 % (642 us at 59 and 61 decode
+// SMs against 571 and 577 us at 60 and 62).
 constexpr double DECODE_BYTES_PER_S_PER_SM = 66e9;
 constexpr double DECODE_BYTES_PER_S_ALL = 6.2e12;
 constexpr double CHUNK_FLOPS_PER_S_PER_SM = 6.0e12;
@@ -381,7 +385,7 @@ int plan_split(double decode_bytes, double chunk_flops, int num_sms) {
   const double serial = decode_bytes / DECODE_BYTES_PER_S_ALL + chunk_flops / (num_sms * CHUNK_FLOPS_PER_S_PER_SM);
   double best = serial;
   int best_n = 0;
-  for (int n = 1; n < num_sms; ++n) {
+  for (int n = 2; n < num_sms; n += 2) {
     const double bw = n * DECODE_BYTES_PER_S_PER_SM < DECODE_BYTES_PER_S_ALL ? n * DECODE_BYTES_PER_S_PER_SM
                                                                              : DECODE_BYTES_PER_S_ALL;
     const double td = decode_bytes / bw, tc = chunk_flops / ((num_sms - n) * CHUNK_FLOPS_PER_S_PER_SM);

@@ -59,22 +59,28 @@ namespace pa {
 namespace {
 
 constexpr int CH_THREADS = 384;
-constexpr int CH_D = 128;
+constexpr int CH_D_MAX = 128;              // head_dim 64 or 128: one or two 64-column panels
 constexpr int CH_M = 128;                   // query rows per M-tile
 constexpr int CH_N = 128;                   // keys per N-tile
 constexpr int PANEL = CH_M * 128;           // one 128-row x 128-byte swizzled panel (16 KB)
-constexpr int Q_BYTES = 2 * PANEL;          // one M-tile of Q: [2 head-dim halves][128 rows][128 B]
-constexpr int KV_BYTES = 2 * PANEL;         // one K (or V) tile
 constexpr int KST = 3;                      // K stages (a K tile is free once QK_B of it is done)
 constexpr int VST = 2;                      // V stages (a V tile is free once PV_B of it is done)
-constexpr int SMEM_Q = 0;                   // Q_A, Q_B
-constexpr int SMEM_K = SMEM_Q + 2 * Q_BYTES;
-constexpr int SMEM_V = SMEM_K + KST * KV_BYTES;
-constexpr int SMEM_TOTAL = SMEM_V + VST * KV_BYTES;           // 224 KB
+// Shared memory for head_dim D (D / 64 panels per row block): Q_A, Q_B, then
+// the K and V rings.  224 KB at D = 128, 112 KB at D = 64.
+template <int D>
+struct ChLayout {
+  static constexpr int NP = D / 64;              // 64-column panels per row
+  static constexpr int Q_BYTES = NP * PANEL;     // one M-tile of Q: [NP panels][128 rows][128 B]
+  static constexpr int KV_BYTES = NP * PANEL;    // one K (or V) tile of 128 keys
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_K = SMEM_Q + 2 * Q_BYTES;
+  static constexpr int SMEM_V = SMEM_K + KST * KV_BYTES;
+  static constexpr int SMEM_TOTAL = SMEM_V + VST * KV_BYTES;
+};
 constexpr uint32_t TMEM_COLS = 512;                           // S_A, S_B, O_A, O_B: 128 columns each
-constexpr uint32_t TMEM_O = 256;                              // O of M-tile w at TMEM_O + 128 w
+constexpr uint32_t TMEM_O = 256;                              // O of M-tile w at TMEM_O + 128 w (D columns)
 constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when the max rises by > 2^8
-constexpr int SLOT_STRIDE = CH_D + 4;  // piece slot row: O[128], m, l, 2 floats of padding
+constexpr int SLOT_STRIDE = CH_D_MAX + 4;  // piece slot row: O[D], then m, l (at D), padding
 constexpr int MIN_UNITS_PER_CTA = 4;   // key tiles
 // What a CTA reads or writes once (Q tiles, piece slots) goes into L2 as
 // first to be evicted, ahead of the K/V tiles the other items re-read.
@@ -239,6 +245,7 @@ __device__ __forceinline__ bool ch_wait_warp(Shared& sh, uint64_t* bar, uint32_t
 // sum_k 2^(m_k - m) l_k; then write the bf16 row (orow == nullptr: a row past
 // the chunk, nothing to write).  Kept out of line: the rare path's registers
 // stay out of the softmax loop's allocation.
+template <int D>
 __device__ __noinline__ void merge_row(const float* __restrict__ partials, int units, int ncta, int ubase, int c_first,
                                        int c_last, int first_slot, int wrow, __nv_bfloat16* orow) {
   float mmax = -INFINITY, lsum = 0.f;
@@ -246,19 +253,19 @@ __device__ __noinline__ void merge_row(const float* __restrict__ partials, int u
     if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;  // no piece
     const int sl = c == c_first ? first_slot : 0;
     const float* src = partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
-    mmax = fmaxf(mmax, __ldcg(src + CH_D));
+    mmax = fmaxf(mmax, __ldcg(src + D));
   }
   for (int c = c_first; c <= c_last; ++c) {
     if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;
     const int sl = c == c_first ? first_slot : 0;
     const float* src = partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(src + CH_D));
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(src + D));
     lsum += ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - mmax) * ml.y;
   }
   if (!orow) return;
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
 #pragma unroll 1
-  for (int cc = 0; cc < CH_D / 32; ++cc) {
+  for (int cc = 0; cc < D / 32; ++cc) {
     float acc[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
@@ -266,7 +273,7 @@ __device__ __noinline__ void merge_row(const float* __restrict__ partials, int u
       if (cta_range_start(units, c + 1, ncta) == cta_range_start(units, c, ncta)) continue;
       const int sl = c == c_first ? first_slot : 0;
       const float* src = partials + ((static_cast<long long>(c) * 2 + sl) * 2 * CH_M + wrow) * SLOT_STRIDE;
-      const float mk = __ldcg(src + CH_D);
+      const float mk = __ldcg(src + D);
       const float wk = mk == -INFINITY ? 0.f : fast_exp2(mk - mmax);
 #pragma unroll
       for (int i = 0; i < 32; i += 4) {
@@ -289,10 +296,12 @@ __device__ __noinline__ void merge_row(const float* __restrict__ partials, int u
   }
 }
 
-template <int G>
+template <int G, int D>
 __global__ void __launch_bounds__(CH_THREADS, 1)
     chunk_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, const ChunkParams p) {
+  static_assert(D == 64 || D == 128, "head_dim");
+  using L = ChLayout<D>;
   constexpr int TOK = CH_M / G;  // tokens per M-tile
   constexpr int PAIR = 2 * TOK;  // tokens per item
   extern __shared__ uint8_t smem_raw[];
@@ -392,33 +401,35 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       if (items > 0 && !ch_wait(sh, &sh.q_empty, (items - 1) & 1, p.status)) break;
       if (lane == 0) {
         const int t0 = it.q0 + it.tp * PAIR;
-        mbar_arrive_expect_tx(&sh.q_full, 2 * Q_BYTES);
+        mbar_arrive_expect_tx(&sh.q_full, 2 * L::Q_BYTES);
         const uint64_t qpol = policy_evict_first();
-        tma_load_3d_hint(smem + SMEM_Q, &tmq, &sh.q_full, 0, it.kvh * G, t0, qpol);
-        tma_load_3d_hint(smem + SMEM_Q + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0, qpol);
-        tma_load_3d_hint(smem + SMEM_Q + Q_BYTES, &tmq, &sh.q_full, 0, it.kvh * G, t0 + TOK, qpol);
-        tma_load_3d_hint(smem + SMEM_Q + Q_BYTES + PANEL, &tmq, &sh.q_full, 64, it.kvh * G, t0 + TOK, qpol);
+#pragma unroll
+        for (int pn = 0; pn < L::NP; ++pn) {  // panel pn: head-dim columns 64 pn .. 64 pn + 63
+          tma_load_3d_hint(smem + L::SMEM_Q + pn * PANEL, &tmq, &sh.q_full, 64 * pn, it.kvh * G, t0, qpol);
+          tma_load_3d_hint(smem + L::SMEM_Q + L::Q_BYTES + pn * PANEL, &tmq, &sh.q_full, 64 * pn, it.kvh * G,
+                           t0 + TOK, qpol);
+        }
       }
       auto load_tile = [&](const CUtensorMap* tm, uint64_t* bars_full, uint64_t* bars_empty, int nst, int base_off,
                            uint32_t t, int blk, int y) -> bool {
         const int st = t % nst;
         const uint32_t use = t / nst;  // earlier fills of this stage
         if (use > 0 && !ch_wait(sh, &bars_empty[st], (use - 1) & 1, p.status)) return false;
-        if (lane == 0) mbar_arrive_expect_tx(&bars_full[st], KV_BYTES);
+        if (lane == 0) mbar_arrive_expect_tx(&bars_full[st], L::KV_BYTES);
         __syncwarp();
-        if (lane < CH_N / 16) {  // 16-row boxes (head-dim half, 16 keys) -> rows 16*lane.. of both panels
+        if (lane < CH_N / 16) {  // 16-row boxes (one 64-column panel, 16 keys) -> rows 16*lane.. of every panel
           if (blk >= p.num_blocks) set_status(p.status, PA_STATUS_BIT(PA_ERR_RANGE));
-          uint8_t* dst = smem + base_off + st * KV_BYTES + lane * 2048;
-          tma_load_4d(dst, tm, &bars_full[st], 0, y, it.kvh, blk, pol);
-          tma_load_4d(dst + PANEL, tm, &bars_full[st], 64, y, it.kvh, blk, pol);
+          uint8_t* dst = smem + base_off + st * L::KV_BYTES + lane * 2048;
+#pragma unroll
+          for (int pn = 0; pn < L::NP; ++pn) tma_load_4d(dst + pn * PANEL, tm, &bars_full[st], 64 * pn, y, it.kvh, blk, pol);
         }
         return true;
       };
       bool ok = true;
       for (int j = j0; ok && j < j1; ++j) {
-        ok = load_tile(&tmk, sh.k_full, sh.k_empty, KST, SMEM_K, tcount + (j - j0), blk_cur, y_cur);
+        ok = load_tile(&tmk, sh.k_full, sh.k_empty, KST, L::SMEM_K, tcount + (j - j0), blk_cur, y_cur);
         if (ok && j > j0)
-          ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + (j - j0) - 1, blk_prev, y_prev);
+          ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, L::SMEM_V, tcount + (j - j0) - 1, blk_prev, y_prev);
         blk_prev = blk_cur;
         y_prev = y_cur;
         blk_cur = blk_next;
@@ -426,7 +437,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         tile_ids(j + 2, blk_next, y_next);  // one tile of lead for the block-table reads
       }
       if (ok && j1 > j0)
-        ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, SMEM_V, tcount + (j1 - j0) - 1, blk_prev, y_prev);
+        ok = load_tile(&tmv, sh.v_full, sh.v_empty, VST, L::SMEM_V, tcount + (j1 - j0) - 1, blk_prev, y_prev);
       tcount += j1 - j0;
       if (!ok) break;
     }
@@ -444,8 +455,8 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     const uint32_t idesc_qk = umma_idesc(CH_M, CH_N, 0, 0);
-    const uint32_t idesc_pv = umma_idesc(CH_M, CH_D, 0, 1);
-    const uint32_t sq = smem_u32(smem + SMEM_Q);
+    const uint32_t idesc_pv = umma_idesc(CH_M, D, 0, 1);
+    const uint32_t sq = smem_u32(smem + L::SMEM_Q);
     uint32_t q_phase = 0, p_phase[2] = {0, 0}, o_phase = 0, kv_count = 0;
     uint32_t pv_commits[2] = {0, 0};  // completions committed to pv_done[w] so far
     bool first_item = true;
@@ -483,10 +494,10 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         if (w == 0 && !ch_wait_warp(sh, &sh.k_full[stage], (t / KST) & 1, p.status)) return false;
         if (j > j0 && !ch_wait_warp(sh, &sh.pv_done[w], (pv_commits[w] - 1) & 1, p.status)) return false;
         tc_fence_after();
-        const uint32_t sk = smem_u32(smem + SMEM_K + stage * KV_BYTES);
-        const uint32_t qw = sq + w * Q_BYTES;
+        const uint32_t sk = smem_u32(smem + L::SMEM_K + stage * L::KV_BYTES);
+        const uint32_t qw = sq + w * L::Q_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < CH_D / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
           umma_f16(tmem + w * CH_N, umma_desc(qw + off, 16, 1024), umma_desc(sk + off, 16, 1024), idesc_qk, kk > 0);
         }
@@ -505,7 +516,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         const int stage = t % VST;
         if (w == 0 && !ch_wait_warp(sh, &sh.v_full[stage], (t / VST) & 1, p.status)) return false;
         tc_fence_after();
-        const uint32_t sv = smem_u32(smem + SMEM_V + stage * KV_BYTES);
+        const uint32_t sv = smem_u32(smem + L::SMEM_V + stage * L::KV_BYTES);
         const uint32_t pt = tmem + w * CH_N;
 #pragma unroll
         for (int kk = 0; kk < CH_N / 16; ++kk)  // keys 16kk.. = P columns 8kk..; V rows 16kk.., both panels
@@ -629,7 +640,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           if (!(ok = ch_wait(sh, &sh.pv_done[w], (pv_count + (j - j0) - 1) & 1, p.status))) break;
           tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < CH_D / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             float v[32];
             tmem_ld32(o_col + c * 32, v);
             tmem_wait_ld();
@@ -646,10 +657,11 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           const uint32_t t = kv_count + (j - j0);
           const int stage = t % VST;
           if (!(ok = ch_wait(sh, &sh.v_full[stage], (t / VST) & 1, p.status))) break;
-          uint8_t* vst = smem + SMEM_V + stage * KV_BYTES;
-          const int nz = (CH_N - max(valid_keys, 0)) * 2 * 8;  // 16-byte chunks in both panels
+          uint8_t* vst = smem + L::SMEM_V + stage * L::KV_BYTES;
+          constexpr int CPR = D / 8;  // 16-byte chunks of a key row, over all panels
+          const int nz = (CH_N - max(valid_keys, 0)) * CPR;
           for (int k = threadIdx.x - 128; k < nz; k += 128) {
-            const int r = max(valid_keys, 0) + k / 16, rest = k % 16;
+            const int r = max(valid_keys, 0) + k / CPR, rest = k % CPR;
             *reinterpret_cast<uint4*>(vst + (rest >> 3) * PANEL + r * 128 + (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
@@ -664,11 +676,11 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       if (!ch_wait(sh, &sh.pv_done[w], (pv_count - 1) & 1, p.status)) break;
       tc_fence_after();
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                            (static_cast<long long>(it.q0 + tok) * p.num_q_heads + it.kvh * G + head_in_group) * CH_D;
+                            (static_cast<long long>(it.q0 + tok) * p.num_q_heads + it.kvh * G + head_in_group) * D;
       if (j0 == 0 && j1 == nt) {  // the whole item: O / l -> bf16 -> out
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < CH_D / 32; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           float v[32];
           if (nt > 0) {
             tmem_ld32(o_col + c * 32, v);
@@ -704,7 +716,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       float* dst = p.partials + ((static_cast<long long>(cta) * 2 + my_slot) * 2 * CH_M + wrow) * SLOT_STRIDE;
       const uint64_t spol = policy_evict_first();
 #pragma unroll
-      for (int c = 0; c < CH_D / 32; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         float v[32];
         tmem_ld32(o_col + c * 32, v);
         tmem_wait_ld();
@@ -713,7 +725,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
           st_global_hint(reinterpret_cast<float4*>(dst + c * 32 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]),
                          spol);
       }
-      __stcg(reinterpret_cast<float2*>(dst + CH_D), make_float2(m_ref, l));
+      __stcg(reinterpret_cast<float2*>(dst + D), make_float2(m_ref, l));
       tc_fence_before();
       mbar_arrive(&sh.o_empty[w]);  // O has been read
       // One count per (item, row): the thread that lands a row's last piece
@@ -728,7 +740,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       if (atomicAdd(cnt, 1) != npieces - 1) continue;
       *cnt = 0;  // every piece of this row has arrived: back to zero for the next call
       __threadfence();
-      merge_row(p.partials, units, ncta, ubase, c_first, c_last, first_slot, wrow, row_valid ? orow : nullptr);
+      merge_row<D>(p.partials, units, ncta, ubase, c_first, c_last, first_slot, wrow, row_valid ? orow : nullptr);
     }
   }
 
@@ -753,14 +765,15 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
 // ------------------------------------------------------------------ host side
 
 int chunk_supported(int group, int head_dim) {
-  return head_dim == CH_D && (group == 1 || group == 2 || group == 4 || group == 8 || group == 16);
+  return (head_dim == 64 || head_dim == 128) && (group == 1 || group == 2 || group == 4 || group == 8 || group == 16);
 }
 
 // q [Tq, Hq, D] bf16 as a 3-D tensor (D, Hq, Tq); box = 64 columns x G heads x 128/G tokens.
 static int encode_q_tmap(CUtensorMap* map, const void* q, int total_q_tokens, int num_q_heads, int group,
-                         EncodeTiledFn fn) {
-  const cuuint64_t dims[3] = {CH_D, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(total_q_tokens)};
-  const cuuint64_t strides[2] = {CH_D * 2, static_cast<cuuint64_t>(num_q_heads) * CH_D * 2};
+                         int head_dim, EncodeTiledFn fn) {
+  const cuuint64_t d = static_cast<cuuint64_t>(head_dim);
+  const cuuint64_t dims[3] = {d, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(total_q_tokens)};
+  const cuuint64_t strides[2] = {d * 2, static_cast<cuuint64_t>(num_q_heads) * d * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(CH_M / group)};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
@@ -771,9 +784,10 @@ static int encode_q_tmap(CUtensorMap* map, const void* q, int total_q_tokens, in
 
 // [num_blocks, Hkv, block_size, D] as a 4-D tensor; box = 64 columns x 16 rows of one (block, head).
 int encode_kv16_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
-                     EncodeTiledFn fn) {
-  const cuuint64_t row = CH_D * 2;
-  const cuuint64_t dims[4] = {CH_D, static_cast<cuuint64_t>(block_size), static_cast<cuuint64_t>(num_kv_heads),
+                     int head_dim, EncodeTiledFn fn) {
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * 2;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(block_size),
+                              static_cast<cuuint64_t>(num_kv_heads),
                               static_cast<cuuint64_t>(num_blocks)};
   const cuuint64_t strides[3] = {row, row * block_size, row * block_size * num_kv_heads};
   const cuuint32_t box[4] = {64, 16, 1, 1};
@@ -784,11 +798,11 @@ int encode_kv16_tmap(CUtensorMap* map, const void* cache, int num_blocks, int nu
   return r == CUDA_SUCCESS ? PA_OK : cu_fail(r, "cuTensorMapEncodeTiled");
 }
 
-template <int G>
+template <int G, int D>
 static int launch_chunk_t(const ChunkParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           cudaStream_t stream, int num_sms, int ctas) {
-  auto kern = chunk_kernel<G>;
-  const int smem = SMEM_TOTAL + 1024;
+  auto kern = chunk_kernel<G, D>;
+  const int smem = ChLayout<D>::SMEM_TOTAL + 1024;
   static PerDevice configured;
   int done = 0;
   const int rc_setup = per_device(
@@ -843,15 +857,24 @@ int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const
   if (!fn) return PA_ERR_CUDA;
   CUtensorMap tq, tk, tv;
   int rc;
-  if ((rc = encode_q_tmap(&tq, q, total_q_tokens, p.num_q_heads, p.group, fn)) != PA_OK) return rc;
-  if ((rc = encode_kv16_tmap(&tk, k_cache, p.num_blocks, p.num_kv_heads, p.block_size, fn)) != PA_OK) return rc;
-  if ((rc = encode_kv16_tmap(&tv, v_cache, p.num_blocks, p.num_kv_heads, p.block_size, fn)) != PA_OK) return rc;
+  if (!chunk_supported(p.group, p.head_dim)) return PA_ERR_UNSUPPORTED;
+  if ((rc = encode_q_tmap(&tq, q, total_q_tokens, p.num_q_heads, p.group, p.head_dim, fn)) != PA_OK) return rc;
+  if ((rc = encode_kv16_tmap(&tk, k_cache, p.num_blocks, p.num_kv_heads, p.block_size, p.head_dim, fn)) != PA_OK)
+    return rc;
+  if ((rc = encode_kv16_tmap(&tv, v_cache, p.num_blocks, p.num_kv_heads, p.block_size, p.head_dim, fn)) != PA_OK)
+    return rc;
+  const bool d64 = p.head_dim == 64;
   switch (p.group) {
-    case 1: return launch_chunk_t<1>(p, tq, tk, tv, stream, num_sms, ctas);
-    case 2: return launch_chunk_t<2>(p, tq, tk, tv, stream, num_sms, ctas);
-    case 4: return launch_chunk_t<4>(p, tq, tk, tv, stream, num_sms, ctas);
-    case 8: return launch_chunk_t<8>(p, tq, tk, tv, stream, num_sms, ctas);
-    case 16: return launch_chunk_t<16>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 1: return d64 ? launch_chunk_t<1, 64>(p, tq, tk, tv, stream, num_sms, ctas)
+                       : launch_chunk_t<1, 128>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 2: return d64 ? launch_chunk_t<2, 64>(p, tq, tk, tv, stream, num_sms, ctas)
+                       : launch_chunk_t<2, 128>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 4: return d64 ? launch_chunk_t<4, 64>(p, tq, tk, tv, stream, num_sms, ctas)
+                       : launch_chunk_t<4, 128>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 8: return d64 ? launch_chunk_t<8, 64>(p, tq, tk, tv, stream, num_sms, ctas)
+                       : launch_chunk_t<8, 128>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 16: return d64 ? launch_chunk_t<16, 64>(p, tq, tk, tv, stream, num_sms, ctas)
+                        : launch_chunk_t<16, 128>(p, tq, tk, tv, stream, num_sms, ctas);
     default: return PA_ERR_UNSUPPORTED;
   }
 }

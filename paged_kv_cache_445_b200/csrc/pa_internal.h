@@ -208,7 +208,7 @@ int launch_verify(const VerifyParams& p, const void* q, const void* k_cache, con
                   int total_q_tokens, cudaStream_t stream, int num_sms, int which = 3);
 
 struct ChunkParams {
-  void* out;                    // bf16 [Tq, Hq, 128]
+  void* out;                    // bf16 [Tq, Hq, head_dim]
   const int32_t* block_tables;  // [B, max_blocks]
   const int32_t* context_lens;  // [B]
   const int32_t* query_start;   // [B + 1]
@@ -217,6 +217,7 @@ struct ChunkParams {
   int num_q_heads;
   int num_kv_heads;
   int group;
+  int head_dim;  // 64 or 128
   int block_size;
   int num_blocks;
   float scale_log2;
@@ -241,7 +242,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 EncodeTiledFn encode_fn();
 // [num_blocks, Hkv, block_size, 128] bf16 as a 4-D tensor; box = 64 columns x 16 rows of one (block, head).
 int encode_kv16_tmap(CUtensorMap* map, const void* cache, int num_blocks, int num_kv_heads, int block_size,
-                     EncodeTiledFn fn);
+                     int head_dim, EncodeTiledFn fn);
 
 struct DeviceInfo {
   int num_sms;

@@ -884,8 +884,8 @@ int launch_verify(const VerifyParams& p, const void* q, const void* k_cache, con
   if (!fn) return PA_ERR_CUDA;
   CUtensorMap tk, tv;
   int rc;
-  if ((rc = encode_kv16_tmap(&tk, k_cache, p.num_blocks, p.num_kv_heads, p.block_size, fn)) != PA_OK) return rc;
-  if ((rc = encode_kv16_tmap(&tv, v_cache, p.num_blocks, p.num_kv_heads, p.block_size, fn)) != PA_OK) return rc;
+  if ((rc = encode_kv16_tmap(&tk, k_cache, p.num_blocks, p.num_kv_heads, p.block_size, VF_D, fn)) != PA_OK) return rc;
+  if ((rc = encode_kv16_tmap(&tv, v_cache, p.num_blocks, p.num_kv_heads, p.block_size, VF_D, fn)) != PA_OK) return rc;
   // columns <= 32 on the 32-wide kernel, 33 .. 64 on the 64-wide one
   CUtensorMap tq;
   if (which & 1) {

@@ -57,11 +57,12 @@ def test_planned_mixed_batch_shares_the_gpu_and_matches_the_oracle_on_every_row(
     assert torch.equal(first.view(torch.int16), ds.out.view(torch.int16))
 
 
-def test_chunk_items_cut_between_ctas_merge_exactly():
+@pytest.mark.parametrize("d", [128, 64])
+def test_chunk_items_cut_between_ctas_merge_exactly(d):
     # more items than CTAs: 20 pairs of M-tiles x 8 KV heads = 160 items of
     # about 13 key tiles on the whole GPU, split into equal unit ranges, so
     # items are cut at CTA boundaries and merged from their pieces
-    w = workloads.custom([1000], [640], 64, 8, 128, 16, seed=61, poison=True)
+    w = workloads.custom([1000], [640], 64, 8, d, 16, seed=61, poison=True)
     ds = DeviceStep(w)
     ds.append()
     ref = _ref(w)
@@ -71,7 +72,7 @@ def test_chunk_items_cut_between_ctas_merge_exactly():
         torch.cuda.synchronize()
         assert int(ds.status.item()) == 0
         outs.append(ds.out.clone())
-    compare(outs[0].float().cpu().numpy(), ref, "160 items cut between CTAs")
+    compare(outs[0].float().cpu().numpy(), ref, f"160 items cut between CTAs, d{d}")
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
 
@@ -96,10 +97,11 @@ PLANNED = [  # prefix list, qlen list, Hq, Hkv, d, bs
     ([3000, 2000], [2, 2], 32, 4, 128, 16),         # verification rows only
     ([1000, 40, 77], [1, 1, 1], 16, 2, 128, 16),    # decodes only
     ([0], [700], 4, 4, 128, 16),                    # one prompt from position 0, G 1
+    ([16384] + [300, 4000, 7000], [512, 1, 1, 1], 64, 8, 64, 16),  # head_dim 64: a chunk and decodes
 ]
 
 
-@pytest.mark.parametrize("case", PLANNED, ids=lambda c: f"Hq{c[2]}-Hkv{c[3]}-q{max(c[1])}-n{len(c[0])}")
+@pytest.mark.parametrize("case", PLANNED, ids=lambda c: f"Hq{c[2]}-Hkv{c[3]}-d{c[4]}-q{max(c[1])}-n{len(c[0])}")
 def test_planned_calls_match_the_oracle(case):
     prefix, qlen, hq, hkv, d, bs = case
     w = workloads.custom(prefix, qlen, hq, hkv, d, bs, seed=sum(prefix) + len(qlen), poison=True)

@@ -115,6 +115,12 @@ SMALL = [  # ctx list, qlen list, Hq, Hkv, d, bs
     ([700], [200], 4, 4, 128, 16),               # G 1: 128 tokens per tile
     ([500, 77], [50, 1], 32, 2, 128, 16),        # G 16: 8 tokens per tile
     ([260, 129, 1], [5, 129, 1], 8, 4, 128, 16), # G 2, several chunks and a decode in one batch
+    # the same on the tcgen05 path at head_dim 64 (one 64-column panel per row)
+    ([300], [300], 8, 1, 64, 16),
+    ([1000, 40], [130, 1], 16, 2, 64, 32),
+    ([700], [200], 4, 4, 64, 16),
+    ([500, 77], [50, 1], 32, 2, 64, 16),
+    ([260, 129, 1], [5, 129, 1], 8, 4, 64, 16),
 ]
 
 
@@ -135,9 +141,10 @@ def test_late_large_scores_rescale_some_rows_of_a_tile():
     # the query rows its score raises the running maximum far above the
     # earlier tiles' (the others see a very negative score), so the rescale of
     # O runs for some rows of a tile and not for others -- on the tensor-core
-    # chunk path (G 8) and on the rows path (G 6, head_dim 64)
+    # chunk path (G 8, head_dim 128 and 64) and on the rows path (G 6, head_dim 64)
     from paged_kv_cache_445_b200.workloads import bf16_bits_to_f32, f32_to_bf16_bits
-    for prefix, qlen, hq, hkv, d, bs in (([870, 39], [130, 1], 16, 2, 128, 32), ([500, 20], [60, 1], 12, 2, 64, 16)):
+    for prefix, qlen, hq, hkv, d, bs in (([870, 39], [130, 1], 16, 2, 128, 32), ([870, 39], [130, 1], 16, 2, 64, 32),
+                                         ([500, 20], [60, 1], 12, 2, 64, 16)):
         w = workloads.custom(prefix, qlen, hq, hkv, d, bs, seed=12, poison=True)
         pos = 300
         blk, off = int(w.block_tables[0, pos // bs]), pos % bs
