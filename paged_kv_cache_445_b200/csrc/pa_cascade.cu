@@ -124,8 +124,9 @@ __device__ __forceinline__ bool cs_wait(CShared& sh, uint64_t* bar, uint32_t pha
   }
 }
 
-// The MMA warp's waits: one answer for the whole warp, which stays converged
-// for the predicated MMA issue.
+// A wait taken by a whole warp: one answer for all its lanes, so the warp
+// stays converged for the predicated MMA issue or the warp-collective
+// tensor-memory loads and stores that follow.
 __device__ __forceinline__ bool cs_wait_warp(CShared& sh, uint64_t* bar, uint32_t phase, int* status) {
   return __all_sync(FULL_MASK, cs_wait(sh, bar, phase, status));
 }
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(CS_THREADS, 1)
       bool ok = true;
       for (int j = 0; j < nt && ok; ++j) {
         const int sb = j & 1;
-        if (!(ok = cs_wait(sh, &sh.s_full[sb], s_phase[sb], p.status))) break;
+        if (!(ok = cs_wait_warp(sh, &sh.s_full[sb], s_phase[sb], p.status))) break;
         s_phase[sb] ^= 1;
         tc_fence_after();
         float s[CS_N];
@@ -366,7 +367,7 @@ __global__ void __launch_bounds__(CS_THREADS, 1)
           // P V(j - 1) (phase pv_count + j - 1; P V(j - 2) was waited for at tile
           // j - 1, and P V(j) needs this tile's P) must be done before O is
           // rescaled and before P buffer j & 1, last read by P V(j - 2), is rewritten
-          if (!(ok = cs_wait(sh, &sh.pv_done, (pv_count + j - 1) & 1, p.status))) break;
+          if (!(ok = cs_wait_warp(sh, &sh.pv_done, (pv_count + j - 1) & 1, p.status))) break;
           tc_fence_after();
           // scale O (warp-uniform: tcgen05.ld/st are warp-collective; rows that
           // keep their max scale by 1)
@@ -390,7 +391,7 @@ __global__ void __launch_bounds__(CS_THREADS, 1)
       pv_count += nt;
       if (!ok) break;
       // ---- epilogue: the unnormalised partial of this row and prefix slice
-      if (!cs_wait(sh, &sh.pv_done, (pv_count - 1) & 1, p.status)) break;
+      if (!cs_wait_warp(sh, &sh.pv_done, (pv_count - 1) & 1, p.status)) break;
       tc_fence_after();
       const int seq = it.s0 + seq_off;
       const bool valid = seq_off < tokm && seq < it.ge;

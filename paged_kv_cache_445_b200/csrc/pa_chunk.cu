@@ -233,8 +233,10 @@ __device__ __forceinline__ bool ch_wait(Shared& sh, uint64_t* bar, uint32_t phas
   }
 }
 
-// The MMA warp's waits: every lane polls, and the warp takes one answer (so
-// the warp stays converged for the predicated MMA issue that follows).
+// A wait taken by a whole warp: every lane polls, and the warp takes one
+// answer, so it stays converged for what follows (the MMA warp's predicated
+// issue, the softmax warps' warp-collective tensor-memory loads and stores)
+// even when the wait runs out in some lanes only.
 __device__ __forceinline__ bool ch_wait_warp(Shared& sh, uint64_t* bar, uint32_t phase, int* status) {
   return __all_sync(FULL_MASK, ch_wait(sh, bar, phase, status));
 }
@@ -563,7 +565,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       float m_ref = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = j0; j < j1 && ok; ++j) {
-        if (!(ok = ch_wait(sh, &sh.s_full[w], s_phase, p.status))) break;
+        if (!(ok = ch_wait_warp(sh, &sh.s_full[w], s_phase, p.status))) break;
         s_phase ^= 1;
         tc_fence_after();
         float s[CH_N];
@@ -637,7 +639,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         if (j > j0 && __any_sync(FULL_MASK, resc)) {
           // pv_done[w] completes once per tile; P V_w(j) cannot have completed
           // (it waits for this thread's P), so the parity names the phase
-          if (!(ok = ch_wait(sh, &sh.pv_done[w], (pv_count + (j - j0) - 1) & 1, p.status))) break;
+          if (!(ok = ch_wait_warp(sh, &sh.pv_done[w], (pv_count + (j - j0) - 1) & 1, p.status))) break;
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -656,7 +658,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
         if (w == 0 && valid_keys < CH_N) {
           const uint32_t t = kv_count + (j - j0);
           const int stage = t % VST;
-          if (!(ok = ch_wait(sh, &sh.v_full[stage], (t / VST) & 1, p.status))) break;
+          if (!(ok = ch_wait_warp(sh, &sh.v_full[stage], (t / VST) & 1, p.status))) break;
           uint8_t* vst = smem + L::SMEM_V + stage * L::KV_BYTES;
           constexpr int CPR = D / 8;  // 16-byte chunks of a key row, over all panels
           const int nz = (CH_N - max(valid_keys, 0)) * CPR;
@@ -673,7 +675,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       pv_count += j1 > j0 ? j1 - j0 : 1;
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> out (after the item's last pv_done completion)
-      if (!ch_wait(sh, &sh.pv_done[w], (pv_count - 1) & 1, p.status)) break;
+      if (!ch_wait_warp(sh, &sh.pv_done[w], (pv_count - 1) & 1, p.status)) break;
       tc_fence_after();
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
                             (static_cast<long long>(it.q0 + tok) * p.num_q_heads + it.kvh * G + head_in_group) * D;
