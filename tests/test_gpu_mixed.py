@@ -46,6 +46,7 @@ def test_planned_mixed_batch_shares_the_gpu_and_matches_the_oracle_on_every_row(
     words = list(plan.words)
     assert words[1] & 4 and words[1] & 8, "the plan sees the chunk and the decode rows"
     assert 0 < words[2] < words[3], "decode rows on part of the SMs, the chunk on the rest"
+    assert words[2] % 2 == 0, "SMs come in pairs: the decode side takes whole pairs"
     got = ds.out.float().cpu().numpy()
     ref = _ref(w)
     compare(got[:512], ref[:512], "planned mixed batch, the chunk")
