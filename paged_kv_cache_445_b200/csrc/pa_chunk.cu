@@ -13,20 +13,22 @@
 //    one KV head (GQA packing: every K/V tile feeds all G heads).  A work item
 //    is a PAIR of consecutive M-tiles (A and B) of one KV head: both multiply
 //    the same K/V tiles, so each tile crosses L2 -> shared memory once per
-//    256 query rows.  Q comes in with one 3-D TMA box per head-dim half and
-//    M-tile (128 rows x 128 bytes, 128-byte swizzle) -- a K-major UMMA operand
-//    as it lands.
+//    256 query rows.  Head dim D = 128 or 64: a row is D/64 panels of 64
+//    columns.  Q comes in with one 3-D TMA box per panel and M-tile (128 rows
+//    x 128 bytes, 128-byte swizzle) -- a K-major UMMA operand as it lands.
 //  * N-tile = 128 keys: 128/block_size blocks, each fetched with 16-row TMA
 //    boxes straight into K-major SW128 panels (K for S = Q K^T) and the same
 //    panels serve as the MN-major B operand of O += P V.
 //  * Warp roles (12 warps, 3 warpgroups): warp 0 issues TMA; warp 1 allocates
-//    tensor memory and issues tcgen05.mma from one thread; warpgroup 1 runs
+//    tensor memory and issues tcgen05.mma (the warp converged, lane 0 under a
+//    predicate: a branch that only lane 0 takes makes each issue cost 2-3
+//    times the MMA's own 64 cycles); warpgroup 1 runs
 //    the softmax of M-tile A, warpgroup 2 that of M-tile B (thread = TMEM lane
 //    = query row).  Warpgroup 0 gives registers to the two softmax
 //    warpgroups (setmaxnreg).  Tensor memory: S_A, S_B (128 fp32 columns
 //    each; P overwrites the first 64 columns of its S as bf16 pairs and is
-//    the A operand of P V straight from tensor memory) and O_A, O_B (128
-//    columns each).  The MMA issue order QK_A(j), QK_B(j), PV_A(j), QK_A(j+1),
+//    the A operand of P V straight from tensor memory) and O_A, O_B (D
+//    columns each, 128 apart).  The MMA issue order QK_A(j), QK_B(j), PV_A(j), QK_A(j+1),
 //    PV_B(j), QK_B(j+1), ... lets the tensor cores work on one M-tile while the
 //    softmax of the other runs.
 //  * Softmax: row max and exp2 on the thread's own row (no shuffles), causal
@@ -34,13 +36,15 @@
 //    maximum rises by more than 2^8 (between rescales the stale maximum is an
 //    exact reference point).  Key rows past the context are zeroed in V
 //    before P V.
-//  * Work split (stream-K): the batch's (item, 128-key tile) units, in item
-//    order, are cut into one equal contiguous range per CTA, so every CTA gets
-//    the same number of tiles whatever the item count.  An item cut by a range
+//  * Work split: with no more items than CTAs, one whole item per CTA (the
+//    CTAs of a KV head then read its key tiles in step, from L2).  Otherwise
+//    stream-K: the batch's (item, 128-key tile) units, in item order, are cut
+//    into one equal contiguous range per CTA, so every CTA gets the same
+//    number of tiles whatever the item count.  An item cut by a range
 //    boundary leaves unnormalised (O, m, l) pieces, one per CTA that touched
-//    it, in that CTA's two piece slots; the CTA that lands the item's last
-//    piece (an atomic count per item, back to zero afterwards) merges them in
-//    CTA order and writes the rows.
+//    it, in that CTA's two piece slots; per (item, row) an atomic count tells
+//    the thread that lands the row's last piece to merge the row's pieces in
+//    CTA order, write it and put the count back to zero.
 //  * Beside the decode kernel: launched after it on part of the GPU, the
 //    kernel takes the other SMs while the decode rows stream; it then waits
 //    for that grid at its end rather than its start (the decode kernel

@@ -29,8 +29,9 @@
 //  * Roles (8 warps): warp 0 loads Q and the K tiles, warp 2 the V tiles (each
 //    refills its own ring as soon as a stage is free; V, read after the
 //    softmax, gets the deeper ring); warp 1 owns tensor memory and issues
-//    tcgen05.mma from one thread as soon as the inputs of an S or a P V are
-//    ready; warps 4-7 run the softmax and the epilogue (thread = TMEM lane).
+//    tcgen05.mma (converged, lane 0 under a predicate) as soon as the inputs
+//    of an S or a P V are ready; warps 4-7 run the softmax and the epilogue
+//    (thread = TMEM lane).
 //    S is double-buffered per tile, P single (written once P V(g - 1) has read
 //    it), Q and O per item.  An item's epilogue runs one tile into the next
 //    item, when its last P V is known to be complete, so item ends do not
