@@ -264,9 +264,9 @@ PA_API int pa_decode_cascade(void* out, const void* q, const void* k_new, const 
  * (speculative verification: the "Speculative decoding" section of
  * "Inference optimization"; batches of at most 512 sequences), the tcgen05
  * chunk kernel for longer chunks, and the decode path for qlen = 1.  At
- * head_dim 64 (same groups) the tcgen05 chunk kernel takes every sequence of
- * 2 or more rows.  Other head dims and groups run every row on the decode
- * path.  A row with no key (p < 0)
+ * head_dim 64 with those groups, and at head_dim 64 or 128 with G = 6 or 12,
+ * the tcgen05 chunk kernel takes every sequence of 2 or more rows.  Other
+ * head dims and groups run every row on the decode path.  A row with no key (p < 0)
  * produces zeros.  Workspace: pa_workspace_bytes(total_q_tokens, ...), under
  * its contract (zero-filled once; the call leaves its counters at zero).
  */

@@ -9,8 +9,10 @@
 // through the block table.
 //
 // How (B200):
-//  * M-tile = 128 query rows = 128/G consecutive tokens x the G query heads of
-//    one KV head (GQA packing: every K/V tile feeds all G heads).  A work item
+//  * M-tile = 128 query rows: TOK consecutive tokens x the G query heads of
+//    one KV head (GQA packing: every K/V tile feeds all G heads); TOK = 128/G
+//    for G = 1, 2, 4, 8, 16, and 20 or 10 tokens (120 rows, 8 of padding) for
+//    G = 6 or 12.  A work item
 //    is a PAIR of consecutive M-tiles (A and B) of one KV head: both multiply
 //    the same K/V tiles, so each tile crosses L2 -> shared memory once per
 //    256 query rows.  Head dim D = 128 or 64: a row is D/64 panels of 64
@@ -82,6 +84,15 @@ struct ChLayout {
   static constexpr int SMEM_TOTAL = SMEM_V + VST * KV_BYTES;
 };
 constexpr uint32_t TMEM_COLS = 512;                           // S_A, S_B, O_A, O_B: 128 columns each
+// Tokens per M-tile: as many as fit in its 128 rows (TOK x G, one row per
+// (token, head)) with a row count that is a multiple of 8 (whole 8-row swizzle
+// atoms for the Q box).  128 / G for G a power of two; 20 tokens (120 rows)
+// at G = 6 and 10 (120) at G = 12, the last rows then padding.
+__host__ __device__ constexpr int chunk_tok(int group) {
+  int t = CH_M / group;
+  while (t > 1 && (t * group) % 8 != 0) --t;
+  return t;
+}
 constexpr uint32_t TMEM_O = 256;                              // O of M-tile w at TMEM_O + 128 w (D columns)
 constexpr float RESCALE_LOG2 = 8.f;                           // rescale O when the max rises by > 2^8
 constexpr int SLOT_STRIDE = CH_D_MAX + 4;  // piece slot row: O[D], then m, l (at D), padding
@@ -308,8 +319,9 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
                  const __grid_constant__ CUtensorMap tmv, const ChunkParams p) {
   static_assert(D == 64 || D == 128, "head_dim");
   using L = ChLayout<D>;
-  constexpr int TOK = CH_M / G;  // tokens per M-tile
-  constexpr int PAIR = 2 * TOK;  // tokens per item
+  constexpr int TOK = chunk_tok(G);  // tokens per M-tile
+  constexpr int QROWS = TOK * G;     // its rows that hold a (token, head); the rest are padding
+  constexpr int PAIR = 2 * TOK;      // tokens per item
   extern __shared__ uint8_t smem_raw[];
   __shared__ Shared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -407,7 +419,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       if (items > 0 && !ch_wait(sh, &sh.q_empty, (items - 1) & 1, p.status)) break;
       if (lane == 0) {
         const int t0 = it.q0 + it.tp * PAIR;
-        mbar_arrive_expect_tx(&sh.q_full, 2 * L::Q_BYTES);
+        mbar_arrive_expect_tx(&sh.q_full, 2 * L::NP * QROWS * 128);  // the boxes' bytes
         const uint64_t qpol = policy_evict_first();
 #pragma unroll
         for (int pn = 0; pn < L::NP; ++pn) {  // panel pn: head-dim columns 64 pn .. 64 pn + 63
@@ -562,7 +574,7 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
       u = ubase + j1;
       const int tok = it.tp * PAIR + w * TOK + tok_in_tile;  // row's token within the chunk
       const int last_key = it.p0 + tok;                       // causal limit (inclusive)
-      const bool row_valid = tok < it.qlen && last_key >= 0;
+      const bool row_valid = row < QROWS && tok < it.qlen && last_key >= 0;
       const int tile_last = it.p0 + it.tp * PAIR + w * TOK;   // first row of this M-tile: keys beyond it are
                                                               // masked for some row of the tile
 
@@ -771,16 +783,17 @@ __global__ void __launch_bounds__(CH_THREADS, 1)
 // ------------------------------------------------------------------ host side
 
 int chunk_supported(int group, int head_dim) {
-  return (head_dim == 64 || head_dim == 128) && (group == 1 || group == 2 || group == 4 || group == 8 || group == 16);
+  return (head_dim == 64 || head_dim == 128) &&
+         (group == 1 || group == 2 || group == 4 || group == 6 || group == 8 || group == 12 || group == 16);
 }
 
-// q [Tq, Hq, D] bf16 as a 3-D tensor (D, Hq, Tq); box = 64 columns x G heads x 128/G tokens.
+// q [Tq, Hq, D] bf16 as a 3-D tensor (D, Hq, Tq); box = 64 columns x G heads x chunk_tok(G) tokens.
 static int encode_q_tmap(CUtensorMap* map, const void* q, int total_q_tokens, int num_q_heads, int group,
                          int head_dim, EncodeTiledFn fn) {
   const cuuint64_t d = static_cast<cuuint64_t>(head_dim);
   const cuuint64_t dims[3] = {d, static_cast<cuuint64_t>(num_q_heads), static_cast<cuuint64_t>(total_q_tokens)};
   const cuuint64_t strides[2] = {d * 2, static_cast<cuuint64_t>(num_q_heads) * d * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(CH_M / group)};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(chunk_tok(group))};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -833,10 +846,11 @@ static int launch_chunk_t(const ChunkParams& p, const CUtensorMap& tq, const CUt
   return check_launch(cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p), "chunk_kernel launch");
 }
 
-// Items of a batch: pairs of M-tiles (256 / G tokens) of each multi-row
-// sequence, times the KV heads; at most (rows * G / 256 + sequences) * Hkv.
+// Items of a batch: pairs of M-tiles (2 chunk_tok(G) tokens) of each multi-row
+// sequence, times the KV heads; at most (rows / (2 chunk_tok(G)) + sequences)
+// * Hkv.
 static size_t chunk_max_items(int num_query_tokens, int num_seqs_bound, int num_kv_heads, int group) {
-  return (static_cast<size_t>(num_query_tokens) * group / (2 * CH_M) + static_cast<size_t>(num_seqs_bound)) *
+  return (static_cast<size_t>(num_query_tokens) / (2 * chunk_tok(group)) + static_cast<size_t>(num_seqs_bound)) *
          static_cast<size_t>(num_kv_heads);
 }
 
@@ -877,8 +891,12 @@ int launch_chunk(const ChunkParams& p, const void* q, const void* k_cache, const
                        : launch_chunk_t<2, 128>(p, tq, tk, tv, stream, num_sms, ctas);
     case 4: return d64 ? launch_chunk_t<4, 64>(p, tq, tk, tv, stream, num_sms, ctas)
                        : launch_chunk_t<4, 128>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 6: return d64 ? launch_chunk_t<6, 64>(p, tq, tk, tv, stream, num_sms, ctas)
+                       : launch_chunk_t<6, 128>(p, tq, tk, tv, stream, num_sms, ctas);
     case 8: return d64 ? launch_chunk_t<8, 64>(p, tq, tk, tv, stream, num_sms, ctas)
                        : launch_chunk_t<8, 128>(p, tq, tk, tv, stream, num_sms, ctas);
+    case 12: return d64 ? launch_chunk_t<12, 64>(p, tq, tk, tv, stream, num_sms, ctas)
+                        : launch_chunk_t<12, 128>(p, tq, tk, tv, stream, num_sms, ctas);
     case 16: return d64 ? launch_chunk_t<16, 64>(p, tq, tk, tv, stream, num_sms, ctas)
                         : launch_chunk_t<16, 128>(p, tq, tk, tv, stream, num_sms, ctas);
     default: return PA_ERR_UNSUPPORTED;

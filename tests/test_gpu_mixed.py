@@ -58,12 +58,13 @@ def test_planned_mixed_batch_shares_the_gpu_and_matches_the_oracle_on_every_row(
     assert torch.equal(first.view(torch.int16), ds.out.view(torch.int16))
 
 
-@pytest.mark.parametrize("d", [128, 64])
-def test_chunk_items_cut_between_ctas_merge_exactly(d):
+@pytest.mark.parametrize("d,hq,qlen", [(128, 64, 640), (64, 64, 640), (128, 48, 800)])
+def test_chunk_items_cut_between_ctas_merge_exactly(d, hq, qlen):
     # more items than CTAs: 20 pairs of M-tiles x 8 KV heads = 160 items of
-    # about 13 key tiles on the whole GPU, split into equal unit ranges, so
-    # items are cut at CTA boundaries and merged from their pieces
-    w = workloads.custom([1000], [640], 64, 8, d, 16, seed=61, poison=True)
+    # about 13 key tiles on the whole GPU (G 8: 32-token pairs; G 6: 40-token
+    # pairs), split into equal unit ranges, so items are cut at CTA
+    # boundaries and merged from their pieces
+    w = workloads.custom([1000], [qlen], hq, 8, d, 16, seed=61, poison=True)
     ds = DeviceStep(w)
     ds.append()
     ref = _ref(w)
@@ -73,7 +74,7 @@ def test_chunk_items_cut_between_ctas_merge_exactly(d):
         torch.cuda.synchronize()
         assert int(ds.status.item()) == 0
         outs.append(ds.out.clone())
-    compare(outs[0].float().cpu().numpy(), ref, f"160 items cut between CTAs, d{d}")
+    compare(outs[0].float().cpu().numpy(), ref, f"items cut between CTAs, d{d}, Hq {hq}")
     for o in outs[1:]:
         assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
 

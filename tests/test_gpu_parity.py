@@ -121,6 +121,11 @@ SMALL = [  # ctx list, qlen list, Hq, Hkv, d, bs
     ([700], [200], 4, 4, 64, 16),
     ([500, 77], [50, 1], 32, 2, 64, 16),
     ([260, 129, 1], [5, 129, 1], 8, 4, 64, 16),
+    # groups that do not divide 128 rows: G 6 and 12 (120-row M-tiles, 8 rows of padding)
+    ([900, 40], [300, 1], 24, 4, 128, 32),       # G 6, the GRPO shape's group
+    ([500, 77, 9], [161, 1, 3], 24, 4, 64, 16),  # G 6 at head_dim 64, a 3-row sequence on the chunk path
+    ([700], [90], 24, 2, 128, 16),               # G 12
+    ([333, 20], [333, 2], 12, 1, 64, 16),        # G 12 at head_dim 64, whole prompt from position 0
 ]
 
 
